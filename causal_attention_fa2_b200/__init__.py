@@ -1,0 +1,146 @@
+"""FlashAttention-2 (causal multi-head attention forward and recomputation
+backward) for NVIDIA B200, sm_100a.
+
+Every step of the computation runs in the CUDA kernels of ``libfa2.so``
+(C ABI declared in ``include/fa2.h``).  This module only marshals arguments:
+it checks tensors, allocates outputs with PyTorch, passes raw device pointers
+and the current CUDA stream to the library, and turns status codes into
+exceptions.  There is no CPU or PyTorch fallback: without the library or a
+B200 the calls raise.
+
+Semantics follow the CS336 A2 Systems handout, section 4.2.2: Algorithm 1 for
+the forward (O and the logsumexp L), Eqs. 13-19 with D = rowsum(O o dO) for
+the backward, and the causal rule of Problem flash_forward (c).
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Tuple
+
+import torch
+
+from . import _native
+from ._native import (FA2_BF16, FA2_FP32, FA2Error, clear_device_status,  # noqa: F401
+                      last_device_status, library_path, status_string)
+
+__all__ = [
+    "forward", "backward", "backward_workspace_bytes", "flash_attention",
+    "FlashAttention2Function", "last_device_status", "clear_device_status",
+    "status_string", "FA2Error", "library_path",
+]
+
+SUPPORTED_HEAD_DIMS = (16, 32, 64, 80, 128)
+_DTYPES = {torch.bfloat16: FA2_BF16, torch.float32: FA2_FP32}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected q, k, v of shape [B, H, N, d]")
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError(f"q, k, v shapes must match, got {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share one dtype")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
+    if k.device != q.device or v.device != q.device:
+        raise ValueError("q, k, v must be on one device")
+    return tuple(q.shape)
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+            scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+            lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O = softmax(scale * Q K^T (+ causal mask)) V and L = logsumexp (fp32).
+
+    q, k, v: contiguous CUDA tensors [B, H, N, d] (bf16 or fp32).
+    Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).
+    """
+    B, H, N, d = _check_qkv(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        _native.check(_native.lib().fa2_forward(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+            B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
+            _stream_handle(q.device)))
+    return out, lse
+
+
+def backward_workspace_bytes(B: int, H: int, N: int, d: int, dtype: torch.dtype) -> int:
+    return int(_native.lib().fa2_backward_workspace_bytes(B, H, N, d, _DTYPES[dtype]))
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, do: torch.Tensor, causal: bool = True,
+             scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+             dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+             dv: Optional[torch.Tensor] = None):
+    """dQ, dK, dV of sum(dO * O) via the recomputation backward.
+
+    ``o`` and ``lse`` are the forward's outputs; ``workspace`` (optional) is a
+    uint8 CUDA tensor of at least backward_workspace_bytes(...) bytes.
+    """
+    B, H, N, d = _check_qkv(q, k, v)
+    for name, t in (("o", o), ("do", do)):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
+    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = backward_workspace_bytes(B, H, N, d, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    with torch.cuda.device(q.device):
+        _native.check(_native.lib().fa2_backward(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
+            int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
+    return dq, dk, dv
+
+
+class FlashAttention2Function(torch.autograd.Function):
+    """autograd wrapper with the handout's interface: forward(ctx, Q, K, V,
+    is_causal=False) saves L, Q, K, V, O and the causal flag; backward(dO)
+    returns dQ, dK, dV (handout section 4.2.2, Problems flash_forward and
+    flash_backward)."""
+
+    @staticmethod
+    def forward(ctx, Q, K, V, is_causal=False):
+        o, lse = forward(Q, K, V, causal=is_causal)
+        ctx.save_for_backward(lse, Q, K, V, o)
+        ctx.is_causal = bool(is_causal)
+        return o
+
+    @staticmethod
+    def backward(ctx, dO):
+        lse, Q, K, V, o = ctx.saved_tensors
+        dq, dk, dv = backward(Q, K, V, o, lse, dO.contiguous(), causal=ctx.is_causal)
+        return dq, dk, dv, None
+
+
+def flash_attention(q, k, v, is_causal: bool = False):
+    """Differentiable attention: FlashAttention2Function.apply(q, k, v, is_causal)."""
+    return FlashAttention2Function.apply(q, k, v, is_causal)

@@ -1,0 +1,336 @@
+// fa2_api.cu -- the C ABI of libfa2.so (declared in include/fa2.h): argument
+// validation, tensor-map construction and kernel launches for the
+// FlashAttention-2 forward and backward passes on sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <cuda_bf16.h>
+
+#include <mutex>
+#include <type_traits>
+
+#include "../../include/fa2.h"
+#include "fa2_bwd.cuh"
+#include "fa2_fwd.cuh"
+
+namespace fa2 {
+namespace {
+
+// Per-device status word written by the kernels' pipeline watchdog.
+__device__ uint32_t g_device_status;
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+constexpr int kMaxDevices = 64;
+constexpr int kMaxN = 1 << 24;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mutex;
+EncodeTiledFn g_encode = nullptr;
+uint32_t* g_status_ptr[kMaxDevices] = {};
+int g_device_cc[kMaxDevices] = {};  // 0 = not queried yet
+
+fa2_status init_device(int* dev_out, uint32_t** status_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_device_cc[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return FA2_ERR_CUDA;
+        g_device_cc[dev] = major * 10 + minor;
+    }
+    if (g_device_cc[dev] != 100) return FA2_ERR_UNSUPPORTED_DEVICE;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return FA2_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return FA2_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<uint32_t*>(p);
+    }
+    *dev_out = dev;
+    *status_out = g_status_ptr[dev];
+    return FA2_OK;
+}
+
+bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 80 || d == 128; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2_dtype dtype) {
+    if (dtype != FA2_BF16 && dtype != FA2_FP32) return FA2_ERR_UNSUPPORTED_DTYPE;
+    if (B < 1 || H < 1 || N < 1 || N > kMaxN) return FA2_ERR_BAD_SHAPE;
+    if (static_cast<long long>(B) * H > (1ll << 31) - 1) return FA2_ERR_BAD_SHAPE;
+    const long long tiles = (N + kTileRows - 1) / kTileRows;
+    if (tiles * B * H > (1ll << 31) - 1) return FA2_ERR_BAD_SHAPE;
+    if (!head_dim_supported(d)) return FA2_ERR_UNSUPPORTED_HEAD_DIM;
+    if (causal != 0 && causal != 1) return FA2_ERR_BAD_ARGUMENT;
+    if (!std::isfinite(scale)) return FA2_ERR_BAD_ARGUMENT;
+    return FA2_OK;
+}
+
+// 3-D view [BH][N][d] of a contiguous [B,H,N,d] tensor, loaded/stored in boxes
+// of box_cols x 128 rows x 1 head.
+fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int N, int BH,
+                    int box_cols, int row_bytes, bool mn_major_f32) {
+    const int es = dtype == FA2_BF16 ? 2 : 4;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es,
+                             static_cast<cuuint64_t>(d) * es * static_cast<cuuint64_t>(N)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kTileRows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMapSwizzle sw = mn_major_f32       ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                            : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                            : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                                               : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUresult r = g_encode(m,
+                          dtype == FA2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          3, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+}
+
+template <int ES, int D>
+fa2_status make_maps_kmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int N, int BH) {
+    using G = TileGeom<ES, D>;
+    return make_map(m, ptr, dtype, D, N, BH, G::kBoxK, G::kRowBK, false);
+}
+
+template <int ES, int D>
+fa2_status make_maps_mnmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int N, int BH) {
+    using G = TileGeom<ES, D>;
+    return make_map(m, ptr, dtype, D, N, BH, G::kBoxMN, G::kRowBMN, G::kF32);
+}
+
+template <class Kernel>
+fa2_status set_smem(Kernel k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+                   cudaSuccess
+               ? FA2_OK
+               : FA2_ERR_CUDA;
+}
+
+template <int ES, int D>
+fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int N, int causal, float scale, fa2_dtype dtype,
+                          cudaStream_t stream, uint32_t* status) {
+    using Cfg = FwdCfg<ES, D>;
+    const int BH = B * H;
+    CUtensorMap mq, mk, mv, mo;
+    fa2_status st;
+    if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_mnmajor<ES, D>(&mv, v, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mo, o, dtype, N, BH)) != FA2_OK) return st;
+    FwdParams p;
+    p.lse = lse;
+    p.status = status;
+    p.N = N;
+    p.BH = BH;
+    p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.causal = causal;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.timeout_ns = kDefaultTimeoutNs;
+    auto kern = fa2_fwd_kernel<ES, D>;
+    if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
+    const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+}
+
+template <int ES>
+fa2_status dispatch_forward(int d, const void* q, const void* k, const void* v, void* o,
+                            float* lse, int B, int H, int N, int causal, float scale,
+                            fa2_dtype dtype, cudaStream_t stream, uint32_t* status) {
+    switch (d) {
+        case 16: return launch_forward<ES, 16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 32: return launch_forward<ES, 32>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 64: return launch_forward<ES, 64>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 80: return launch_forward<ES, 80>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 128: return launch_forward<ES, 128>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        default: return FA2_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+}
+
+template <int ES, int D>
+fa2_status launch_backward_t(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int H, int N, int causal, float scale, fa2_dtype dtype,
+                             uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
+                             uint32_t* status, unsigned long long timeout_ns) {
+    using T = typename std::conditional<ES == 2, __nv_bfloat16, float>::type;
+    using Cfg = BwdCfg<ES, D>;
+    const int BH = B * H;
+    float* l2 = reinterpret_cast<float*>(ws_base + ws.l2_off);
+    float* dvec = reinterpret_cast<float*>(ws_base + ws.d_off);
+    float* dq_acc = reinterpret_cast<float*>(ws_base + ws.dq_off);
+    fa2_status st;
+    // 1. D, log2-scaled L, zeroed dQ accumulator.
+    const long long rows = static_cast<long long>(BH) * ws.n_pad;
+    fa2_bwd_pre_kernel<T, D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, dq_acc, N, ws.n_pad,
+        rows);
+    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+    // 2. Main key/value-tile-outer pass.
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+    if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mv, v, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdo, dout, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdk, dk, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdv, dv, dtype, N, BH)) != FA2_OK) return st;
+    BwdParams p;
+    p.l2 = l2;
+    p.dvec = dvec;
+    p.dq_acc = dq_acc;
+    p.status = status;
+    p.N = N;
+    p.BH = BH;
+    p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.n_pad = ws.n_pad;
+    p.causal = causal;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.timeout_ns = timeout_ns;
+    auto kern = fa2_bwd_kernel<ES, D>;
+    if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
+    const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+    // 3. dQ = scale * accumulator.
+    const long long n4 = static_cast<long long>(BH) * N * D / 4;
+    fa2_bwd_dq_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<T*>(dq), scale, n4);
+    return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+}
+
+fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                           int H, int N, int d, int causal, float scale, fa2_dtype dtype,
+                           uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
+                           uint32_t* status, unsigned long long timeout_ns) {
+    if (dtype != FA2_BF16) return FA2_ERR_UNSUPPORTED_DTYPE;
+#define FA2_BWD_CASE(DD)                                                                      \
+    case DD:                                                                                  \
+        return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal,   \
+                                        scale, dtype, ws_base, ws, stream, status, timeout_ns);
+    switch (d) {
+        FA2_BWD_CASE(16)
+        FA2_BWD_CASE(32)
+        FA2_BWD_CASE(64)
+        FA2_BWD_CASE(80)
+        FA2_BWD_CASE(128)
+        default: return FA2_ERR_UNSUPPORTED_HEAD_DIM;
+    }
+#undef FA2_BWD_CASE
+}
+
+}  // namespace
+}  // namespace fa2
+
+using namespace fa2;
+
+extern "C" {
+
+fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int H, int N, int d, int causal, float scale, fa2_dtype dtype,
+                       fa2_stream_t stream) {
+    fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
+    if (st != FA2_OK) return st;
+    if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_PTR;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return FA2_ERR_MISALIGNED;
+    int dev;
+    uint32_t* status;
+    if ((st = init_device(&dev, &status)) != FA2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == FA2_BF16)
+        return dispatch_forward<2>(d, q, k, v, o, lse, B, H, N, causal, scale, dtype, s, status);
+    return dispatch_forward<4>(d, q, k, v, o, lse, B, H, N, causal, scale, dtype, s, status);
+}
+
+size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype) {
+    if (check_common(B, H, N, d, 0, 1.f, dtype) != FA2_OK) return 0;
+    return bwd_workspace_layout(B * H, N, d).total;
+}
+
+fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                        int H, int N, int d, int causal, float scale, fa2_dtype dtype,
+                        void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+    fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
+    if (st != FA2_OK) return st;
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return FA2_ERR_NULL_PTR;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4) || !aligned(workspace, 256))
+        return FA2_ERR_MISALIGNED;
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d);
+    if (workspace_bytes < ws.total) return FA2_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    uint32_t* status;
+    if ((st = init_device(&dev, &status)) != FA2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype,
+                           static_cast<uint8_t*>(workspace), ws, s, status, kDefaultTimeoutNs);
+}
+
+fa2_status fa2_last_device_status(void) {
+    int dev;
+    uint32_t* status;
+    fa2_status st = init_device(&dev, &status);
+    if (st != FA2_OK) return st;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FA2_ERR_CUDA;
+    return static_cast<fa2_status>(v);
+}
+
+fa2_status fa2_clear_device_status(void) {
+    int dev;
+    uint32_t* status;
+    fa2_status st = init_device(&dev, &status);
+    if (st != FA2_OK) return st;
+    const uint32_t zero = 0;
+    if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return FA2_ERR_CUDA;
+    return FA2_OK;
+}
+
+const char* fa2_status_string(fa2_status status) {
+    switch (status) {
+        case FA2_OK: return "FA2_OK";
+        case FA2_ERR_NULL_PTR: return "FA2_ERR_NULL_PTR: a required pointer is NULL";
+        case FA2_ERR_BAD_SHAPE: return "FA2_ERR_BAD_SHAPE: B, H or N out of range";
+        case FA2_ERR_UNSUPPORTED_HEAD_DIM: return "FA2_ERR_UNSUPPORTED_HEAD_DIM: d must be 16, 32, 64, 80 or 128";
+        case FA2_ERR_UNSUPPORTED_DTYPE: return "FA2_ERR_UNSUPPORTED_DTYPE: dtype must be FA2_BF16 or FA2_FP32";
+        case FA2_ERR_MISALIGNED: return "FA2_ERR_MISALIGNED: tensors need 16-byte, lse 4-byte, workspace 256-byte alignment";
+        case FA2_ERR_WORKSPACE_TOO_SMALL: return "FA2_ERR_WORKSPACE_TOO_SMALL: see fa2_backward_workspace_bytes";
+        case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call or kernel launch failed";
+        case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel pipeline wait expired";
+        case FA2_ERR_UNSUPPORTED_DEVICE: return "FA2_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
+        case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1 and scale finite";
+    }
+    return "unknown fa2_status";
+}
+
+}  // extern "C"

@@ -1,0 +1,369 @@
+// fa2_fwd.cuh -- FlashAttention-2 forward kernel for sm_100a.
+//
+// Computes, for one 128-row query tile Q_i of one head (CS336 A2 Systems
+// handout section 4.2.2, Algorithm 1):
+//   for each key/value tile j:   S = scale * Q_i K_j^T            (step 9)
+//                                m_new = max(m, rowmax S)         (step 10)
+//                                P~ = exp(S - m_new)              (step 11)
+//                                l = exp(m - m_new) l + rowsum P~ (step 12)
+//                                O = diag(exp(m - m_new)) O + P~ V_j (step 13)
+//   O = O / l,  L = m + log l                                      (steps 15-18)
+// with the causal rule of Problem flash_forward (c): key tiles entirely above
+// the diagonal are skipped, and on the diagonal tile scores of keys after the
+// query are excluded (set to -inf, which is what the handout's -1e6 offset
+// amounts to once exponentiated).
+//
+// B200 mapping (one CTA per (query tile, head); 6 warps, warp-specialised):
+//   warp 0    TMA producer: Q_i once, then K_j and V_j into two rings of
+//             shared-memory stages guarded by full/empty mbarriers.
+//   warp 1    MMA issuer (one thread): S_j = Q_i K_j^T into one of two
+//             tensor-memory (TMEM) score buffers; O += P_j V_j with P_j read
+//             from TMEM and O accumulated in TMEM (fp32).  Completion is
+//             signalled with tcgen05.commit on mbarriers.
+//   warps 2-5 softmax warpgroup: thread t owns query row t (TMEM lane t).  It
+//             loads its score row from TMEM, applies the mask, updates the
+//             running max / sum, writes P (bf16, or fp32 for the TF32 path)
+//             back into the score buffer for the next MMA, and rescales its O
+//             row in TMEM when the running max grows.  After the last tile it
+//             normalises O, stages it in shared memory for a TMA store and
+//             writes L.
+// Scores are kept in log2 units (scale * log2(e) folded into one multiply)
+// so every exponential is a single ex2.  The running max used as the
+// exponent's reference is only raised when the row max grows by more than
+// 2^8, which keeps P <= 256 and skips most O rescales; the final O / l and L
+// are exact whatever reference was used.
+#pragma once
+
+#include <cstdint>
+
+#include "fa2_traits.cuh"
+
+namespace fa2 {
+
+struct FwdParams {
+    float* lse;            // [BH][N] natural-log logsumexp
+    uint32_t* status;      // device status word
+    int N;                 // sequence length (queries = keys)
+    int BH;                // batch * heads
+    int n_tiles;           // ceil(N / 128)
+    int causal;
+    float scale_log2;      // scale * log2(e)
+    unsigned long long timeout_ns;
+};
+
+template <int ES, int D>
+struct FwdCfg {
+    using G = TileGeom<ES, D>;
+    static constexpr int kThreads = 192;
+    static constexpr int kBudget = 227 * 1024 - 2048;
+    static constexpr int kFree = kBudget - G::kTileBytesK;
+    // Ring depths for K and V (at most 4 each), as many as fit.
+    static constexpr int kKV = G::kTileBytesK + G::kTileBytesMN;
+    static constexpr int kPairs = kFree / kKV;
+    static constexpr int kKSt0 = kPairs > 4 ? 4 : kPairs;
+    static constexpr int kKSt = (kKSt0 < 4 && kFree - kKSt0 * kKV >= G::kTileBytesK) ? kKSt0 + 1 : kKSt0;
+    static constexpr int kVSt = kKSt0;
+    static_assert(kVSt >= 1, "shared memory too small for one K/V stage");
+    static constexpr int kSmemBytes =
+        1024 + G::kTileBytesK * (1 + kKSt) + G::kTileBytesMN * kVSt;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kOCol = 256;
+};
+
+template <int ES, int D>
+__global__ void __launch_bounds__(192, 1)
+fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const FwdParams p) {
+    using Cfg = FwdCfg<ES, D>;
+    using G = typename Cfg::G;
+    constexpr int KST = Cfg::kKSt;
+    constexpr int VST = Cfg::kVSt;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar_q_full;
+    __shared__ uint64_t bar_k_full[KST], bar_k_empty[KST];
+    __shared__ uint64_t bar_v_full[VST], bar_v_empty[VST];
+    __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done, bar_drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile uint32_t abort_flag;
+
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + G::kTileBytesK;
+    uint8_t* sV = sK + KST * G::kTileBytesK;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: causal query tiles are issued longest first.
+    const int item = blockIdx.x;
+    const int tile_rank = item / p.BH;
+    const int bh = item - tile_rank * p.BH;
+    const int q_tile = p.causal ? (p.n_tiles - 1 - tile_rank) : tile_rank;
+    const int n_kv = p.causal ? (q_tile + 1) : p.n_tiles;
+    const int q_row0 = q_tile * kTileRows;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        ptx::mbar_init(&bar_q_full, 1);
+        for (int s = 0; s < KST; ++s) { ptx::mbar_init(&bar_k_full[s], 1); ptx::mbar_init(&bar_k_empty[s], 1); }
+        for (int s = 0; s < VST; ++s) { ptx::mbar_init(&bar_v_full[s], 1); ptx::mbar_init(&bar_v_empty[s], 1); }
+        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bar_s_full[b], 1); ptx::mbar_init(&bar_p_full[b], 4); }
+        ptx::mbar_init(&bar_o_done, 1);
+        ptx::mbar_init(&bar_drain, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_q);
+            ptx::prefetch_tmap(&tm_k);
+            ptx::prefetch_tmap(&tm_v);
+            ptx::mbar_arrive_expect_tx(&bar_q_full, G::kTileBytesK);
+            for (int b = 0; b < G::kNBoxK; ++b)
+                ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full, b * G::kBoxK, q_row0, bh);
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int ks = j % KST;
+                if (j >= KST && !ptx::mbar_wait(&bar_k_empty[ks], ((j / KST) & 1) ^ 1, &abort_flag, tmo)) break;
+                uint8_t* dk = sK + ks * G::kTileBytesK;
+                ptx::mbar_arrive_expect_tx(&bar_k_full[ks], G::kTileBytesK);
+                for (int b = 0; b < G::kNBoxK; ++b)
+                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, j * kTileRows, bh);
+                k_issued = j + 1;
+                const int vs = j % VST;
+                if (j >= VST && !ptx::mbar_wait(&bar_v_empty[vs], ((j / VST) & 1) ^ 1, &abort_flag, tmo)) break;
+                uint8_t* dv = sV + vs * G::kTileBytesMN;
+                ptx::mbar_arrive_expect_tx(&bar_v_full[vs], G::kTileBytesMN);
+                for (int b = 0; b < G::kNBoxMN; ++b)
+                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, j * kTileRows, bh);
+                v_issued = j + 1;
+            }
+            if (abort_flag) {
+                // Let copies already in flight land before the CTA exits.
+                constexpr uint64_t kDrainNs = 20000000ull;
+                ptx::mbar_wait_drain(&bar_q_full, 0, kDrainNs);
+                for (int t = k_issued - 1; t >= 0 && t >= k_issued - KST; --t)
+                    ptx::mbar_wait_drain(&bar_k_full[t % KST], (t / KST) & 1, kDrainNs);
+                for (int t = v_issued - 1; t >= 0 && t >= v_issued - VST; --t)
+                    ptx::mbar_wait_drain(&bar_v_full[t % VST], (t / VST) & 1, kDrainNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
+            constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
+            const uint32_t q_addr = ptx::smem_addr(sQ);
+            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            auto issue_pv = [&](int jj) -> bool {
+                if (!ptx::mbar_wait(&bar_p_full[jj & 1], (jj >> 1) & 1, &abort_flag, tmo)) return false;
+                const int vs = jj % VST;
+                if (!ptx::mbar_wait(&bar_v_full[vs], (jj / VST) & 1, &abort_flag, tmo)) return false;
+                ptx::tc_fence_after();
+                const uint32_t v_addr = ptx::smem_addr(sV + vs * G::kTileBytesMN);
+                const uint32_t p_tmem = tmem + (jj & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsRows; ++kk) {
+                    const uint64_t bdesc = desc_mnmajor<G>(v_addr, kk);
+                    if constexpr (G::kF32)
+                        ptx::mma_tf32_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    else
+                        ptx::mma_f16_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                }
+                ptx::mma_commit(&bar_o_done);
+                ptx::mma_commit(&bar_v_empty[vs]);
+                return true;
+            };
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int ks = j % KST;
+                if (!ptx::mbar_wait(&bar_k_full[ks], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t k_addr = ptx::smem_addr(sK + ks * G::kTileBytesK);
+                const uint32_t s_tmem = tmem + (j & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk) {
+                    const uint64_t adesc = desc_kmajor<G>(q_addr, kk);
+                    const uint64_t bdesc = desc_kmajor<G>(k_addr, kk);
+                    if constexpr (G::kF32)
+                        ptx::mma_tf32_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(&bar_s_full[j & 1]);
+                ptx::mma_commit(&bar_k_empty[ks]);
+                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok) ok = issue_pv(n_kv - 1);
+            if (!ok) {
+                // Drain: every MMA issued so far must finish before TMEM is freed.
+                ptx::mma_commit(&bar_drain);
+                ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax warpgroup
+        const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+        const int r = quarter * 32 + lane;      // query row inside the tile
+        const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
+        const uint32_t o_tmem = lane_base + Cfg::kOCol;
+        const float sl2 = p.scale_log2;
+        float m_ref = -INFINITY;                // reference max (log2 units)
+        float l = 0.f;                          // running sum of 2^(t - m_ref)
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            if (!ptx::mbar_wait(&bar_s_full[j & 1], (j >> 1) & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+            const uint32_t s_tmem = lane_base + (j & 1) * 128;
+            float s[128];
+            {
+                uint32_t u[32];
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    ptx::tmem_ld32(s_tmem + c0, u);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(u[c]);
+                }
+            }
+            // Mask: causal diagonal tile (key > query), or keys past N.
+            const bool diag = p.causal && (j == q_tile);
+            const int kv_valid = p.N - j * kTileRows;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                float t = s[c] * sl2;
+                if ((diag && c > r) || c >= kv_valid) t = -INFINITY;
+                s[c] = t;
+                mx = fmaxf(mx, t);
+            }
+            const float m_new = fmaxf(m_ref, mx);
+            float alpha = 1.f;
+            const bool raise = (m_new - m_ref) > 8.f;   // true on the first tile
+            if (raise) {
+                alpha = ptx::ex2_approx(m_ref - m_new);
+                m_ref = m_new;
+            }
+            if (j > 0) {
+                // PV_{j-1} must be done before O is touched.
+                if (!ptx::mbar_wait(&bar_o_done, (j - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+                    for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+                        uint32_t u[16];
+                        ptx::tmem_ld16(o_tmem + c0, u);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+                        ptx::tmem_st16(o_tmem + c0, u);
+                    }
+                }
+            }
+            l *= alpha;
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) {
+                const float pc = ptx::ex2_approx(s[c] - m_ref);
+                s[c] = pc;
+                rs += pc;
+            }
+            l += rs;
+            // P back into the score buffer (A operand of the PV MMA).
+            if constexpr (G::kF32) {
+#pragma unroll
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(s[c0 + c]);
+                    ptx::tmem_st32(s_tmem + c0, u);
+                }
+            } else {
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 32) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) u[c] = ptx::pack_bf16x2(s[2 * (c0 + c)], s[2 * (c0 + c) + 1]);
+                    ptx::tmem_st32(s_tmem + c0, u);
+                }
+            }
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_p_full[j & 1]);
+        }
+        // ---------------- epilogue: O / l -> shared memory -> TMA store; L.
+        if (ok) ok = ptx::mbar_wait(&bar_o_done, (n_kv - 1) & 1, &abort_flag, tmo);
+        if (ok) {
+            ptx::tc_fence_after();
+            const float inv_l = 1.f / l;
+#pragma unroll
+            for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+                uint32_t u[16];
+                ptx::tmem_ld16(o_tmem + c0, u);
+                ptx::tmem_wait_ld();
+                if constexpr (G::kF32) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int col = c0 + 4 * q4;
+                        if (col < D) {
+                            uint4 w;
+                            w.x = __float_as_uint(__uint_as_float(u[4 * q4 + 0]) * inv_l);
+                            w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * inv_l);
+                            w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * inv_l);
+                            w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * inv_l);
+                            *reinterpret_cast<uint4*>(sQ + kmajor_chunk_offset<G>(r, col)) = w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int h8 = 0; h8 < 2; ++h8) {
+                        const int col = c0 + 8 * h8;
+                        if (col < D) {
+                            uint4 w;
+                            const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
+                            w.x = ptx::pack_bf16x2(f[0] * inv_l, f[1] * inv_l);
+                            w.y = ptx::pack_bf16x2(f[2] * inv_l, f[3] * inv_l);
+                            w.z = ptx::pack_bf16x2(f[4] * inv_l, f[5] * inv_l);
+                            w.w = ptx::pack_bf16x2(f[6] * inv_l, f[7] * inv_l);
+                            *reinterpret_cast<uint4*>(sQ + kmajor_chunk_offset<G>(r, col)) = w;
+                        }
+                    }
+                }
+            }
+            const int q_row = q_row0 + r;
+            if (q_row < p.N)
+                p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+            ptx::fence_async_smem();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && threadIdx.x == 64) {
+            for (int b = 0; b < G::kNBoxK; ++b)
+                ptx::tma_store_3d(&tm_o, sQ + b * kTileRows * G::kRowBK, b * G::kBoxK, q_row0, bh);
+            ptx::tma_store_commit();
+            ptx::tma_store_wait_all();
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+    if (threadIdx.x == 0 && abort_flag) atomicCAS(p.status, 0u, kDevStatusTimeout);
+}
+
+}  // namespace fa2

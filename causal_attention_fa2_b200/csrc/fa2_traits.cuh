@@ -1,0 +1,90 @@
+// fa2_traits.cuh -- compile-time tile geometry shared by the forward and
+// backward kernels, and the shared-memory tile layouts the tensor memory
+// accelerator (TMA) writes and the tcgen05 MMA reads.
+//
+// A "tile" is 128 consecutive rows (queries or keys) of one head, all d
+// columns.  The handout does not tile the head dimension (CS336 A2 Systems
+// handout section 4.2.2: "we will not tile along the hidden dimension d"), and
+// neither do we: a tile is staged in shared memory as NBOX boxes of BOX
+// columns each (one TMA copy per box), BOX chosen so that one box row is the
+// width of a hardware swizzle pattern.
+//
+// Two staging geometries exist for the same tensor:
+//   K-major  - the operand's contraction dimension runs along d (Q and K in
+//              S = Q K^T).  Rows are ROWB = BOX*ES bytes, swizzled with the
+//              32/64/128-byte pattern of that width.
+//   MN-major - the contraction runs along the 128 rows and d is the output
+//              dimension (V in O += P V).  16-bit types reuse the K-major
+//              staging.  32-bit (TF32) operands must use 128-byte rows with
+//              32-byte swizzle atoms, whose 8-row groups are 512 bytes apart.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fa2 {
+
+constexpr int kTileRows = 128;  // B_q = B_k = 128 rows per tile
+
+// Device status codes the kernels record (same values as fa2_status).
+constexpr uint32_t kDevStatusTimeout = 8;
+
+template <int ES, int D>
+struct TileGeom {
+    static constexpr int kES = ES;
+    static constexpr int kD = D;
+    static constexpr bool kF32 = (ES == 4);
+    // K-major staging.
+    static constexpr int kBoxK = (D * ES >= 128) ? (128 / ES) : D;
+    static constexpr int kRowBK = kBoxK * ES;
+    static constexpr int kNBoxK = (D + kBoxK - 1) / kBoxK;
+    static constexpr int kTileBytesK = kNBoxK * kTileRows * kRowBK;
+    static constexpr uint32_t kLayoutK = ptx::layout_for_row_bytes(kRowBK);
+    // MN-major staging.
+    static constexpr int kBoxMN = kF32 ? 32 : kBoxK;
+    static constexpr int kRowBMN = kBoxMN * ES;
+    static constexpr int kNBoxMN = (D + kBoxMN - 1) / kBoxMN;
+    static constexpr int kTileBytesMN = kNBoxMN * kTileRows * kRowBMN;
+    static constexpr uint32_t kLayoutMN = kF32 ? 1u : kLayoutK;
+    static constexpr uint32_t kSboMN = kF32 ? 512u : 8u * kRowBMN;
+    // MMA shape facts.
+    static constexpr int kKStep = 32 / ES;                        // K per MMA instruction
+    static constexpr int kStepsD = (D + kKStep - 1) / kKStep;    // MMAs to contract over d
+    static constexpr int kStepsRows = kTileRows / kKStep;        // MMAs to contract over 128 rows
+    static constexpr int kNOut = (D + 15) / 16 * 16;              // MMA N when d is the output dim
+    static constexpr uint32_t kFmt = kF32 ? ptx::kFmtTF32 : ptx::kFmtBF16;
+    static constexpr int kPCols = kF32 ? 128 : 64;                // TMEM columns of a 128-wide P row
+};
+
+// Descriptor of the k-th contraction step of a K-major staged tile whose
+// boxes each hold `rows` rows.
+template <class G>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_addr, int k, int rows = kTileRows) {
+    const int off = k * 32;  // 32 bytes of K per MMA instruction
+    const uint32_t a = tile_addr + (off / G::kRowBK) * rows * G::kRowBK + (off % G::kRowBK);
+    return ptx::smem_desc(a, 16, 8 * G::kRowBK, G::kLayoutK);
+}
+
+// Descriptor of the k-th contraction step (k-th group of kKStep rows) of an
+// MN-major staged tile whose boxes each hold `rows` rows.
+template <class G>
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_addr, int k, int rows = kTileRows) {
+    const uint32_t a = tile_addr + k * G::kKStep * G::kRowBMN;
+    return ptx::smem_desc(a, rows * G::kRowBMN, G::kSboMN, G::kLayoutMN);
+}
+
+// Byte offset, inside a K-major staged tile, of the 16-byte chunk holding
+// columns [col, col + 16/ES) of `row` (col a multiple of 16/ES).  Applies the
+// swizzle the TMA uses for rows of kRowBK bytes (16-byte chunk index XOR the
+// row's position inside the 1024/512/256-byte swizzle period).
+template <class G>
+__device__ __forceinline__ uint32_t kmajor_chunk_offset(int row, int col) {
+    const int box = col / G::kBoxK;
+    const int chunk = (col % G::kBoxK) * G::kES / 16;
+    constexpr int kChunks = G::kRowBK / 16;
+    const int sw = ((row * G::kRowBK) >> 7) & (kChunks - 1);
+    return box * kTileRows * G::kRowBK + row * G::kRowBK + ((chunk ^ sw) * 16);
+}
+
+}  // namespace fa2

@@ -1,0 +1,133 @@
+/*
+ * fa2.h -- C ABI of libfa2.so: FlashAttention-2 style (causal) multi-head
+ * attention forward and recomputation backward for NVIDIA B200 (sm_100a).
+ *
+ * The operation (CS336 A2 Systems handout, section 4.2.2):
+ *   forward   S = scale * Q K^T                       (Eq. 4; scale = 1/sqrt(d)
+ *                                                      in the handout)
+ *             causal: key j is visible to query i iff j <= i
+ *                                                     (Problem flash_forward (c))
+ *             P = softmax_row(S), O = P V             (Eqs. 5-6)
+ *             L_i = log sum_j exp(S_ij)               (Eq. 12, natural log)
+ *             computed tile by tile with the online softmax of Algorithm 1.
+ *   backward  D_i = rowsum(O o dO)_i                  ("backward pass with
+ *                                                      recomputation")
+ *             P_ij = exp(S_ij - L_i), dV = P^T dO, dP = dO V^T,
+ *             dS_ij = P_ij (dP_ij - D_i), dQ = scale dS K, dK = scale dS^T Q
+ *                                                     (Eqs. 13-19)
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are dense, contiguous, row-major [B, H, N, d] arrays in device
+ *     memory (q, k, v, o, dout, dq, dk, dv), in the element type `dtype`.
+ *     lse is a dense [B, H, N] float32 device array (natural log).
+ *   - Supported: B >= 1, H >= 1, 1 <= N <= 2^24, d in {16, 32, 64, 80, 128}.
+ *     N need not be a multiple of any tile size.
+ *   - Tensor pointers must be 16-byte aligned (they are read and written by
+ *     the tensor memory accelerator); lse must be 4-byte aligned; the
+ *     backward workspace must be 256-byte aligned.
+ *   - The caller owns every buffer.  The library never allocates or frees
+ *     device memory and keeps no pointer after a call returns.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Calls are asynchronous and never synchronise the host.
+ *   - Arguments are validated on the host before anything is enqueued; on a
+ *     validation error nothing is launched and the outputs are untouched.
+ *   - A device-side pipeline watchdog bounds every wait inside the kernels.
+ *     If one expires, the kernel stops early, leaves its outputs undefined
+ *     and records FA2_ERR_DEVICE_TIMEOUT in a per-device status word that
+ *     fa2_last_device_status() reads once the caller has synchronised.
+ *   - Thread safety: entry points may be called concurrently from several
+ *     host threads; the only shared host state is a mutex-guarded cache of
+ *     per-device kernel attributes.
+ */
+#ifndef FA2_H_
+#define FA2_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of q, k, v, o, dout, dq, dk, dv.  Accumulation is always fp32.
+ * FA2_FP32 inputs are consumed by the tensor cores as TF32. */
+typedef enum {
+    FA2_BF16 = 0,
+    FA2_FP32 = 1
+} fa2_dtype;
+
+typedef enum {
+    FA2_OK = 0,
+    FA2_ERR_NULL_PTR = 1,             /* a required pointer is NULL                */
+    FA2_ERR_BAD_SHAPE = 2,            /* B, H or N out of range                    */
+    FA2_ERR_UNSUPPORTED_HEAD_DIM = 3, /* d not in {16, 32, 64, 80, 128}            */
+    FA2_ERR_UNSUPPORTED_DTYPE = 4,    /* dtype not a fa2_dtype value               */
+    FA2_ERR_MISALIGNED = 5,           /* a pointer breaks the alignment rules      */
+    FA2_ERR_WORKSPACE_TOO_SMALL = 6,  /* workspace_bytes < fa2_backward_workspace_bytes */
+    FA2_ERR_CUDA = 7,                 /* a CUDA runtime/driver call or launch failed */
+    FA2_ERR_DEVICE_TIMEOUT = 8,       /* a kernel's pipeline watchdog expired      */
+    FA2_ERR_UNSUPPORTED_DEVICE = 9,   /* the current device is not sm_100          */
+    FA2_ERR_BAD_ARGUMENT = 10         /* scale not finite, causal not 0/1, ...     */
+} fa2_status;
+
+/* Opaque CUDA stream handle; identical to cudaStream_t / CUstream. */
+typedef struct CUstream_st* fa2_stream_t;
+
+/*
+ * Forward pass (handout section 4.2.2, Algorithm 1 with the causal rule of
+ * Problem flash_forward (c)).
+ *   q, k, v  in : [B, H, N, d] `dtype`
+ *   o        out: [B, H, N, d] `dtype`, O = softmax(scale Q K^T (+mask)) V,
+ *                 rounded once from fp32
+ *   lse      out: [B, H, N] float32, L_i = log sum_j exp(S_ij)
+ *   causal   1 = causal mask, 0 = full attention
+ *   scale    finite multiplier of Q K^T (1/sqrt(d) in the handout)
+ * Returns FA2_OK once the work is enqueued, or a validation / launch error.
+ */
+fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int N, int d, int causal, float scale,
+                       fa2_dtype dtype, fa2_stream_t stream);
+
+/*
+ * Bytes of device workspace fa2_backward needs for these sizes (fp32 D and
+ * log2-scaled L vectors plus an fp32 dQ accumulator).  Returns 0 for
+ * arguments fa2_backward would reject.
+ */
+size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype);
+
+/*
+ * Backward pass with recomputation (handout section 4.2.2, Eqs. 13-19;
+ * D = rowsum(O o dO)), key/value-tile outer loop, dQ accumulated in fp32.
+ *   q, k, v, o, dout  in : [B, H, N, d] `dtype` (o as produced by fa2_forward)
+ *   lse               in : [B, H, N] float32 from fa2_forward
+ *   dq, dk, dv        out: [B, H, N, d] `dtype`
+ *   workspace         scratch of at least fa2_backward_workspace_bytes bytes,
+ *                     256-byte aligned, owned by the caller; its contents on
+ *                     entry do not matter and on return are unspecified
+ * The result of dQ depends on the order of fp32 additions across thread
+ * blocks, so it may differ in the last bits from run to run; O, L, dK and dV
+ * are deterministic.
+ */
+fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        int B, int H, int N, int d, int causal, float scale, fa2_dtype dtype,
+                        void* workspace, size_t workspace_bytes, fa2_stream_t stream);
+
+/*
+ * Status recorded by the kernels on the current device since the last call
+ * of fa2_clear_device_status (FA2_OK or FA2_ERR_DEVICE_TIMEOUT).  Call it
+ * after synchronising the streams the kernels ran on.  Returns FA2_ERR_CUDA
+ * if the status word cannot be read.
+ */
+fa2_status fa2_last_device_status(void);
+
+/* Reset the current device's status word to FA2_OK (synchronous). */
+fa2_status fa2_clear_device_status(void);
+
+/* Static, human-readable name of a status code. */
+const char* fa2_status_string(fa2_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA2_H_ */

@@ -1,0 +1,115 @@
+"""Host-only checks of the C ABI: libfa2.so builds for sm_100a, loads without a
+GPU, exports every function include/fa2.h declares, and rejects bad
+arguments with the documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa2.h")
+
+
+@pytest.fixture(scope="module")
+def fa2lib():
+    from causal_attention_fa2_b200 import build, _native
+    build.build()
+    return _native.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa2_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(fa2lib):
+    from causal_attention_fa2_b200 import _native
+    declared = header_functions()
+    assert declared, "no declarations parsed from fa2.h"
+    assert set(declared) == set(_native.SIGNATURES), "binding and header disagree"
+    for name in declared:
+        assert hasattr(fa2lib, name), f"libfa2.so does not export {name}"
+
+
+def test_status_strings(fa2lib):
+    from causal_attention_fa2_b200 import _native
+    seen = set()
+    for code in range(11):
+        s = _native.status_string(code)
+        assert s.startswith("FA2_"), s
+        seen.add(s)
+    assert len(seen) == 11
+    assert "unknown" in _native.status_string(99)
+
+
+# Fake, 256-byte aligned, never dereferenced: every call below fails host-side
+# validation before anything reaches the device.
+P = 0x10000
+BAD = 0x10002
+
+
+def fwd(lib, q=P, k=P, v=P, o=P, lse=P, B=1, H=1, N=128, d=64, causal=1, scale=0.125, dtype=0):
+    return lib.fa2_forward(q, k, v, o, lse, B, H, N, d, causal, scale, dtype, None)
+
+
+def bwd(lib, ws_bytes=1 << 30, ws=P, d=64, dtype=0, N=128, dq=P, lse=P, causal=1):
+    return lib.fa2_backward(P, P, P, P, lse, P, dq, P, P, 1, 1, N, d, causal, 0.125, dtype, ws,
+                            ws_bytes, None)
+
+
+def test_forward_validation(fa2lib):
+    L = fa2lib
+    assert fwd(L, q=None) == 1                     # FA2_ERR_NULL_PTR
+    assert fwd(L, lse=None) == 1
+    assert fwd(L, N=0) == 2                        # FA2_ERR_BAD_SHAPE
+    assert fwd(L, B=0) == 2
+    assert fwd(L, H=-1) == 2
+    assert fwd(L, N=(1 << 24) + 1) == 2
+    for d in (0, 8, 48, 96, 256):
+        assert fwd(L, d=d) == 3                    # FA2_ERR_UNSUPPORTED_HEAD_DIM
+    assert fwd(L, dtype=2) == 4                    # FA2_ERR_UNSUPPORTED_DTYPE
+    assert fwd(L, q=BAD) == 5                      # FA2_ERR_MISALIGNED
+    assert fwd(L, o=P + 8) == 5
+    assert fwd(L, lse=P + 2) == 5
+    assert fwd(L, causal=2) == 10                  # FA2_ERR_BAD_ARGUMENT
+    assert fwd(L, scale=float("inf")) == 10
+    assert fwd(L, scale=float("nan")) == 10
+
+
+def test_backward_validation(fa2lib):
+    L = fa2lib
+    need = L.fa2_backward_workspace_bytes(1, 1, 128, 64, 0)
+    assert bwd(L, ws_bytes=need - 1) == 6          # FA2_ERR_WORKSPACE_TOO_SMALL
+    assert bwd(L, ws=P + 16) == 5                  # workspace must be 256-byte aligned
+    assert bwd(L, dq=None) == 1
+    assert bwd(L, d=96) == 3
+    assert bwd(L, dtype=5) == 4
+    assert bwd(L, causal=-1) == 10
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 1, 1, 16), (2, 3, 200, 80), (1, 36, 4096, 128)])
+def test_workspace_size(fa2lib, B, H, N, d):
+    """D and log2-scaled L (fp32, padded to whole 128-row tiles) and an fp32
+    dQ accumulator, each region rounded up to 256 bytes."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    n_pad = (N + 127) // 128 * 128
+    expect = 2 * up(B * H * n_pad * 4) + up(B * H * N * d * 4)
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, 24, 0) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path only")
+def test_valid_call_without_gpu_reports_cuda_error(fa2lib):
+    assert fwd(fa2lib) in (7, 9)                   # FA2_ERR_CUDA / UNSUPPORTED_DEVICE
+    assert fa2lib.fa2_last_device_status() in (7, 9)
+
+
+def test_binding_rejects_cpu_tensors():
+    import causal_attention_fa2_b200 as fa2
+    x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa2.forward(x, x, x)
