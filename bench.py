@@ -1,0 +1,380 @@
+"""Benchmark: causal FlashAttention-2 forward + backward on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+fa2_forward (O, L) then fa2_backward (D pre-pass, key/value-tile main pass,
+dQ finalisation), on the 10B-model head shape (B=1, H=36, N=4096, d=128,
+bf16, causal) unless --workload names another.
+
+Metric: attention TFLOP/s with causal FLOPs counted (forward 4*d*P_c,
+backward 10*d*P_c, P_c = B*H*N(N+1)/2 unmasked query/key pairs).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa2|reference]
+
+For N > 1 run under torchrun: each rank runs the same workload on its own
+seeded batch (heads are independent; no collective on the data path), and the
+reported value is the total FLOPs of all ranks over the slowest rank's time.
+``--impl reference`` times the fp64 CPU oracle on the host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import fa2_inputs  # noqa: E402
+
+METRIC = "attention TFLOP/s (causal) fwd and fwd+bwd at 1 B200; % of bf16 tensor peak"
+UNIT = "TFLOP/s"
+SPEC_BF16_TFLOPS = 2250.0      # dense bf16 tensor peak of a B200 (spec sheet)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes per launch of the main backward kernel from an ncu capture of
+# the same kernel build (None until one has been taken for this build).
+BWD_MAIN_TRAFFIC_BYTES = 893907456  # profiles/fa2_bwd_kernel_d128_10b.md
+
+
+def causal_pairs(w) -> float:
+    return w.B * w.H * w.N * (w.N + 1) / 2 if w.causal else w.B * w.H * w.N * w.N
+
+
+def flops(w):
+    pc = causal_pairs(w)
+    return 4.0 * w.d * pc, 10.0 * w.d * pc
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return {k: float(m[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        target = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            target = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self.cmd = ["nvidia-smi", "-i", target, f"--query-gpu={self.FIELDS}",
+                    "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- CPU oracle
+
+def oracle_step(w, sel):
+    """fp64 oracle forward + backward on `sel` (a causal prefix of one head of
+    the workload's inputs).  Returns (seconds, algorithmic FLOPs done)."""
+    import oracle
+    rows = sel["q"].shape[0]
+    t0 = time.perf_counter()
+    oracle.forward(sel["q"], sel["k"], sel["v"], w.causal, w.scale)
+    oracle.backward(sel["q"], sel["k"], sel["v"], sel["do"], w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    pairs = rows * (rows + 1) / 2 if w.causal else rows * rows
+    return dt, 14.0 * w.d * pairs
+
+
+def cpu_baseline(w, heads: int = 8):
+    """The oracle as it stands, timed on the host cores on `heads` full heads."""
+    import oracle
+    inp = fa2_inputs.workload_inputs(w)
+    t = 0.0
+    for hh in range(min(heads, w.heads)):
+        b, h = divmod(hh, w.H)
+        sel = {n: inp[n][b, h].double().numpy() for n in ("q", "k", "v", "do")}
+        t0 = time.perf_counter()
+        oracle.forward(sel["q"], sel["k"], sel["v"], w.causal, w.scale)
+        oracle.backward(sel["q"], sel["k"], sel["v"], sel["do"], w.causal, w.scale)
+        t += time.perf_counter() - t0
+    n = min(heads, w.heads)
+    f = 14.0 * w.d * (w.N * (w.N + 1) / 2 if w.causal else w.N * w.N) * n
+    return {"value": f / t / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.heads} heads at full N={w.N}, d={w.d}, fwd+bwd, fp64",
+            "seconds": round(t, 3)}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    # Bounded per-step sample: a causal prefix of one head, sized so the whole
+    # run stays within a few minutes.
+    steps = args.steps + args.warmup
+    rows = min(w.N, max(256, int(w.N * math.sqrt(60.0 / max(steps, 1)))))
+    rows = max(128, rows // 128 * 128)
+    inp = fa2_inputs.workload_inputs(w)
+    sel = {n: inp[n][0, 0, :rows].double().numpy() for n in ("q", "k", "v", "do")}
+    del inp
+    for _ in range(args.warmup):
+        oracle_step(w, sel)
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, f = oracle_step(w, sel)
+        tot_t += dt
+        tot_f += f
+    value = tot_f / tot_t / 1e12
+    sample = f"causal prefix of {rows} rows of head 0 (of {w.heads} heads, N={w.N}), fwd+bwd, fp64"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "dtype": w.dtype,
+            "causal": w.causal, "scale": "1/sqrt(d)", "global_batch": w.B * n,
+            "parallelism": f"replicas x{n} (independent heads, no collective)",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+# --------------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fa2", choices=["fa2", "reference"])
+    ap.add_argument("--workload", default="10b-b1h36-n4096-d128")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = fa2_inputs.WORKLOADS[args.workload]
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import causal_attention_fa2_b200 as fa2
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # Inputs: each rank its own seeded batch (weak scaling).
+    inp = fa2_inputs.make_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed + rank)
+    host = {n: t.pin_memory() for n, t in inp.items()}
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    f_fwd, f_bwd = flops(w)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        fa2.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws,
+                     dq=dq, dk=dk, dv=dv, events=None if evs is None else evs[1:5])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    for e in evs:          # materialise the event handles before handing them out
+        for x in e:
+            x.record()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()                      # evict the previous step from L2
+            step(evs[i])
+        torch.cuda.synchronize()
+        barrier()
+    t_fwd = [e[0].elapsed_time(e[1]) for e in evs]          # forward kernel
+    t_bwd = [e[1].elapsed_time(e[4]) for e in evs]          # whole backward call
+    t_pre = [e[1].elapsed_time(e[2]) for e in evs]
+    t_main = [e[2].elapsed_time(e[3]) for e in evs]         # main backward kernel
+    t_fin = [e[3].elapsed_time(e[4]) for e in evs]
+    t_step = [a + b for a, b in zip(t_fwd, t_bwd)]
+    total_ms = sum(t_step)
+    fwd_ms, bwd_ms = sum(t_fwd), sum(t_bwd)
+    if dist is not None:
+        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, fwd_ms, bwd_ms = t.tolist()
+    status = fa2.last_device_status()
+    if status != 0:
+        raise SystemExit(f"device status after timing: {fa2.status_string(status)}")
+
+    # ---------------- end to end through the public API with host buffers
+    out_host = {n: torch.empty_like(t if n != "lse" else lse, device="cpu").pin_memory()
+                for n, t in (("o", q), ("lse", lse), ("dq", q), ("dk", q), ("dv", q))}
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "do"))
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    K_e2e = max(3, min(K, 50))
+
+    def e2e_step():
+        for n, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
+            dst.copy_(host[n], non_blocking=True)
+        fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        fa2.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws,
+                     dq=dq, dk=dk, dv=dv)
+        for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            out_host[n].copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    for _ in range(K_e2e):
+        e2e_step()
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    barrier()
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        value = world * (f_fwd + f_bwd) * K / (total_ms * 1e-3) / 1e12
+        fwd_tf = world * f_fwd * K / (fwd_ms * 1e-3) / 1e12
+        bwd_tf = world * f_bwd * K / (bwd_ms * 1e-3) / 1e12
+        avg_fwd = sum(t_fwd) / K
+        avg_main = sum(t_main) / K
+        # Dominant kernel: the one with the larger share of the step.
+        if avg_main >= avg_fwd:
+            kname, kflops, kms = f"fa2_bwd_kernel<bf16,d={w.d}>", f_bwd, avg_main
+            ktraffic = BWD_MAIN_TRAFFIC_BYTES
+        else:
+            kname, kflops, kms = f"fa2_fwd_kernel<bf16,d={w.d}>", f_fwd, avg_fwd
+            ktraffic = None
+        achieved = kflops / (kms * 1e-3) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": config_of(w, world),
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_tf,
+            "fwd_frac_of_spec_bf16": fwd_tf / world / SPEC_BF16_TFLOPS,
+            "bwd_frac_of_spec_bf16": bwd_tf / world / SPEC_BF16_TFLOPS,
+            "fwd_frac_of_measured_bf16": fwd_tf / world / peaks["bf16_tflops"],
+            "bwd_frac_of_measured_bf16": bwd_tf / world / peaks["bf16_tflops"],
+            "ms": {"fwd": avg_fwd, "bwd_pre": sum(t_pre) / K, "bwd_main": avg_main,
+                   "bwd_dq_finalize": sum(t_fin) / K},
+            "e2e": {"value": world * (f_fwd + f_bwd) * K_e2e / (e2e_ms * 1e-3) / 1e12,
+                    "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": K_e2e},
+            "gpu_launches": 4 * K,
+            "roofline": {"bound": "tensor", "kernel": kname, "achieved": achieved,
+                         "peak": peaks["bf16_tflops"], "unit": UNIT,
+                         "frac": achieved / peaks["bf16_tflops"],
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "flops_per_launch": kflops, "ms_per_launch": kms,
+                         "traffic": ktraffic},
+            "clocks": sampler.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            oracle.build()
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

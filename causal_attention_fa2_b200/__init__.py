@@ -14,6 +14,7 @@ the backward, and the causal rule of Problem flash_forward (c).
 """
 from __future__ import annotations
 
+import ctypes
 import math
 from typing import Optional, Tuple
 
@@ -92,11 +93,14 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              lse: torch.Tensor, do: torch.Tensor, causal: bool = True,
              scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
              dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
-             dv: Optional[torch.Tensor] = None):
+             dv: Optional[torch.Tensor] = None, events=None):
     """dQ, dK, dV of sum(dO * O) via the recomputation backward.
 
     ``o`` and ``lse`` are the forward's outputs; ``workspace`` (optional) is a
     uint8 CUDA tensor of at least backward_workspace_bytes(...) bytes.
+    ``events`` (optional, for profiling): four recorded-once torch.cuda.Event
+    objects the library records at its kernel boundaries (before the D/L
+    pre-pass, after it, after the main pass, after the dQ finalisation).
     """
     B, H, N, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
@@ -112,12 +116,17 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    ev_arr = None
+    if events is not None:
+        if len(events) != 4:
+            raise ValueError("events must hold four torch.cuda.Event objects")
+        ev_arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
     with torch.cuda.device(q.device):
-        _native.check(_native.lib().fa2_backward(
+        _native.check(_native.lib().fa2_backward_timed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
             do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d,
             int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
-            workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
+            workspace.numel() * workspace.element_size(), _stream_handle(q.device), ev_arr))
     return dq, dk, dv
 
 

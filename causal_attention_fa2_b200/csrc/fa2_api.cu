@@ -174,8 +174,13 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
                              int B, int H, int N, int causal, float scale, fa2_dtype dtype,
                              uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
-                             uint32_t* status, unsigned long long timeout_ns) {
+                             uint32_t* status, unsigned long long timeout_ns,
+                             void* const* events) {
     using T = typename std::conditional<ES == 2, __nv_bfloat16, float>::type;
+    auto mark = [&](int i) -> bool {
+        if (!events || !events[i]) return true;
+        return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
+    };
     using Cfg = BwdCfg<ES, D>;
     const int BH = B * H;
     float* l2 = reinterpret_cast<float*>(ws_base + ws.l2_off);
@@ -184,10 +189,11 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     fa2_status st;
     // 1. D, log2-scaled L, zeroed dQ accumulator.
     const long long rows = static_cast<long long>(BH) * ws.n_pad;
+    if (!mark(0)) return FA2_ERR_CUDA;
     fa2_bwd_pre_kernel<T, D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
         static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, dq_acc, N, ws.n_pad,
         rows);
-    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     // 2. Main key/value-tile-outer pass.
     CUtensorMap mq, mk, mv, mdo, mdk, mdv;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
@@ -213,24 +219,24 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
     kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
-    if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     // 3. dQ = scale * accumulator.
     const long long n4 = static_cast<long long>(BH) * N * D / 4;
     fa2_bwd_dq_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<T*>(dq), scale, n4);
-    return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
+    return (cudaGetLastError() == cudaSuccess && mark(3)) ? FA2_OK : FA2_ERR_CUDA;
 }
 
 fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                            int H, int N, int d, int causal, float scale, fa2_dtype dtype,
                            uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
-                           uint32_t* status, unsigned long long timeout_ns) {
+                           uint32_t* status, unsigned long long timeout_ns, void* const* events) {
     if (dtype != FA2_BF16) return FA2_ERR_UNSUPPORTED_DTYPE;
 #define FA2_BWD_CASE(DD)                                                                      \
     case DD:                                                                                  \
         return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal,   \
-                                        scale, dtype, ws_base, ws, stream, status, timeout_ns);
+                                        scale, dtype, ws_base, ws, stream, status, timeout_ns, events);
     switch (d) {
         FA2_BWD_CASE(16)
         FA2_BWD_CASE(32)
@@ -272,10 +278,11 @@ size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype)
     return bwd_workspace_layout(B * H, N, d).total;
 }
 
-fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
-                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                        int H, int N, int d, int causal, float scale, fa2_dtype dtype,
-                        void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, int causal, float scale,
+                              fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                              fa2_stream_t stream, void* const* events) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
@@ -291,7 +298,16 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
     if ((st = init_device(&dev, &status)) != FA2_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype,
-                           static_cast<uint8_t*>(workspace), ws, s, status, kDefaultTimeoutNs);
+                           static_cast<uint8_t*>(workspace), ws, s, status, kDefaultTimeoutNs,
+                           events);
+}
+
+fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                        int H, int N, int d, int causal, float scale, fa2_dtype dtype,
+                        void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+    return fa2_backward_timed(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale,
+                              dtype, workspace, workspace_bytes, stream, nullptr);
 }
 
 fa2_status fa2_last_device_status(void) {

@@ -113,6 +113,23 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
                         void* workspace, size_t workspace_bytes, fa2_stream_t stream);
 
 /*
+ * fa2_backward plus timing hooks, for profiling: identical arguments and
+ * behaviour, and additionally records the caller's CUDA events (cudaEvent_t
+ * handles created on the current device; any entry may be NULL) on `stream`
+ * at the boundaries of the three kernels the backward enqueues:
+ *   events[0] before the D / L pre-pass,   events[1] after it,
+ *   events[2] after the key/value-tile main pass,
+ *   events[3] after the dQ finalisation.
+ * `events` itself may be NULL (then this is fa2_backward).  The library only
+ * records the events; the caller owns and destroys them.
+ */
+fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const void* o,
+                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, int causal, float scale,
+                              fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                              fa2_stream_t stream, void* const* events);
+
+/*
  * Status recorded by the kernels on the current device since the last call
  * of fa2_clear_device_status (FA2_OK or FA2_ERR_DEVICE_TIMEOUT).  Call it
  * after synchronising the streams the kernels ran on.  Returns FA2_ERR_CUDA
