@@ -32,6 +32,8 @@ SIGNATURES = {
     "fa2_backward_timed": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                            + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                               ctypes.c_void_p, ctypes.c_void_p]),
+    "fa2_backward_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
+                             + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "fa2_last_device_status": (ctypes.c_int, []),
     "fa2_clear_device_status": (ctypes.c_int, []),
     "fa2_status_string": (ctypes.c_char_p, [ctypes.c_int]),

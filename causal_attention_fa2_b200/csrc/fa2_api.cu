@@ -345,8 +345,64 @@ const char* fa2_status_string(fa2_status status) {
         case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel pipeline wait expired";
         case FA2_ERR_UNSUPPORTED_DEVICE: return "FA2_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
         case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1 and scale finite";
+        case FA2_ERR_SCRATCH_TOO_SMALL: return "FA2_ERR_SCRATCH_TOO_SMALL: the problem needs more than the 64 MiB built-in scratch of fa2_backward_noalloc; use fa2_backward with a workspace";
     }
     return "unknown fa2_status";
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fa2_backward_noalloc: the backward pass with its scratch in a fixed device
+// array, for callers that cannot allocate device memory (see fa2.h).
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+
+// The scratch itself.  In host code this name is only a stand-in for the
+// symbol, not a device address: the address is looked up per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+unsigned char* g_noalloc_ptr[fa2::kMaxDevices] = {};
+
+// Device address of the scratch array on the current device `dev`, looked up
+// once per device (with that device current) and cached.
+fa2_status noalloc_scratch(int dev, unsigned char** out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr) return FA2_ERR_CUDA;
+        g_noalloc_ptr[dev] = static_cast<unsigned char*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return FA2_OK;
+}
+
+}  // namespace
+
+extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v,
+                                           const void* o, const float* lse, const void* dout,
+                                           void* dq, void* dk, void* dv, int B, int H, int N,
+                                           int d, int causal, float scale, fa2_dtype dtype,
+                                           fa2_stream_t stream) {
+    fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
+    if (st != FA2_OK) return st;
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA2_ERR_NULL_PTR;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(lse, 4))
+        return FA2_ERR_MISALIGNED;
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d);
+    if (ws.total > kNoAllocScratchBytes) return FA2_ERR_SCRATCH_TOO_SMALL;
+    int dev;
+    uint32_t* status;
+    if ((st = init_device(&dev, &status)) != FA2_OK) return st;
+    unsigned char* scratch = nullptr;
+    if ((st = noalloc_scratch(dev, &scratch)) != FA2_OK) return st;
+    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, causal, scale, dtype,
+                           scratch, ws, reinterpret_cast<cudaStream_t>(stream), status,
+                           kDefaultTimeoutNs, nullptr);
+}

@@ -66,7 +66,8 @@ typedef enum {
     FA2_ERR_CUDA = 7,                 /* a CUDA runtime/driver call or launch failed */
     FA2_ERR_DEVICE_TIMEOUT = 8,       /* a kernel's pipeline watchdog expired      */
     FA2_ERR_UNSUPPORTED_DEVICE = 9,   /* the current device is not sm_100          */
-    FA2_ERR_BAD_ARGUMENT = 10         /* scale not finite, causal not 0/1, ...     */
+    FA2_ERR_BAD_ARGUMENT = 10,        /* scale not finite, causal not 0/1, ...     */
+    FA2_ERR_SCRATCH_TOO_SMALL = 11    /* problem too big for fa2_backward_noalloc  */
 } fa2_status;
 
 /* Opaque CUDA stream handle; identical to cudaStream_t / CUstream. */
@@ -128,6 +129,40 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
                               int B, int H, int N, int d, int causal, float scale,
                               fa2_dtype dtype, void* workspace, size_t workspace_bytes,
                               fa2_stream_t stream, void* const* events);
+
+/*
+ * fa2_backward_noalloc -- the backward pass for callers that cannot allocate
+ * device memory.  (Not part of the method the handout describes; it has no
+ * counterpart there.)
+ *
+ * Who needs it: code that is handed only its input and output buffers and has
+ * no allocator of its own -- for example a plugin running inside an inference
+ * or training engine whose memory pool owns all of the GPU's memory, or a hot
+ * path that must not call cudaMalloc because it would synchronise the device
+ * or fragment a fully reserved heap.  Such a caller cannot provide the
+ * workspace fa2_backward asks for.
+ *
+ * Arguments and results are those of fa2_backward without the workspace: the
+ * scratch (D, log2-scaled L and the fp32 dQ accumulator) lives in a fixed
+ * 64 MiB array that the library places in device memory of every GPU that
+ * loads it, held until the process exits.  Problems whose workspace would
+ * exceed it (fa2_backward_workspace_bytes(...) > 64 MiB, e.g. B*H*N*d above
+ * about 16 million elements) are rejected with FA2_ERR_SCRATCH_TOO_SMALL
+ * before anything is enqueued.  The call allocates nothing: no cudaMalloc,
+ * cudaFree, or allocating library routine.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the one array:
+ * the kernels re-initialise all of it that must start from zero, but two
+ * calls whose work overlaps on the GPU (different streams, no ordering
+ * between them) race on it and give wrong results.  Order such calls on one
+ * stream or with events.
+ */
+fa2_status fa2_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                const float* lse, const void* dout, void* dq, void* dk,
+                                void* dv, int B, int H, int N, int d, int causal, float scale,
+                                fa2_dtype dtype, fa2_stream_t stream);
 
 /*
  * Status recorded by the kernels on the current device since the last call

@@ -37,11 +37,11 @@ def test_exports_every_declared_function(fa2lib):
 def test_status_strings(fa2lib):
     from causal_attention_fa2_b200 import _native
     seen = set()
-    for code in range(11):
+    for code in range(12):
         s = _native.status_string(code)
         assert s.startswith("FA2_"), s
         seen.add(s)
-    assert len(seen) == 11
+    assert len(seen) == 12
     assert "unknown" in _native.status_string(99)
 
 
