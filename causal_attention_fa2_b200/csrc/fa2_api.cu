@@ -15,6 +15,7 @@
 #include "../../include/fa2.h"
 #include "fa2_bwd.cuh"
 #include "fa2_fwd.cuh"
+#include "fa2_fwd2.cuh"
 
 namespace fa2 {
 namespace {
@@ -79,7 +80,7 @@ fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2
     if (tiles * B * H > (1ll << 31) - 1) return FA2_ERR_BAD_SHAPE;
     if (!head_dim_supported(d)) return FA2_ERR_UNSUPPORTED_HEAD_DIM;
     if (causal != 0 && causal != 1) return FA2_ERR_BAD_ARGUMENT;
-    if (!std::isfinite(scale)) return FA2_ERR_BAD_ARGUMENT;
+    if (!std::isfinite(scale) || !(scale > 0.f)) return FA2_ERR_BAD_ARGUMENT;
     return FA2_OK;
 }
 
@@ -127,6 +128,14 @@ fa2_status set_smem(Kernel k, int bytes) {
                : FA2_ERR_CUDA;
 }
 
+// The two-query-tile forward needs two Q tiles plus at least one K/V stage in
+// shared memory; fp32 (TF32) inputs at d = 128 do not fit and use the
+// one-tile kernel.
+template <int ES, int D>
+constexpr bool use_two_tile_forward() {
+    return Fwd2Cfg<ES, D>::kFits;
+}
+
 template <int ES, int D>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int H, int N, int causal, float scale, fa2_dtype dtype,
@@ -148,10 +157,19 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
-    auto kern = fa2_fwd_kernel<ES, D>;
-    if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
-    const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    if constexpr (use_two_tile_forward<ES, D>()) {
+        // Two query tiles per CTA (softmax of one overlaps the MMAs of the other).
+        using Cfg2 = Fwd2Cfg<ES, D>;
+        auto kern = fa2_fwd2_kernel<ES, D>;
+        if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
+        const unsigned pairs = static_cast<unsigned>((p.n_tiles + 1) / 2);
+        kern<<<pairs * static_cast<unsigned>(BH), Cfg2::kThreads, Cfg2::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    } else {
+        auto kern = fa2_fwd_kernel<ES, D>;
+        if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
+        const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+    }
     return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
@@ -344,7 +362,7 @@ const char* fa2_status_string(fa2_status status) {
         case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call or kernel launch failed";
         case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel pipeline wait expired";
         case FA2_ERR_UNSUPPORTED_DEVICE: return "FA2_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
-        case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1 and scale finite";
+        case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1 and scale finite and > 0";
         case FA2_ERR_SCRATCH_TOO_SMALL: return "FA2_ERR_SCRATCH_TOO_SMALL: the problem needs more than the 64 MiB built-in scratch of fa2_backward_noalloc; use fa2_backward with a workspace";
     }
     return "unknown fa2_status";

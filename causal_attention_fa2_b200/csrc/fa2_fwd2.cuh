@@ -1,0 +1,426 @@
+// fa2_fwd2.cuh -- FlashAttention-2 forward for sm_100a, two query tiles per CTA.
+//
+// Same computation as fa2_fwd.cuh (CS336 A2 Systems handout section 4.2.2,
+// Algorithm 1, with the causal rule of Problem flash_forward (c)), organised so
+// that the exponentials of one query tile overlap the tensor-core work of the
+// other:
+//
+//   warp 0     TMA producer: Q_A and Q_B (two adjacent 128-row query tiles of
+//              one head) once, then K_j / V_j through rings of shared-memory
+//              stages.
+//   warp 1     MMA issuer (one thread).  Per key tile j it issues, in order,
+//                PV_A(j-1) -> S_A(j) ... as soon as each operand is ready:
+//                  O_A += P_A(j) V_j ; S_A(j+1) = Q_A K_{j+1}^T ;
+//                  O_B += P_B(j) V_j ; S_B(j+1) = Q_B K_{j+1}^T
+//              so while softmax warpgroup A works on S_A(j+1) the tensor core
+//              runs PV_B(j) and S_B(j+1), and the other way round.
+//   warps 2-5  softmax warpgroup for tile A; warps 6-9 for tile B.  Thread t
+//              owns query row t of its tile (tensor-memory lane t).
+//
+// Tensor memory (512 columns): S_A | S_B | O_A | O_B, 128 columns each; P is
+// written over its S buffer (bf16 pairs, or fp32 for the TF32 path) and read
+// by the PV MMA as its A operand.
+//
+// Per-row arithmetic: the running max is kept on raw scores (scale > 0), so
+// each exponent is one fused multiply-add feeding ex2:
+//   p = 2^(s * scale*log2(e) - m * scale*log2(e)).
+// The reference max is raised only when a row's max grows by more than 2^8 in
+// the exponent (then O and l are rescaled); O / l and L are exact for any
+// reference.
+#pragma once
+
+#include <cstdint>
+
+#include "fa2_traits.cuh"
+#include "fa2_fwd.cuh"
+
+namespace fa2 {
+
+template <int ES, int D>
+struct Fwd2Cfg {
+    using G = TileGeom<ES, D>;
+    static constexpr int kThreads = 320;
+    static constexpr int kBudget = 227 * 1024 - 2048;
+    static constexpr int kQBytes = 2 * G::kTileBytesK;
+    static constexpr int kFree = kBudget - kQBytes;
+    static constexpr int kKV = G::kTileBytesK + G::kTileBytesMN;
+    static constexpr int kPairs = kFree / kKV;
+    static constexpr int kStages = kPairs > 4 ? 4 : kPairs;
+    static constexpr bool kFits = kPairs >= 1;
+    static constexpr int kSmemBytes = 1024 + kQBytes + (kStages > 0 ? kStages : 1) * kKV;
+    static constexpr uint32_t kTmemCols = 512;
+    // TMEM columns of tile t's score buffer and output accumulator.
+    static __device__ __forceinline__ uint32_t col_s(int t) { return 128u * t; }
+    static __device__ __forceinline__ uint32_t col_o(int t) { return 256u + 128u * t; }
+};
+
+// One softmax warpgroup: processes query tile `t` (0 = A, 1 = B) for key
+// tiles 0 .. n_kv-1, then writes its O tile and L rows.
+template <int ES, int D>
+__device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_tile, int n_kv,
+                                             int bh, uint32_t tmem, uint8_t* sQt,
+                                             uint64_t* bar_s_full, uint64_t* bar_p_full,
+                                             uint64_t* bar_o_done,
+                                             volatile uint32_t* abort_flag,
+                                             const CUtensorMap* tm_o) {
+    using Cfg = Fwd2Cfg<ES, D>;
+    using G = typename Cfg::G;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
+    const uint32_t s_tmem = lane_base + Cfg::col_s(t);
+    const uint32_t o_tmem = lane_base + Cfg::col_o(t);
+    const uint64_t tmo = p.timeout_ns;
+    const float sl2 = p.scale_log2;
+    const int q_row0 = q_tile * kTileRows;
+    float m_raw = -INFINITY;    // reference max of raw scores
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+        if (!ptx::mbar_wait(bar_s_full, j & 1, abort_flag, tmo)) { ok = false; break; }
+        ptx::tc_fence_after();
+        float s[128];
+        {
+            uint32_t u[32];
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                ptx::tmem_ld32(s_tmem + c0, u);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(u[c]);
+            }
+        }
+        const int kv_valid = p.N - j * kTileRows;
+        if (p.causal && j == q_tile) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c > r) s[c] = -INFINITY;
+        }
+        if (kv_valid < kTileRows) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+                if (c >= kv_valid) s[c] = -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+            mx0 = fmaxf(mx0, s[c]);
+            mx1 = fmaxf(mx1, s[c + 1]);
+            mx2 = fmaxf(mx2, s[c + 2]);
+            mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_new = fmaxf(m_raw, mx);
+        const bool raise = (m_new - m_raw) * sl2 > 8.f;   // true on the first tile
+        float alpha = 1.f;
+        if (raise) {
+            alpha = ptx::ex2_approx((m_raw - m_new) * sl2);
+            m_raw = m_new;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+            // PV(j-1) must have finished before O is rescaled.
+            if (!ptx::mbar_wait(bar_o_done, (j - 1) & 1, abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+                uint32_t u[16];
+                ptx::tmem_ld16(o_tmem + c0, u);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c) u[c] = __float_as_uint(__uint_as_float(u[c]) * alpha);
+                ptx::tmem_st16(o_tmem + c0, u);
+            }
+        }
+        l *= alpha;
+        const float neg = -m_raw * sl2;
+        float rs0 = 0.f, rs1 = 0.f;
+        // Exponentiate 32 columns at a time and store them as P right away.
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+                s[c0 + c] = ptx::ex2_approx(fmaf(s[c0 + c], sl2, neg));
+                s[c0 + c + 1] = ptx::ex2_approx(fmaf(s[c0 + c + 1], sl2, neg));
+                rs0 += s[c0 + c];
+                rs1 += s[c0 + c + 1];
+            }
+            if constexpr (G::kF32) {
+                uint32_t u[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(s[c0 + c]);
+                ptx::tmem_st32(s_tmem + c0, u);
+            } else {
+                uint32_t u[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) u[c] = ptx::pack_bf16x2(s[c0 + 2 * c], s[c0 + 2 * c + 1]);
+                ptx::tmem_st16(s_tmem + c0 / 2, u);
+            }
+        }
+        l += rs0 + rs1;
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar_p_full);
+    }
+    // ---------------- epilogue: O / l -> shared memory (this tile's Q slot) -> TMA.
+    if (ok) ok = ptx::mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag, tmo);
+    if (ok) {
+        ptx::tc_fence_after();
+        const float inv_l = 1.f / l;
+#pragma unroll
+        for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+            uint32_t u[16];
+            ptx::tmem_ld16(o_tmem + c0, u);
+            ptx::tmem_wait_ld();
+            if constexpr (G::kF32) {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int col = c0 + 4 * q4;
+                    if (col < D) {
+                        uint4 w;
+                        w.x = __float_as_uint(__uint_as_float(u[4 * q4 + 0]) * inv_l);
+                        w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * inv_l);
+                        w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * inv_l);
+                        w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * inv_l);
+                        *reinterpret_cast<uint4*>(sQt + kmajor_chunk_offset<G>(r, col)) = w;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int h8 = 0; h8 < 2; ++h8) {
+                    const int col = c0 + 8 * h8;
+                    if (col < D) {
+                        uint4 w;
+                        const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
+                        w.x = ptx::pack_bf16x2(f[0] * inv_l, f[1] * inv_l);
+                        w.y = ptx::pack_bf16x2(f[2] * inv_l, f[3] * inv_l);
+                        w.z = ptx::pack_bf16x2(f[4] * inv_l, f[5] * inv_l);
+                        w.w = ptx::pack_bf16x2(f[6] * inv_l, f[7] * inv_l);
+                        *reinterpret_cast<uint4*>(sQt + kmajor_chunk_offset<G>(r, col)) = w;
+                    }
+                }
+            }
+        }
+        const int q_row = q_row0 + r;
+        if (q_row < p.N)
+            p.lse[static_cast<size_t>(bh) * p.N + q_row] =
+                (m_raw * sl2 + __log2f(l)) * 0.69314718055994531f;
+        ptx::fence_async_smem();
+    }
+    if (t == 0)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+    else
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+    if (ok && (threadIdx.x & 127) == 0) {
+        for (int b = 0; b < G::kNBoxK; ++b)
+            ptx::tma_store_3d(tm_o, sQt + b * kTileRows * G::kRowBK, b * G::kBoxK, q_row0, bh);
+        ptx::tma_store_commit();
+        ptx::tma_store_wait_all();
+    }
+}
+
+template <int ES, int D>
+__global__ void __launch_bounds__(320, 1)
+fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const FwdParams p) {
+    using Cfg = Fwd2Cfg<ES, D>;
+    using G = typename Cfg::G;
+    constexpr int ST = Cfg::kStages;
+    static_assert(ST >= 1, "two query tiles and one K/V stage do not fit in shared memory");
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar_q_full;
+    __shared__ uint64_t bar_k_full[ST], bar_k_empty[ST], bar_v_full[ST], bar_v_empty[ST];
+    __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2], bar_drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile uint32_t abort_flag;
+
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sQ[2] = {smem, smem + G::kTileBytesK};
+    uint8_t* sK = smem + Cfg::kQBytes;
+    uint8_t* sV = sK + ST * G::kTileBytesK;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: a pair of adjacent query tiles (2t, 2t+1) of one head;
+    // causal pairs are issued longest first.
+    const int n_pairs = (p.n_tiles + 1) >> 1;
+    const int item = blockIdx.x;
+    const int rank = item / p.BH;
+    const int bh = item - rank * p.BH;
+    const int pair = p.causal ? (n_pairs - 1 - rank) : rank;
+    const int tile[2] = {2 * pair, 2 * pair + 1};
+    const bool has_b = tile[1] < p.n_tiles;
+    const int n_kv_t[2] = {p.causal ? tile[0] + 1 : p.n_tiles,
+                           has_b ? (p.causal ? tile[1] + 1 : p.n_tiles) : 0};
+    const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        ptx::mbar_init(&bar_q_full, 1);
+        for (int s = 0; s < ST; ++s) {
+            ptx::mbar_init(&bar_k_full[s], 1);
+            ptx::mbar_init(&bar_k_empty[s], 1);
+            ptx::mbar_init(&bar_v_full[s], 1);
+            ptx::mbar_init(&bar_v_empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            ptx::mbar_init(&bar_s_full[t], 1);
+            ptx::mbar_init(&bar_p_full[t], 4);
+            ptx::mbar_init(&bar_o_done[t], 1);
+        }
+        ptx::mbar_init(&bar_drain, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_q);
+            ptx::prefetch_tmap(&tm_k);
+            ptx::prefetch_tmap(&tm_v);
+            const uint64_t keep = ptx::policy_evict_last();
+            ptx::mbar_arrive_expect_tx(&bar_q_full, (has_b ? 2 : 1) * G::kTileBytesK);
+            for (int t = 0; t < (has_b ? 2 : 1); ++t)
+                for (int b = 0; b < G::kNBoxK; ++b)
+                    ptx::tma_load_3d(sQ[t] + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full,
+                                     b * G::kBoxK, tile[t] * kTileRows, bh);
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % ST;
+                const uint32_t ph = ((j / ST) & 1) ^ 1;
+                if (j >= ST && !ptx::mbar_wait(&bar_k_empty[s], ph, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_k_full[s], G::kTileBytesK);
+                for (int b = 0; b < G::kNBoxK; ++b)
+                    ptx::tma_load_3d_hint(sK + s * G::kTileBytesK + b * kTileRows * G::kRowBK, &tm_k,
+                                          &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh, keep);
+                k_issued = j + 1;
+                if (j >= ST && !ptx::mbar_wait(&bar_v_empty[s], ph, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_v_full[s], G::kTileBytesMN);
+                for (int b = 0; b < G::kNBoxMN; ++b)
+                    ptx::tma_load_3d_hint(sV + s * G::kTileBytesMN + b * kTileRows * G::kRowBMN, &tm_v,
+                                          &bar_v_full[s], b * G::kBoxMN, j * kTileRows, bh, keep);
+                v_issued = j + 1;
+            }
+            if (abort_flag) {
+                constexpr uint64_t kDrainNs = 20000000ull;
+                ptx::mbar_wait_drain(&bar_q_full, 0, kDrainNs);
+                for (int t = k_issued - 1; t >= 0 && t >= k_issued - ST; --t)
+                    ptx::mbar_wait_drain(&bar_k_full[t % ST], (t / ST) & 1, kDrainNs);
+                for (int t = v_issued - 1; t >= 0 && t >= v_issued - ST; --t)
+                    ptx::mbar_wait_drain(&bar_v_full[t % ST], (t / ST) & 1, kDrainNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
+            constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
+            const uint32_t q_addr[2] = {ptx::smem_addr(sQ[0]), ptx::smem_addr(sQ[1])};
+            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            auto issue_s = [&](int t, int j) {
+                const uint32_t k_addr = ptx::smem_addr(sK + (j % ST) * G::kTileBytesK);
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk) {
+                    const uint64_t a = desc_kmajor<G>(q_addr[t], kk);
+                    const uint64_t b = desc_kmajor<G>(k_addr, kk);
+                    if constexpr (G::kF32)
+                        ptx::mma_tf32_ss(tmem + Cfg::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_f16_ss(tmem + Cfg::col_s(t), a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                ptx::mma_commit(&bar_s_full[t]);
+            };
+            auto issue_pv = [&](int t, int j) -> bool {
+                if (!ptx::mbar_wait(&bar_p_full[t], j & 1, &abort_flag, tmo)) return false;
+                ptx::tc_fence_after();
+                const uint32_t v_addr = ptx::smem_addr(sV + (j % ST) * G::kTileBytesMN);
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsRows; ++kk) {
+                    const uint64_t b = desc_mnmajor<G>(v_addr, kk);
+                    const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+                    if constexpr (G::kF32)
+                        ptx::mma_tf32_ts(tmem + Cfg::col_o(t), tmem + Cfg::col_s(t) + kk * 8, b, idesc_pv, acc);
+                    else
+                        ptx::mma_f16_ts(tmem + Cfg::col_o(t), tmem + Cfg::col_s(t) + kk * 8, b, idesc_pv, acc);
+                }
+                ptx::mma_commit(&bar_o_done[t]);
+                return true;
+            };
+            // Prologue: S_A(0), S_B(0).
+            if (ok) ok = ptx::mbar_wait(&bar_k_full[0], 0, &abort_flag, tmo);
+            if (ok) {
+                ptx::tc_fence_after();
+                issue_s(0, 0);
+                if (n_kv_t[1] > 0) issue_s(1, 0);
+                ptx::mma_commit(&bar_k_empty[0]);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % ST;
+                const bool next_k = (j + 1) < n_kv;
+                if (!ptx::mbar_wait(&bar_v_full[s], (j / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                bool k_waited = false;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j < n_kv_t[t]) {
+                        if (!issue_pv(t, j)) { ok = false; break; }
+                    }
+                    if (j + 1 < n_kv_t[t]) {
+                        if (!k_waited) {
+                            const int s1 = (j + 1) % ST;
+                            if (!ptx::mbar_wait(&bar_k_full[s1], ((j + 1) / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            k_waited = true;
+                        }
+                        issue_s(t, j + 1);
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(&bar_v_empty[s]);
+                if (next_k) {
+                    if (!k_waited) {
+                        // No tile uses K_{j+1}; keep the ring's bookkeeping.
+                        const int s1 = (j + 1) % ST;
+                        if (!ptx::mbar_wait(&bar_k_full[s1], ((j + 1) / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                    }
+                    ptx::mma_commit(&bar_k_empty[(j + 1) % ST]);
+                }
+            }
+            if (!ok) {
+                ptx::mma_commit(&bar_drain);
+                ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+            }
+        }
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        const int t = (warp - 2) >> 2;       // 0: warps 2-5 (tile A), 1: warps 6-9 (tile B)
+        if (n_kv_t[t] > 0) {
+            fwd2_softmax<ES, D>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
+                                &bar_p_full[t], &bar_o_done[t], &abort_flag, &tm_o);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+    if (threadIdx.x == 0 && abort_flag) atomicCAS(p.status, 0u, kDevStatusTimeout);
+}
+
+}  // namespace fa2

@@ -66,7 +66,7 @@ typedef enum {
     FA2_ERR_CUDA = 7,                 /* a CUDA runtime/driver call or launch failed */
     FA2_ERR_DEVICE_TIMEOUT = 8,       /* a kernel's pipeline watchdog expired      */
     FA2_ERR_UNSUPPORTED_DEVICE = 9,   /* the current device is not sm_100          */
-    FA2_ERR_BAD_ARGUMENT = 10,        /* scale not finite, causal not 0/1, ...     */
+    FA2_ERR_BAD_ARGUMENT = 10,        /* scale not finite and > 0, causal not 0/1  */
     FA2_ERR_SCRATCH_TOO_SMALL = 11    /* problem too big for fa2_backward_noalloc  */
 } fa2_status;
 
@@ -81,7 +81,7 @@ typedef struct CUstream_st* fa2_stream_t;
  *                 rounded once from fp32
  *   lse      out: [B, H, N] float32, L_i = log sum_j exp(S_ij)
  *   causal   1 = causal mask, 0 = full attention
- *   scale    finite multiplier of Q K^T (1/sqrt(d) in the handout)
+ *   scale    finite, positive multiplier of Q K^T (1/sqrt(d) in the handout)
  * Returns FA2_OK once the work is enqueued, or a validation / launch error.
  */
 fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse,

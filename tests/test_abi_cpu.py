@@ -77,6 +77,8 @@ def test_forward_validation(fa2lib):
     assert fwd(L, causal=2) == 10                  # FA2_ERR_BAD_ARGUMENT
     assert fwd(L, scale=float("inf")) == 10
     assert fwd(L, scale=float("nan")) == 10
+    assert fwd(L, scale=0.0) == 10                 # the scale must be positive
+    assert fwd(L, scale=-0.125) == 10
 
 
 def test_backward_validation(fa2lib):
