@@ -213,7 +213,8 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
         rows);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     // 2. Main key/value-tile-outer pass.
-    CUtensorMap mq, mk, mv, mdo, mdk, mdv;
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
+    if ((st = make_maps_kmajor<4, D>(&mdq, dq_acc, FA2_FP32, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mv, v, dtype, N, BH)) != FA2_OK) return st;
@@ -236,7 +237,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     auto kern = fa2_bwd_kernel<ES, D>;
     if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
     if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     // 3. dQ = scale * accumulator.
     const long long n4 = static_cast<long long>(BH) * N * D / 4;

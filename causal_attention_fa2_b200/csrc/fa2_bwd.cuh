@@ -117,50 +117,71 @@ template <int ES, int D>
 struct BwdCfg {
     using G = TileGeom<ES, D>;
     using GS = TileGeom<ES, 128>;          // a 128 x 128 dS tile, K-major along queries
+    using G4 = TileGeom<4, D>;             // the fp32 dQ accumulator's boxes
     static_assert(ES == 2, "the backward kernel is written for 16-bit inputs");
+    // One fp32 dQ box (128 rows x kBoxK columns) staged for a TMA reduce-add.
+    static constexpr int kStageBytes = kTileRows * G4::kRowBK;
     static constexpr int kThreads = 320;   // 10 warps
     static constexpr int kTile = G::kTileBytesK;
     // 227 KB minus the alignment pad and the static shared memory (per-warp
     // L/D vectors and barriers).
     static constexpr int kBudget = 227 * 1024 - 1024 - 9 * 1024;
-    // K, V resident; dS staging; Q_i / dO_i share one ring of slots.
-    static constexpr int kFixed = 2 * kTile + GS::kTileBytesK;
+    // K, V resident; dS staging; Q_i in a ring of kQSlots, dO_i in a ring of
+    // kDOSlots.  Q_i lives from S(i) to dK(i), dO_i from dP(i) to dV(i).
+    static constexpr int kFixed = 2 * kTile + GS::kTileBytesK + kStageBytes;
     static constexpr int kSlots0 = (kBudget - kFixed) / kTile;
     static constexpr int kSlots = kSlots0 > 4 ? 4 : kSlots0;
-    static_assert(kSlots >= 2, "shared memory too small for the Q/dO ring");
+    static_assert(kSlots >= 3, "shared memory too small for the Q/dO rings");
+    static constexpr int kQSlots = 2;
+    static constexpr int kDOSlots = kSlots - 2;
     static constexpr int kSmemBytes = 1024 + kFixed + kSlots * kTile;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 128, kColDV = 256, kColDK = 384;
 };
 
+// Key/value-tile-outer backward.  One CTA per (key tile j, head), looping over
+// the query tiles i that see key tile j.  Per query tile the MMA issuer runs
+//   dV += P^T(i) dO(i); S^T(i+1) = K Q(i+1)^T;
+//   dK += dS^T(i) Q(i); dQ(i) = dS(i) K; dP^T(i+1) = V dO(i+1)^T
+// so that S^T(i+1) overlaps the dS(i) computation and dK(i)/dQ(i)/dP^T(i+1)
+// overlap the P(i+1) computation.  Warps: 0 TMA producer, 1 MMA issuer, 2-5
+// P/dS warpgroup (one key row per thread), 6-9 dQ warpgroup (one query row per
+// thread).
 template <int ES, int D>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-               const BwdParams p) {
+               const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using Cfg = BwdCfg<ES, D>;
     using G = typename Cfg::G;
     using GS = typename Cfg::GS;
-    constexpr int NS = Cfg::kSlots;
+    using G4 = typename Cfg::G4;
+    constexpr int QS = Cfg::kQSlots;
+    constexpr int DS = Cfg::kDOSlots;
     constexpr int TB = Cfg::kTile;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full;
-    __shared__ uint64_t bar_slot_full[NS], bar_slot_empty[NS];
-    __shared__ uint64_t bar_s_full, bar_pds_ready, bar_dq_full, bar_dq_free, bar_dkv_full, bar_drain;
+    __shared__ uint64_t bar_q_full[QS], bar_q_empty[QS], bar_do_full[DS], bar_do_empty[DS];
+    __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready;
+    __shared__ uint64_t bar_dq_full, bar_dq_free, bar_dkv_full, bar_drain;
+    __shared__ uint64_t bar_stage_full, bar_stage_free;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     // Per-warp copies of the current query tile's L*log2(e) and D vectors
     // (double-buffered; each warp syncs only itself).
-    __shared__ float sL2[4][2][kTileRows], sDv[4][2][kTileRows];
+    __shared__ __align__(16) float sL2[4][2][kTileRows];
+    __shared__ __align__(16) float sDv[4][2][kTileRows];
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t* sK = smem;
     uint8_t* sV = sK + TB;
     uint8_t* sDS = sV + TB;
-    uint8_t* sSlots = sDS + GS::kTileBytesK;
+    uint8_t* sQr = sDS + GS::kTileBytesK;
+    uint8_t* sDOr = sQr + QS * TB;
+    uint8_t* sStage = sDOr + DS * TB;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -177,13 +198,18 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (threadIdx.x == 0) {
         abort_flag = 0u;
         ptx::mbar_init(&bar_kv_full, 1);
-        for (int s = 0; s < NS; ++s) { ptx::mbar_init(&bar_slot_full[s], 1); ptx::mbar_init(&bar_slot_empty[s], 1); }
+        for (int s = 0; s < QS; ++s) { ptx::mbar_init(&bar_q_full[s], 1); ptx::mbar_init(&bar_q_empty[s], 1); }
+        for (int s = 0; s < DS; ++s) { ptx::mbar_init(&bar_do_full[s], 1); ptx::mbar_init(&bar_do_empty[s], 1); }
         ptx::mbar_init(&bar_s_full, 1);
-        ptx::mbar_init(&bar_pds_ready, 4);
+        ptx::mbar_init(&bar_dp_full, 1);
+        ptx::mbar_init(&bar_p_ready, 4);
+        ptx::mbar_init(&bar_ds_ready, 4);
         ptx::mbar_init(&bar_dq_full, 1);
         ptx::mbar_init(&bar_dq_free, 4);
         ptx::mbar_init(&bar_dkv_full, 1);
         ptx::mbar_init(&bar_drain, 1);
+        ptx::mbar_init(&bar_stage_full, 4);
+        ptx::mbar_init(&bar_stage_free, 1);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -206,24 +232,29 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ptx::tma_load_3d(sK + b * kTileRows * G::kRowBK, &tm_k, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
                 ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
             }
-            // Load t = 2*it is Q_i, t = 2*it + 1 is dO_i; slot t % NS.
-            int issued = 0;
-            for (int t = 0; t < 2 * n_q; ++t) {
-                const int s = t % NS;
-                if (t >= NS && !ptx::mbar_wait(&bar_slot_empty[s], ((t / NS) & 1) ^ 1, &abort_flag, tmo)) break;
-                const int i = i_begin + (t >> 1);
-                const CUtensorMap* map = (t & 1) ? &tm_do : &tm_q;
-                uint8_t* dst = sSlots + s * TB;
-                ptx::mbar_arrive_expect_tx(&bar_slot_full[s], TB);
+            int q_issued = 0, do_issued = 0;
+            for (int it = 0; it < n_q; ++it) {
+                const int row0 = (i_begin + it) * kTileRows;
+                const int qs = it % QS;
+                if (it >= QS && !ptx::mbar_wait(&bar_q_empty[qs], ((it / QS) & 1) ^ 1, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_q_full[qs], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(dst + b * kTileRows * G::kRowBK, map, &bar_slot_full[s], b * G::kBoxK, i * kTileRows, bh);
-                issued = t + 1;
+                    ptx::tma_load_3d(sQr + qs * TB + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full[qs], b * G::kBoxK, row0, bh);
+                q_issued = it + 1;
+                const int ds = it % DS;
+                if (it >= DS && !ptx::mbar_wait(&bar_do_empty[ds], ((it / DS) & 1) ^ 1, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_do_full[ds], TB);
+                for (int b = 0; b < G::kNBoxK; ++b)
+                    ptx::tma_load_3d(sDOr + ds * TB + b * kTileRows * G::kRowBK, &tm_do, &bar_do_full[ds], b * G::kBoxK, row0, bh);
+                do_issued = it + 1;
             }
             if (abort_flag) {
                 constexpr uint64_t kDrainNs = 20000000ull;
                 ptx::mbar_wait_drain(&bar_kv_full, 0, kDrainNs);
-                for (int t = issued - 1; t >= 0 && t >= issued - NS; --t)
-                    ptx::mbar_wait_drain(&bar_slot_full[t % NS], (t / NS) & 1, kDrainNs);
+                for (int t = q_issued - 1; t >= 0 && t >= q_issued - QS; --t)
+                    ptx::mbar_wait_drain(&bar_q_full[t % QS], (t / QS) & 1, kDrainNs);
+                for (int t = do_issued - 1; t >= 0 && t >= do_issued - DS; --t)
+                    ptx::mbar_wait_drain(&bar_do_full[t % DS], (t / DS) & 1, kDrainNs);
             }
         }
     } else if (warp == 1) {
@@ -235,45 +266,60 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t k_addr = ptx::smem_addr(sK);
             const uint32_t v_addr = ptx::smem_addr(sV);
             const uint32_t ds_addr = ptx::smem_addr(sDS);
-            bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
-            for (int it = 0; ok && it < n_q; ++it) {
-                const int tq = 2 * it, tdo = 2 * it + 1;
-                const int sq = tq % NS, sdo = tdo % NS;
-                const uint32_t q_addr = ptx::smem_addr(sSlots + sq * TB);
-                const uint32_t do_addr = ptx::smem_addr(sSlots + sdo * TB);
-                // S^T = K_j Q_i^T   (Eq. 13, transposed: rows are keys)
-                if (!ptx::mbar_wait(&bar_slot_full[sq], (tq / NS) & 1, &abort_flag, tmo)) { ok = false; break; }
+            auto q_addr = [&](int it) { return ptx::smem_addr(sQr + (it % QS) * TB); };
+            auto do_addr = [&](int it) { return ptx::smem_addr(sDOr + (it % DS) * TB); };
+            // S^T = K_j Q_i^T   (Eq. 13, transposed: rows are keys)
+            auto issue_s = [&](int it) -> bool {
+                if (!ptx::mbar_wait(&bar_q_full[it % QS], (it / QS) & 1, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
+                const uint32_t qa = q_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_f16_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(q_addr, kk), idesc_s, kk > 0 ? 1u : 0u);
-                // dP^T = V_j dO_i^T   (Eq. 16, transposed); its columns also
-                // hold the previous dQ tile, which must have been drained.
-                if (it > 0 && !ptx::mbar_wait(&bar_dq_free, (it - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
-                if (!ptx::mbar_wait(&bar_slot_full[sdo], (tdo / NS) & 1, &abort_flag, tmo)) { ok = false; break; }
-                ptx::tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_f16_ss(tmem + Cfg::kColDP, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(do_addr, kk), idesc_s, kk > 0 ? 1u : 0u);
+                    ptx::mma_f16_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk), idesc_s, kk > 0 ? 1u : 0u);
                 ptx::mma_commit(&bar_s_full);
-                // P^T (in TMEM) and dS^T (in shared memory) are ready.
-                if (!ptx::mbar_wait(&bar_pds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                return true;
+            };
+            // dP^T = V_j dO_i^T   (Eq. 16, transposed)
+            auto issue_dp = [&](int it) -> bool {
+                if (!ptx::mbar_wait(&bar_do_full[it % DS], (it / DS) & 1, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
-                // dV_j += P^T dO_i   (Eq. 15)
+                const uint32_t da = do_addr(it);
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk)
+                    ptx::mma_f16_ss(tmem + Cfg::kColDP, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_dp_full);
+                return true;
+            };
+            bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
+            if (ok) ok = issue_s(0) && issue_dp(0);
+            for (int it = 0; ok && it < n_q; ++it) {
+                // dV_j += P^T dO_i   (Eq. 15), P^T read from the score columns.
+                if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t da = do_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8, desc_mnmajor<G>(do_addr, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar_slot_empty[sdo]);
-                // dK_j += dS^T Q_i   (Eq. 19 without the scale)
+                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8, desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(&bar_do_empty[it % DS]);
+                // Next query tile's scores while the P/dS warps work on dS(i).
+                if (it + 1 < n_q && !issue_s(it + 1)) { ok = false; break; }
+                // dK_j += dS^T Q_i  and  dQ_i = dS K_j   (Eqs. 19 and 18 without the scale)
+                if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t qa = q_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ss(tmem + Cfg::kColDK, desc_kmajor<GS>(ds_addr, kk), desc_mnmajor<G>(q_addr, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar_slot_empty[sq]);
-                // dQ_i (partial) = dS K_j   (Eq. 18 without the scale)
+                    ptx::mma_f16_ss(tmem + Cfg::kColDK, desc_kmajor<GS>(ds_addr, kk), desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(&bar_q_empty[it % QS]);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
                     ptx::mma_f16_ss(tmem + Cfg::kColDQ, desc_mnmajor<GS>(ds_addr, kk), desc_mnmajor<G>(k_addr, kk), idesc_dq, kk > 0 ? 1u : 0u);
                 ptx::mma_commit(&bar_dq_full);
+                // dP^T(i+1) reuses the dQ columns once the dQ warps have read them.
+                if (it + 1 < n_q) {
+                    if (!ptx::mbar_wait(&bar_dq_free, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                    if (!issue_dp(it + 1)) { ok = false; break; }
+                }
             }
             if (ok) {
                 ptx::mma_commit(&bar_dkv_full);
@@ -314,45 +360,72 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     nd[m] = p.dvec[vec_base + static_cast<size_t>(i + 1) * kTileRows + lane + 32 * m];
                 }
             }
+            const bool diag = p.causal && (i == kv_tile);
+            // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14)
             if (!ptx::mbar_wait(&bar_s_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            const bool diag = p.causal && (i == kv_tile);
+            uint32_t pk[64];                               // P^T row as bf16 pairs
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                uint32_t us[32], ud[32];
-                ptx::tmem_ld32(lane_base + Cfg::kColS + c0, us);
-                ptx::tmem_ld32(lane_base + Cfg::kColDP + c0, ud);
+            for (int h0 = 0; h0 < 128; h0 += 32) {
+                uint32_t us[32];
+                ptx::tmem_ld32(lane_base + Cfg::kColS + h0, us);
                 ptx::tmem_wait_ld();
-                uint32_t pw[16], dw[16];
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    float pv[2], dsv[2];
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 lv = *reinterpret_cast<const float4*>(&sL2[wq][b][h0 + c]);
+                    const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+                    float pv[4];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int q = c0 + c + h;
-                        float pe = ptx::ex2_approx(__uint_as_float(us[c + h]) * sl2 - sL2[wq][b][q]);
+                    for (int h = 0; h < 4; ++h) {
+                        const int q = h0 + c + h;
+                        float pe = ptx::ex2_approx(fmaf(__uint_as_float(us[c + h]), sl2, -lq[h]));
                         if ((diag && r > q) || !key_valid) pe = 0.f;
                         pv[h] = pe;
-                        dsv[h] = pe * (__uint_as_float(ud[c + h]) - sDv[wq][b][q]);
                     }
-                    pw[c >> 1] = ptx::pack_bf16x2(pv[0], pv[1]);
-                    dw[c >> 1] = ptx::pack_bf16x2(dsv[0], dsv[1]);
+                    pk[(h0 + c) >> 1] = ptx::pack_bf16x2(pv[0], pv[1]);
+                    pk[((h0 + c) >> 1) + 1] = ptx::pack_bf16x2(pv[2], pv[3]);
                 }
-                // P^T chunk -> TMEM columns [c0/2, c0/2 + 16) of the score
-                // buffer (already read), as the A operand of dV += P^T dO.
-                ptx::tmem_st16(lane_base + Cfg::kColS + c0 / 2, pw);
-                // dS^T chunk -> shared memory row r, queries [c0, c0 + 32).
+            }
+            // P^T -> TMEM score columns [0, 64) as the A operand of dV += P^T dO.
+            ptx::tmem_st32(lane_base + Cfg::kColS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+            ptx::tmem_st32(lane_base + Cfg::kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_p_ready);
+            // ---- dS^T = P^T o (dP^T - D)   (Eq. 17) -> shared memory
+            if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t ud[32];
+                ptx::tmem_ld32(lane_base + Cfg::kColDP + c0, ud);
+                ptx::tmem_wait_ld();
+                uint32_t dw[16];
+#pragma unroll
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 dv4 = *reinterpret_cast<const float4*>(&sDv[wq][b][c0 + c]);
+                    const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+                    for (int h = 0; h < 4; h += 2) {
+                        const uint32_t pw = pk[(c0 + c + h) >> 1];
+                        const float p0 = __uint_as_float(pw << 16);
+                        const float p1 = __uint_as_float(pw & 0xffff0000u);
+                        const float d0 = p0 * (__uint_as_float(ud[c + h]) - dq4[h]);
+                        const float d1 = p1 * (__uint_as_float(ud[c + h + 1]) - dq4[h + 1]);
+                        dw[(c + h) >> 1] = ptx::pack_bf16x2(d0, d1);
+                    }
+                }
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     uint4 w = make_uint4(dw[4 * k4], dw[4 * k4 + 1], dw[4 * k4 + 2], dw[4 * k4 + 3]);
                     *reinterpret_cast<uint4*>(sDS + kmajor_chunk_offset<GS>(r, c0 + 8 * k4)) = w;
                 }
             }
-            ptx::tmem_wait_st();
             ptx::fence_async_smem();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_pds_ready);
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
         }
         // ---------------- epilogue: dK, dV rows -> shared memory -> TMA store.
         if (ok) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
@@ -396,34 +469,56 @@ fa2_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else {
         // ------------------------------------------------ dQ warpgroup
+        // Drains each dQ tile from TMEM into registers (so the next dP^T MMA
+        // can reuse the columns), then adds it into the fp32 accumulator one
+        // box of columns at a time: rows are written to a swizzled staging box
+        // in shared memory and one thread issues a TMA reduce-add, which does
+        // the additions in L2 without occupying the SM's load/store path.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // query row inside tile i
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
-        for (int it = 0; it < n_q; ++it) {
-            const int q_row = (i_begin + it) * kTileRows + r;
-            if (!ptx::mbar_wait(&bar_dq_full, it & 1, &abort_flag, tmo)) break;
+        const bool issuer = threadIdx.x == 192;
+        constexpr int NB4 = G4::kNBoxK;
+        constexpr int kChunks = G4::kRowBK / 16;         // 16-byte chunks per staged row
+        bool ok = true;
+        for (int it = 0; it < n_q && ok; ++it) {
+            const int q_row0 = (i_begin + it) * kTileRows;
+            if (!ptx::mbar_wait(&bar_dq_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.N + q_row) * D;
+            uint32_t u[G::kNOut];
 #pragma unroll
-            for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
-                uint32_t u[16];
-                ptx::tmem_ld16(lane_base + Cfg::kColDQ + c0, u);
-                ptx::tmem_wait_ld();
-                if (q_row < p.N) {
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        if (c0 + 4 * k4 < D) {
-                            float4 v = make_float4(__uint_as_float(u[4 * k4]), __uint_as_float(u[4 * k4 + 1]),
-                                                   __uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3]));
-                            atomicAdd(reinterpret_cast<float4*>(dst + c0 + 4 * k4), v);
-                        }
-                    }
-                }
-            }
+            for (int c0 = 0; c0 < G::kNOut; c0 += 16)
+                ptx::tmem_ld16(lane_base + Cfg::kColDQ + c0, *reinterpret_cast<uint32_t(*)[16]>(u + c0));
+            ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_dq_free);
+#pragma unroll
+            for (int c = 0; c < NB4; ++c) {
+                const int round = it * NB4 + c;
+                if (round > 0 && !ptx::mbar_wait(&bar_stage_free, (round - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
+#pragma unroll
+                for (int k = 0; k < kChunks; ++k) {
+                    const int col = c * G4::kBoxK + 4 * k;
+                    if (col < D) {
+                        const int sw = ((r * G4::kRowBK) >> 7) & (kChunks - 1);
+                        *reinterpret_cast<uint4*>(sStage + r * G4::kRowBK + ((k ^ sw) * 16)) =
+                            make_uint4(u[col], u[col + 1], u[col + 2], u[col + 3]);
+                    }
+                }
+                ptx::fence_async_smem();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_stage_full);
+                if (issuer) {
+                    if (!ptx::mbar_wait(&bar_stage_full, round & 1, &abort_flag, tmo)) { ok = false; break; }
+                    ptx::tma_reduce_add_3d(&tm_dq, sStage, c * G4::kBoxK, q_row0, bh);
+                    ptx::tma_store_commit();
+                    ptx::tma_store_wait_read_all();
+                    ptx::mbar_arrive(&bar_stage_free);
+                }
+            }
         }
+        if (issuer) ptx::tma_store_wait_all();
     }
 
     ptx::tc_fence_before();

@@ -4,9 +4,8 @@ fp64 oracle on identical seeded inputs.
 Small shapes are compared in full (all of O, L, dQ, dK, dV), spanning several
 128-row tiles, ragged tails, N < one tile, every supported head dim, causal
 and full attention.  The named workloads (the model-table head shapes) run at
-full size in the launch configuration the benchmark uses and are compared on
-two sampled heads: O and L in full for those heads, dQ / dK / dV on seeded
-sampled rows.
+full size in the launch configuration the benchmark uses; their first and
+last heads are compared in full.
 
 Tolerance per element: |gpu - ref| <= atol + rtol |ref| with atol = rtol =
 1e-2 for bf16 inputs and 2e-3 for fp32 (TF32 tensor-core) inputs.
@@ -85,23 +84,20 @@ BF16_WORKLOADS = [w for w in fa2_inputs.WORKLOADS.values() if w.dtype == "bf16"]
 
 
 @pytest.mark.parametrize("w", BF16_WORKLOADS, ids=[w.name for w in BF16_WORKLOADS])
-def test_workload_sampled_parity(oracle_mod, w):
-    """Full-size workload on the GPU; two heads checked against the oracle."""
+def test_workload_full_heads_parity(oracle_mod, w):
+    """Full-size workload on the GPU (the benchmark's launch configuration);
+    the first and the last head are compared element by element (all rows of
+    O, L, dQ, dK, dV) with the oracle."""
     inp = fa2_inputs.workload_inputs(w)
     got = gpu_fwd_bwd(inp, w.causal, w.scale)
     heads = sorted({0, w.heads - 1})
-    rows = fa2_inputs.sample_rows(w.N, 96, seed=w.seed + 1)
     for hh in heads:
         b, h = divmod(hh, w.H)
         q, k, v, do = (to64(inp[n][b, h].float()) for n in ("q", "k", "v", "do"))
         o, lse = oracle_mod.forward(q, k, v, w.causal, w.scale)
-        assert_close(to64(got["o"][b, h]), o, w.dtype, f"o[{hh}]")
-        assert_close(to64(got["lse"][b, h]), lse, w.dtype, f"lse[{hh}]")
-        res = oracle_mod.head_sampled(q, k, v, do, w.causal, w.scale, rows, rows,
-                                      want_forward=False)
-        assert_close(to64(got["dq"][b, h])[rows], res["dq"], w.dtype, f"dq[{hh}]")
-        assert_close(to64(got["dk"][b, h])[rows], res["dk"], w.dtype, f"dk[{hh}]")
-        assert_close(to64(got["dv"][b, h])[rows], res["dv"], w.dtype, f"dv[{hh}]")
+        dq, dk, dv = oracle_mod.backward(q, k, v, do, w.causal, w.scale)
+        for name, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            assert_close(to64(got[name][b, h]), ref, w.dtype, f"{name}[head {hh}]")
 
 
 def test_fp32_workload_forward_full(oracle_mod):
