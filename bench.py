@@ -39,9 +39,12 @@ UNIT = "TFLOP/s"
 SPEC_BF16_TFLOPS = 2250.0      # dense bf16 tensor peak of a B200 (spec sheet)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes per launch of the main backward kernel from an ncu capture of
-# the same kernel build (None until one has been taken for this build).
-BWD_MAIN_TRAFFIC_BYTES = 893907456  # profiles/fa2_bwd_kernel_d128_10b.md
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each
+# kernel from an ncu capture of the same kernel build; None until one has
+# been taken for the current build.
+FWD_TRAFFIC_BYTES = None
+DKDV_TRAFFIC_BYTES = None
+DQ_TRAFFIC_BYTES = None
 
 
 def causal_pairs(w) -> float:
@@ -281,8 +284,8 @@ def main():
     t_fwd = [e[0].elapsed_time(e[1]) for e in evs]          # forward kernel
     t_bwd = [e[1].elapsed_time(e[4]) for e in evs]          # whole backward call
     t_pre = [e[1].elapsed_time(e[2]) for e in evs]
-    t_main = [e[2].elapsed_time(e[3]) for e in evs]         # main backward kernel
-    t_fin = [e[3].elapsed_time(e[4]) for e in evs]
+    t_dkdv = [e[2].elapsed_time(e[3]) for e in evs]         # dK/dV pass kernel
+    t_dq = [e[3].elapsed_time(e[4]) for e in evs]           # dQ pass kernel
     t_step = [a + b for a, b in zip(t_fwd, t_bwd)]
     total_ms = sum(t_step)
     fwd_ms, bwd_ms = sum(t_fwd), sum(t_bwd)
@@ -333,14 +336,17 @@ def main():
         fwd_tf = world * f_fwd * K / (fwd_ms * 1e-3) / 1e12
         bwd_tf = world * f_bwd * K / (bwd_ms * 1e-3) / 1e12
         avg_fwd = sum(t_fwd) / K
-        avg_main = sum(t_main) / K
-        # Dominant kernel: the one with the larger share of the step.
-        if avg_main >= avg_fwd:
-            kname, kflops, kms = f"fa2_bwd_kernel<bf16,d={w.d}>", f_bwd, avg_main
-            ktraffic = BWD_MAIN_TRAFFIC_BYTES
-        else:
-            kname, kflops, kms = f"fa2_fwd_kernel<bf16,d={w.d}>", f_fwd, avg_fwd
-            ktraffic = None
+        avg_dkdv = sum(t_dkdv) / K
+        avg_dq = sum(t_dq) / K
+        # Dominant kernel: the one with the largest share of the step.  Its
+        # algorithmic FLOPs: forward 4*d*P_c; dK/dV pass S, dP, dV, dK =
+        # 8*d*P_c; dQ pass dQ = 2*d*P_c (its recomputed S and dP are not
+        # algorithmic work).
+        pc4 = f_fwd / 4.0
+        cands = [(avg_fwd, f"fa2_fwd2_kernel<bf16,d={w.d}>", f_fwd, FWD_TRAFFIC_BYTES),
+                 (avg_dkdv, f"fa2_bwd_dkdv_kernel<bf16,d={w.d}>", 8 * pc4, DKDV_TRAFFIC_BYTES),
+                 (avg_dq, f"fa2_bwd_dq_kernel<bf16,d={w.d}>", 2 * pc4, DQ_TRAFFIC_BYTES)]
+        kms, kname, kflops, ktraffic = max(cands, key=lambda c: c[0])
         achieved = kflops / (kms * 1e-3) / 1e12
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -352,8 +358,8 @@ def main():
             "bwd_frac_of_spec_bf16": bwd_tf / world / SPEC_BF16_TFLOPS,
             "fwd_frac_of_measured_bf16": fwd_tf / world / peaks["bf16_tflops"],
             "bwd_frac_of_measured_bf16": bwd_tf / world / peaks["bf16_tflops"],
-            "ms": {"fwd": avg_fwd, "bwd_pre": sum(t_pre) / K, "bwd_main": avg_main,
-                   "bwd_dq_finalize": sum(t_fin) / K},
+            "ms": {"fwd": avg_fwd, "bwd_pre": sum(t_pre) / K, "bwd_dkdv": avg_dkdv,
+                   "bwd_dq": avg_dq},
             "e2e": {"value": world * (f_fwd + f_bwd) * K_e2e / (e2e_ms * 1e-3) / 1e12,
                     "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": K_e2e},

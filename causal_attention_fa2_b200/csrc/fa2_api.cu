@@ -87,13 +87,13 @@ fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2
 // 3-D view [BH][N][d] of a contiguous [B,H,N,d] tensor, loaded/stored in boxes
 // of box_cols x 128 rows x 1 head.
 fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int N, int BH,
-                    int box_cols, int row_bytes, bool mn_major_f32) {
+                    int box_cols, int row_bytes, bool mn_major_f32, int box_rows = kTileRows) {
     const int es = dtype == FA2_BF16 ? 2 : 4;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es,
                              static_cast<cuuint64_t>(d) * es * static_cast<cuuint64_t>(N)};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kTileRows), 1};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUtensorMapSwizzle sw = mn_major_f32       ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                             : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
@@ -195,36 +195,32 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
                              uint32_t* status, unsigned long long timeout_ns,
                              void* const* events) {
     using T = typename std::conditional<ES == 2, __nv_bfloat16, float>::type;
+    using Cfg = BwdCfg<ES, D>;
     auto mark = [&](int i) -> bool {
         if (!events || !events[i]) return true;
         return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
     };
-    using Cfg = BwdCfg<ES, D>;
     const int BH = B * H;
     float* l2 = reinterpret_cast<float*>(ws_base + ws.l2_off);
     float* dvec = reinterpret_cast<float*>(ws_base + ws.d_off);
-    float* dq_acc = reinterpret_cast<float*>(ws_base + ws.dq_off);
     fa2_status st;
-    // 1. D, log2-scaled L, zeroed dQ accumulator.
+    // 1. D and log2-scaled L.
     const long long rows = static_cast<long long>(BH) * ws.n_pad;
     if (!mark(0)) return FA2_ERR_CUDA;
     fa2_bwd_pre_kernel<T, D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
-        static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, dq_acc, N, ws.n_pad,
-        rows);
+        static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
-    // 2. Main key/value-tile-outer pass.
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
-    if ((st = make_maps_kmajor<4, D>(&mdq, dq_acc, FA2_FP32, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mv, v, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdo, dout, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdk, dk, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdv, dv, dtype, N, BH)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdq, dq, dtype, N, BH)) != FA2_OK) return st;
     BwdParams p;
     p.l2 = l2;
     p.dvec = dvec;
-    p.dq_acc = dq_acc;
     p.status = status;
     p.N = N;
     p.BH = BH;
@@ -234,16 +230,22 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
-    auto kern = fa2_bwd_kernel<ES, D>;
-    if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-    kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, mdq, p);
-    if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
-    // 3. dQ = scale * accumulator.
-    const long long n4 = static_cast<long long>(BH) * N * D / 4;
-    fa2_bwd_dq_kernel<T><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, stream>>>(
-        dq_acc, static_cast<T*>(dq), scale, n4);
-    return (cudaGetLastError() == cudaSuccess && mark(3)) ? FA2_OK : FA2_ERR_CUDA;
+    // 2. dK, dV: key/value-tile-outer pass.
+    {
+        auto kern = fa2_bwd_dkdv_kernel<ES, D>;
+        if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
+    }
+    // 3. dQ: query-tile-outer pass.
+    {
+        auto kern = fa2_bwd_dq_kernel<ES, D>;
+        if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
+    }
+    return FA2_OK;
 }
 
 fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,

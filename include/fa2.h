@@ -89,24 +89,26 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
                        fa2_dtype dtype, fa2_stream_t stream);
 
 /*
- * Bytes of device workspace fa2_backward needs for these sizes (fp32 D and
- * log2-scaled L vectors plus an fp32 dQ accumulator).  Returns 0 for
- * arguments fa2_backward would reject.
+ * Bytes of device workspace fa2_backward needs for these sizes: the fp32 D
+ * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes
+ * (each rounded up to 256 bytes).  Returns 0 for arguments fa2_backward
+ * would reject.
  */
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype);
 
 /*
  * Backward pass with recomputation (handout section 4.2.2, Eqs. 13-19;
- * D = rowsum(O o dO)), key/value-tile outer loop, dQ accumulated in fp32.
+ * D = rowsum(O o dO)), organised as the handout's Algorithm 2 (section
+ * 4.2.3): one pass over key/value tiles accumulates dK and dV, a second pass
+ * over query tiles recomputes P and accumulates dQ, so nothing is added
+ * across thread blocks.
  *   q, k, v, o, dout  in : [B, H, N, d] `dtype` (o as produced by fa2_forward)
  *   lse               in : [B, H, N] float32 from fa2_forward
  *   dq, dk, dv        out: [B, H, N, d] `dtype`
  *   workspace         scratch of at least fa2_backward_workspace_bytes bytes,
  *                     256-byte aligned, owned by the caller; its contents on
  *                     entry do not matter and on return are unspecified
- * The result of dQ depends on the order of fp32 additions across thread
- * blocks, so it may differ in the last bits from run to run; O, L, dK and dV
- * are deterministic.
+ * Every output is deterministic (bitwise equal from run to run).
  */
 fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
@@ -119,8 +121,7 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
  * handles created on the current device; any entry may be NULL) on `stream`
  * at the boundaries of the three kernels the backward enqueues:
  *   events[0] before the D / L pre-pass,   events[1] after it,
- *   events[2] after the key/value-tile main pass,
- *   events[3] after the dQ finalisation.
+ *   events[2] after the dK / dV pass,      events[3] after the dQ pass.
  * `events` itself may be NULL (then this is fa2_backward).  The library only
  * records the events; the caller owns and destroys them.
  */
@@ -143,12 +144,12 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
  * workspace fa2_backward asks for.
  *
  * Arguments and results are those of fa2_backward without the workspace: the
- * scratch (D, log2-scaled L and the fp32 dQ accumulator) lives in a fixed
- * 64 MiB array that the library places in device memory of every GPU that
- * loads it, held until the process exits.  Problems whose workspace would
- * exceed it (fa2_backward_workspace_bytes(...) > 64 MiB, e.g. B*H*N*d above
- * about 16 million elements) are rejected with FA2_ERR_SCRATCH_TOO_SMALL
- * before anything is enqueued.  The call allocates nothing: no cudaMalloc,
+ * scratch (the fp32 D and log2-scaled L vectors) lives in a fixed 64 MiB
+ * array that the library places in device memory of every GPU that loads it,
+ * held until the process exits.  Problems whose workspace would exceed it
+ * (fa2_backward_workspace_bytes(...) > 64 MiB, i.e. B*H*ceil(N/128)*128 above
+ * about 8.3 million rows) are rejected with FA2_ERR_SCRATCH_TOO_SMALL before
+ * anything is enqueued.  The call allocates nothing: no cudaMalloc,
  * cudaFree, or allocating library routine.
  *
  * The first call on each device looks up the array's device address

@@ -94,12 +94,12 @@ def test_backward_validation(fa2lib):
 
 @pytest.mark.parametrize("B,H,N,d", [(1, 1, 1, 16), (2, 3, 200, 80), (1, 36, 4096, 128)])
 def test_workspace_size(fa2lib, B, H, N, d):
-    """D and log2-scaled L (fp32, padded to whole 128-row tiles) and an fp32
-    dQ accumulator, each region rounded up to 256 bytes."""
+    """D and log2-scaled L (fp32, padded to whole 128-row tiles), each region
+    rounded up to 256 bytes."""
     def up(x):
         return (x + 255) // 256 * 256
     n_pad = (N + 127) // 128 * 128
-    expect = 2 * up(B * H * n_pad * 4) + up(B * H * N * d * 4)
+    expect = 2 * up(B * H * n_pad * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, 24, 0) == 0
 

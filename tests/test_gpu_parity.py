@@ -139,7 +139,7 @@ def test_outputs_stay_in_bounds():
         assert torch.isfinite(t.float()).all()
 
 
-def test_forward_and_dkdv_deterministic():
+def test_forward_and_backward_deterministic():
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
     inp = fa2_inputs.make_inputs(2, 4, 640, 128, "bf16", seed=9)
@@ -149,7 +149,7 @@ def test_forward_and_dkdv_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
     g1 = fa2.backward(q, k, v, o1, l1, do)
     g2 = fa2.backward(q, k, v, o1, l1, do)
-    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    assert all(torch.equal(a, b) for a, b in zip(g1, g2))
     torch.cuda.synchronize()
 
 
@@ -164,8 +164,7 @@ def test_autograd_function_matches_direct_calls():
     o_ref, lse = fa2.forward(q.detach(), k.detach(), v.detach(), causal=True)
     dq, dk, dv = fa2.backward(q.detach(), k.detach(), v.detach(), o_ref, lse, do, causal=True)
     assert torch.equal(o.detach(), o_ref)
-    assert torch.equal(k.grad, dk) and torch.equal(v.grad, dv)
-    torch.testing.assert_close(q.grad.float(), dq.float(), atol=1e-2, rtol=1e-2)
+    assert torch.equal(q.grad, dq) and torch.equal(k.grad, dk) and torch.equal(v.grad, dv)
 
 
 def test_device_status_clean():
