@@ -14,6 +14,7 @@
 
 #include "../../include/fa2.h"
 #include "fa2_bwd.cuh"
+#include "fa2_bwd32.cuh"
 #include "fa2_fwd.cuh"
 #include "fa2_fwd2.cuh"
 
@@ -128,12 +129,12 @@ fa2_status set_smem(Kernel k, int bytes) {
                : FA2_ERR_CUDA;
 }
 
-// The two-query-tile forward needs two Q tiles plus at least one K/V stage in
-// shared memory; fp32 (TF32) inputs at d = 128 do not fit and use the
-// one-tile kernel.
+// The two-query-tile forward serves 16-bit inputs.  fp32 (TF32) inputs use the
+// one-tile kernel, whose extra warp rounds every operand tile to TF32 in
+// shared memory (the rounding the backward pass's operand copies use too).
 template <int ES, int D>
 constexpr bool use_two_tile_forward() {
-    return Fwd2Cfg<ES, D>::kFits;
+    return ES == 2 && Fwd2Cfg<ES, D>::kFits;
 }
 
 template <int ES, int D>
@@ -248,14 +249,98 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     return FA2_OK;
 }
 
+// fp32 inputs: TF32 kernels whose streamed operands arrive in sub-tiles of
+// W rows and, where a contraction runs over rows, in a second (MN-major) copy.
+template <int D>
+fa2_status launch_backward32_t(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               int B, int H, int N, int causal, float scale, uint8_t* ws_base,
+                               const BwdWorkspace& ws, cudaStream_t stream, uint32_t* status,
+                               unsigned long long timeout_ns, void* const* events) {
+    using Cfg = Bwd32Cfg<D>;
+    using G = typename Cfg::G;
+    constexpr fa2_dtype dt = FA2_FP32;
+    auto mark = [&](int i) -> bool {
+        if (!events || !events[i]) return true;
+        return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
+    };
+    const int BH = B * H;
+    float* l2 = reinterpret_cast<float*>(ws_base + ws.l2_off);
+    float* dvec = reinterpret_cast<float*>(ws_base + ws.d_off);
+    fa2_status st;
+    const long long rows = static_cast<long long>(BH) * ws.n_pad;
+    if (!mark(0)) return FA2_ERR_CUDA;
+    // TF32-rounded copies of the operands; every tensor map below reads those.
+    float* qr = reinterpret_cast<float*>(ws_base + ws.q_off);
+    float* kr = reinterpret_cast<float*>(ws_base + ws.k_off);
+    float* vr = reinterpret_cast<float*>(ws_base + ws.v_off);
+    float* dor = reinterpret_cast<float*>(ws_base + ws.do_off);
+    fa2_bwd32_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+        static_cast<const float*>(o), static_cast<const float*>(dout), lse, qr, kr, vr, dor, l2,
+        dvec, N, ws.n_pad, rows);
+    if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
+    q = qr;
+    k = kr;
+    v = vr;
+    dout = dor;
+    auto kmap = [&](CUtensorMap* m, const void* ptr, int box_rows) {
+        return make_map(m, ptr, dt, D, N, BH, G::kBoxK, G::kRowBK, false, box_rows);
+    };
+    auto mnmap = [&](CUtensorMap* m, const void* ptr, int box_rows) {
+        return make_map(m, ptr, dt, D, N, BH, G::kBoxMN, G::kRowBMN, true, box_rows);
+    };
+    BwdParams p;
+    p.l2 = l2;
+    p.dvec = dvec;
+    p.status = status;
+    p.N = N;
+    p.BH = BH;
+    p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.n_pad = ws.n_pad;
+    p.causal = causal;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.scale = scale;
+    p.timeout_ns = timeout_ns;
+    const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
+    {
+        constexpr int W = Cfg::kWkv;
+        CUtensorMap mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv;
+        if ((st = kmap(&mqk, q, W)) != FA2_OK || (st = mnmap(&mqmn, q, W)) != FA2_OK ||
+            (st = kmap(&mk, k, kTileRows)) != FA2_OK || (st = kmap(&mv, v, kTileRows)) != FA2_OK ||
+            (st = kmap(&mdok, dout, W)) != FA2_OK || (st = mnmap(&mdomn, dout, W)) != FA2_OK ||
+            (st = kmap(&mdk, dk, kTileRows)) != FA2_OK || (st = kmap(&mdv, dv, kTileRows)) != FA2_OK)
+            return st;
+        auto kern = fa2_bwd32_dkdv_kernel<D>;
+        if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemKV, stream>>>(mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
+    }
+    {
+        constexpr int W = Cfg::kWq;
+        CUtensorMap mq, mdo, mkk, mkmn, mvk, mdq;
+        if ((st = kmap(&mq, q, kTileRows)) != FA2_OK || (st = kmap(&mdo, dout, kTileRows)) != FA2_OK ||
+            (st = kmap(&mkk, k, W)) != FA2_OK || (st = mnmap(&mkmn, k, W)) != FA2_OK ||
+            (st = kmap(&mvk, v, W)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows)) != FA2_OK)
+            return st;
+        auto kern = fa2_bwd32_dq_kernel<D>;
+        if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemQ, stream>>>(mq, mdo, mkk, mkmn, mvk, mdq, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
+    }
+    return FA2_OK;
+}
+
 fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                            int H, int N, int d, int causal, float scale, fa2_dtype dtype,
                            uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                            uint32_t* status, unsigned long long timeout_ns, void* const* events) {
-    if (dtype != FA2_BF16) return FA2_ERR_UNSUPPORTED_DTYPE;
 #define FA2_BWD_CASE(DD)                                                                      \
     case DD:                                                                                  \
+        if (dtype == FA2_FP32)                                                                \
+            return launch_backward32_t<DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal, \
+                                           scale, ws_base, ws, stream, status, timeout_ns, events); \
         return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal,   \
                                         scale, dtype, ws_base, ws, stream, status, timeout_ns, events);
     switch (d) {
@@ -296,7 +381,7 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
 
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype) {
     if (check_common(B, H, N, d, 0, 1.f, dtype) != FA2_OK) return 0;
-    return bwd_workspace_layout(B * H, N, d).total;
+    return bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2).total;
 }
 
 fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const void* o,
@@ -312,7 +397,7 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4) || !aligned(workspace, 256))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d);
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
     if (workspace_bytes < ws.total) return FA2_ERR_WORKSPACE_TOO_SMALL;
     int dev;
     uint32_t* status;
@@ -416,7 +501,7 @@ extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const v
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d);
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
     if (ws.total > kNoAllocScratchBytes) return FA2_ERR_SCRATCH_TOO_SMALL;
     int dev;
     uint32_t* status;

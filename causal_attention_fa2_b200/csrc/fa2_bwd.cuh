@@ -38,21 +38,31 @@
 namespace fa2 {
 
 // Workspace carved out of the caller's buffer (every region 256-byte aligned):
-// L*log2(e) and D, fp32, [BH][n_pad].
+// L*log2(e) and D, fp32, [BH][n_pad]; for 4-byte inputs also copies of q, k,
+// v and dout rounded to TF32, [BH][N][d] each (offsets 0 when absent).
 struct BwdWorkspace {
-    size_t l2_off, d_off, total;
+    size_t l2_off, d_off, q_off, k_off, v_off, do_off, total;
     int n_pad;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-inline BwdWorkspace bwd_workspace_layout(int BH, int N, int /*d*/) {
+inline BwdWorkspace bwd_workspace_layout(int BH, int N, int d, int elem_bytes) {
     BwdWorkspace w;
     w.n_pad = (N + kTileRows - 1) / kTileRows * kTileRows;
     const size_t vec = align256(static_cast<size_t>(BH) * w.n_pad * sizeof(float));
     w.l2_off = 0;
     w.d_off = vec;
     w.total = 2 * vec;
+    w.q_off = w.k_off = w.v_off = w.do_off = 0;
+    if (elem_bytes == 4) {
+        const size_t t = align256(static_cast<size_t>(BH) * N * d * sizeof(float));
+        w.q_off = w.total;
+        w.k_off = w.q_off + t;
+        w.v_off = w.k_off + t;
+        w.do_off = w.v_off + t;
+        w.total = w.do_off + t;
+    }
     return w;
 }
 

@@ -1,0 +1,666 @@
+// fa2_bwd32.cuh -- the FlashAttention-2 backward pass for fp32 inputs, on
+// TF32 tensor cores (tcgen05.mma kind::tf32), for sm_100a.
+//
+// Same equations (CS336 A2 Systems handout section 4.2.2, Eqs. 13-19) and the
+// same two-pass organisation as the 16-bit kernels in fa2_bwd.cuh: a pass that
+// owns a key/value tile and accumulates its dK and dV, then a pass that owns a
+// query tile and accumulates its dQ (the handout's Algorithm 2, section
+// 4.2.3), after a pre-processing kernel of its own.  Three things differ with
+// 4-byte elements:
+//
+//  * A TF32 operand contracted over tile rows (dO and Q in the dK/dV pass, K
+//    in the dQ pass) must sit in shared memory with the 128-byte swizzle of
+//    32-byte atoms, which the contraction over d cannot read.  Those operands
+//    are staged twice, once per layout (two TMA copies of the same rows).
+//  * A 128-row tile is up to 64 KB, so the streamed operand arrives in
+//    sub-tiles of W rows: the largest W in {128, 64, 32, 16} that leaves room
+//    for two pipeline stages beside the two resident 128-row tiles.
+//  * P and dS stay fp32 in tensor memory, one column per element, written over
+//    the scores they came from; the next MMA reads them there as TF32.
+//
+// Every TF32 operand is rounded to nearest before the tensor core sees it: the
+// pre-processing kernel writes rounded copies of q, k, v and dout into the
+// workspace (the kernels' TMA loads read those), and P and dS are rounded as
+// they are written to tensor memory.  The tensor core itself would drop the 13
+// low bits of an fp32 operand, a biased error that puts a few gradient
+// elements past the 2e-3 tolerance.  D = rowsum(O o dO) is formed from the
+// rounded dO, the dO every dP entry is computed from, so that D_i stays equal
+// to sum_j P_ij dP_ij as the kernels compute them.
+//
+// Both kernels use 6 warps: 0 TMA producer, 1 MMA issuer (one thread), 2-5
+// one elementwise warpgroup.  The thread holding TMEM lane t owns row t of the
+// CTA's 128-row tile and all W columns of the current sub-tile.
+#pragma once
+
+#include <cstdint>
+
+#include "fa2_bwd.cuh"
+
+namespace fa2 {
+
+template <int D>
+struct Bwd32Cfg {
+    using G = TileGeom<4, D>;
+    static constexpr int kThreads = 192;
+    // 227 KB minus the 1024-byte alignment pad and the static shared memory.
+    static constexpr int kBudget = 227 * 1024 - 1024 - 1024;
+    __host__ __device__ static constexpr int tile_k(int rows) { return G::kNBoxK * rows * G::kRowBK; }
+    __host__ __device__ static constexpr int tile_mn(int rows) { return G::kNBoxMN * rows * G::kRowBMN; }
+    static constexpr int kResident = 2 * tile_k(kTileRows);
+    __host__ __device__ static constexpr int stages_for(int stage_bytes) {
+        const int s = (kBudget - kResident) / stage_bytes;
+        return s > 4 ? 4 : s;
+    }
+    // dK/dV pass, per stage: W query rows of Q and of dO, each K-major and MN-major.
+    __host__ __device__ static constexpr int kv_stage(int w) { return 2 * tile_k(w) + 2 * tile_mn(w); }
+    // dQ pass, per stage: W key rows of K (K-major and MN-major) and of V (K-major).
+    __host__ __device__ static constexpr int q_stage(int w) { return 2 * tile_k(w) + tile_mn(w); }
+    __host__ __device__ static constexpr int pick_kv() {
+        for (int w = kTileRows; w > 16; w /= 2)
+            if (stages_for(kv_stage(w)) >= 2) return w;
+        return 16;
+    }
+    __host__ __device__ static constexpr int pick_q() {
+        for (int w = kTileRows; w > 16; w /= 2)
+            if (stages_for(q_stage(w)) >= 2) return w;
+        return 16;
+    }
+    static constexpr int kWkv = pick_kv();
+    static constexpr int kStKV = stages_for(kv_stage(kWkv));
+    static constexpr int kWq = pick_q();
+    static constexpr int kStQ = stages_for(q_stage(kWq));
+    static_assert(kStKV >= 2 && kStQ >= 2, "shared memory too small for two pipeline stages");
+    static constexpr int kSmemKV = 1024 + kResident + kStKV * kv_stage(kWkv);
+    static constexpr int kSmemQ = 1024 + kResident + kStQ * q_stage(kWq);
+    static constexpr uint32_t kTmemCols = 512;
+    // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
+    static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
+};
+
+// ------------------------------------------------------------------ pre-processing
+
+// One warp per query row (8 rows per block): TF32-rounded copies of the q, k,
+// v and dout rows, D_i = sum_t round(dO_it) O_it, and L_i * log2(e); rows past
+// N (up to the padded length) get D = 0 and L = +inf.
+template <int D>
+__global__ void __launch_bounds__(256)
+fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                     const float* __restrict__ v, const float* __restrict__ o,
+                     const float* __restrict__ dout, const float* __restrict__ lse,
+                     float* __restrict__ qr, float* __restrict__ kr, float* __restrict__ vr,
+                     float* __restrict__ dor, float* __restrict__ l2, float* __restrict__ dvec,
+                     int N, int n_pad, long long rows_total) {
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows_total) return;
+    const long long bh = row / n_pad;
+    const int n = static_cast<int>(row - bh * n_pad);
+    if (n >= N) {
+        if (lane == 0) {
+            l2[row] = INFINITY;
+            dvec[row] = 0.f;
+        }
+        return;
+    }
+    const size_t base = (static_cast<size_t>(bh) * N + n) * D;
+    float acc = 0.f;
+    for (int e = lane; e < D; e += 32) {
+        const float g = __uint_as_float(ptx::to_tf32_rna(dout[base + e]));
+        dor[base + e] = g;
+        qr[base + e] = __uint_as_float(ptx::to_tf32_rna(q[base + e]));
+        kr[base + e] = __uint_as_float(ptx::to_tf32_rna(k[base + e]));
+        vr[base + e] = __uint_as_float(ptx::to_tf32_rna(v[base + e]));
+        acc += o[base + e] * g;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) {
+        dvec[row] = acc;
+        l2[row] = lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f;
+    }
+}
+
+// W consecutive TMEM columns of this warp's 32 lanes, one 32-bit word each.
+template <int W>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&u)[W]) {
+    if constexpr (W == 16) {
+        ptx::tmem_ld16(taddr, u);
+    } else {
+#pragma unroll
+        for (int c = 0; c < W; c += 32)
+            ptx::tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
+    }
+}
+
+template <int W>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&u)[W]) {
+    if constexpr (W == 16) {
+        ptx::tmem_st16(taddr, u);
+    } else {
+#pragma unroll
+        for (int c = 0; c < W; c += 32)
+            ptx::tmem_st32(taddr + c, *reinterpret_cast<const uint32_t(*)[32]>(u + c));
+    }
+}
+
+// P (fp32 bit patterns in `pu`) rounded to TF32 -> W TMEM columns at `col`;
+// `pu` keeps the unrounded values for dS.
+template <int W>
+__device__ __forceinline__ void bwd32_store_p(uint32_t col, const uint32_t (&pu)[W]) {
+    constexpr int C = W < 32 ? W : 32;
+#pragma unroll
+    for (int c0 = 0; c0 < W; c0 += C) {
+        uint32_t u[C];
+#pragma unroll
+        for (int c = 0; c < C; ++c) u[c] = ptx::to_tf32_rna(__uint_as_float(pu[c0 + c]));
+        tmem_st_cols<C>(col + c0, u);
+    }
+}
+
+// dS = P o (dP - D) over W columns held in TMEM at `dp_col`, rounded to TF32
+// and written back in place; P (fp32 bit patterns) is in `pu`, D per column or
+// per row from `dval`.
+template <int W, class DOf>
+__device__ __forceinline__ void bwd32_ds_inplace(uint32_t dp_col, const uint32_t (&pu)[W], DOf dval) {
+    constexpr int C = W < 32 ? W : 32;
+#pragma unroll
+    for (int c0 = 0; c0 < W; c0 += C) {
+        uint32_t u[C];
+        tmem_ld_cols<C>(dp_col + c0, u);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+            u[c] = ptx::to_tf32_rna(__uint_as_float(pu[c0 + c]) * (__uint_as_float(u[c]) - dval(c0 + c)));
+        tmem_st_cols<C>(dp_col + c0, u);
+    }
+    ptx::tmem_wait_st();
+}
+
+// 128 x D fp32 accumulator in TMEM (this thread's row r) times `mul` -> the
+// K-major staging layout of an fp32 tile in shared memory.
+template <class G>
+__device__ __forceinline__ void bwd32_stage_rows(uint32_t acc_col, int r, float mul, uint8_t* stage) {
+#pragma unroll
+    for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+        uint32_t u[16];
+        ptx::tmem_ld16(acc_col + c0, u);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const int col = c0 + 4 * q4;
+            if (col < G::kD) {
+                uint4 w;
+                w.x = __float_as_uint(__uint_as_float(u[4 * q4 + 0]) * mul);
+                w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * mul);
+                w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * mul);
+                w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * mul);
+                *reinterpret_cast<uint4*>(stage + kmajor_chunk_offset<G>(r, col)) = w;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ dK / dV pass
+
+// One CTA per (key tile j, head); K_j and V_j stay resident, the query rows
+// that see key tile j stream through in sub-tiles of W rows.  Per sub-tile
+// the MMA issuer runs S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q,
+// issuing the next sub-tile's S^T right after dV and its dP^T right after dK.
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_constant__ CUtensorMap tm_qmn,
+                      const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_dok, const __grid_constant__ CUtensorMap tm_domn,
+                      const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                      const BwdParams p) {
+    using Cfg = Bwd32Cfg<D>;
+    using G = typename Cfg::G;
+    constexpr int W = Cfg::kWkv;
+    constexpr int ST = Cfg::kStKV;
+    constexpr int TK = Cfg::tile_k(kTileRows);
+    constexpr int SK = Cfg::tile_k(W);
+    constexpr int SM = Cfg::tile_mn(W);
+    constexpr int SB = Cfg::kv_stage(W);
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar_kv_full, bar_full[ST], bar_empty[ST];
+    __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_dkv_full, bar_drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile uint32_t abort_flag;
+
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sK = smem;
+    uint8_t* sV = sK + TK;
+    uint8_t* sStage = sV + TK;
+    // Stage s: Q (K-major) | dO (K-major) | Q (MN-major) | dO (MN-major).
+    auto st_qk = [&](int s) { return sStage + s * SB; };
+    auto st_dok = [&](int s) { return sStage + s * SB + SK; };
+    auto st_qmn = [&](int s) { return sStage + s * SB + 2 * SK; };
+    auto st_domn = [&](int s) { return sStage + s * SB + 2 * SK + SM; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: with the causal mask, key tile j is seen by query rows >= 128 j,
+    // so small j carries the most work and is issued first.
+    const int item = blockIdx.x;
+    const int kv_tile = item / p.BH;
+    const int bh = item - kv_tile * p.BH;
+    const int kv_row0 = kv_tile * kTileRows;
+    const int n_sub = (p.N + W - 1) / W;
+    const int sub_begin = p.causal ? kv_row0 / W : 0;
+    const int n_q = n_sub - sub_begin;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        ptx::mbar_init(&bar_kv_full, 1);
+        for (int s = 0; s < ST; ++s) {
+            ptx::mbar_init(&bar_full[s], 1);
+            ptx::mbar_init(&bar_empty[s], 1);
+        }
+        ptx::mbar_init(&bar_s_full, 1);
+        ptx::mbar_init(&bar_dp_full, 1);
+        ptx::mbar_init(&bar_p_ready, 4);
+        ptx::mbar_init(&bar_ds_ready, 4);
+        ptx::mbar_init(&bar_dkv_full, 1);
+        ptx::mbar_init(&bar_drain, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_qk);
+            ptx::prefetch_tmap(&tm_qmn);
+            ptx::prefetch_tmap(&tm_dok);
+            ptx::prefetch_tmap(&tm_domn);
+            ptx::mbar_arrive_expect_tx(&bar_kv_full, 2 * TK);
+            for (int b = 0; b < G::kNBoxK; ++b) {
+                ptx::tma_load_3d(sK + b * kTileRows * G::kRowBK, &tm_k, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
+                ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
+            }
+            int issued = 0;
+            for (int it = 0; it < n_q; ++it) {
+                const int s = it % ST;
+                if (it >= ST && !ptx::mbar_wait(&bar_empty[s], ((it / ST) & 1) ^ 1, &abort_flag, tmo)) break;
+                const int row0 = (sub_begin + it) * W;
+                ptx::mbar_arrive_expect_tx(&bar_full[s], SB);
+                for (int b = 0; b < G::kNBoxK; ++b) {
+                    ptx::tma_load_3d(st_qk(s) + b * W * G::kRowBK, &tm_qk, &bar_full[s], b * G::kBoxK, row0, bh);
+                    ptx::tma_load_3d(st_dok(s) + b * W * G::kRowBK, &tm_dok, &bar_full[s], b * G::kBoxK, row0, bh);
+                }
+                for (int b = 0; b < G::kNBoxMN; ++b) {
+                    ptx::tma_load_3d(st_qmn(s) + b * W * G::kRowBMN, &tm_qmn, &bar_full[s], b * G::kBoxMN, row0, bh);
+                    ptx::tma_load_3d(st_domn(s) + b * W * G::kRowBMN, &tm_domn, &bar_full[s], b * G::kBoxMN, row0, bh);
+                }
+                issued = it + 1;
+            }
+            if (abort_flag) {
+                constexpr uint64_t kDrainNs = 20000000ull;
+                ptx::mbar_wait_drain(&bar_kv_full, 0, kDrainNs);
+                for (int t = issued - 1; t >= 0 && t >= issued - ST; --t)
+                    ptx::mbar_wait_drain(&bar_full[t % ST], (t / ST) & 1, kDrainNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, W, false, false);
+            constexpr uint32_t idesc_kv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
+            const uint32_t k_addr = ptx::smem_addr(sK);
+            const uint32_t v_addr = ptx::smem_addr(sV);
+            // S^T = K_j Q_i^T   (Eq. 13, transposed: rows are keys)
+            auto issue_s = [&](int it) -> bool {
+                const int s = it % ST;
+                if (!ptx::mbar_wait(&bar_full[s], (it / ST) & 1, &abort_flag, tmo)) return false;
+                ptx::tc_fence_after();
+                const uint32_t qa = ptx::smem_addr(st_qk(s));
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk)
+                    ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_s_full);
+                return true;
+            };
+            // dP^T = V_j dO_i^T   (Eq. 16, transposed); the stage is already full.
+            auto issue_dp = [&](int it) {
+                const uint32_t da = ptx::smem_addr(st_dok(it % ST));
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk)
+                    ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_dp_full);
+            };
+            bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
+            if (ok) ok = issue_s(0);
+            if (ok) issue_dp(0);
+            for (int it = 0; ok && it < n_q; ++it) {
+                const int s = it % ST;
+                // dV_j += P^T dO_i   (Eq. 15); P^T read from the score columns.
+                if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t dmn = ptx::smem_addr(st_domn(s));
+#pragma unroll
+                for (int kk = 0; kk < W / G::kKStep; ++kk)
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                if (it + 1 < n_q && !issue_s(it + 1)) { ok = false; break; }
+                // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
+                if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t qmn = ptx::smem_addr(st_qmn(s));
+#pragma unroll
+                for (int kk = 0; kk < W / G::kKStep; ++kk)
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(&bar_empty[s]);
+                if (it + 1 < n_q) issue_dp(it + 1);
+            }
+            if (ok) {
+                ptx::mma_commit(&bar_dkv_full);
+            } else {
+                ptx::mma_commit(&bar_drain);
+                ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+            }
+        }
+    } else {
+        // ------------------------------------------------ P / dS warpgroup
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;               // key row inside the tile
+        const bool key_valid = kv_row0 + r < p.N;
+        const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int it = 0; it < n_q; ++it) {
+            const int q0 = (sub_begin + it) * W;
+            const float* l2q = p.l2 + static_cast<size_t>(bh) * p.n_pad + q0;
+            const float* dvq = p.dvec + static_cast<size_t>(bh) * p.n_pad + q0;
+            // Some query of this sub-tile precedes some key of the tile.
+            const bool mask = p.causal && q0 < kv_row0 + kTileRows - 1;
+            // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14), in place
+            if (!ptx::mbar_wait(&bar_s_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+            uint32_t pu[W];
+            tmem_ld_cols<W>(lane_base + Cfg::kColS, pu);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < W; c += 4) {
+                const float4 lv = __ldg(reinterpret_cast<const float4*>(l2q + c));
+                const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    float pe = ptx::ex2_approx(fmaf(__uint_as_float(pu[c + h]), sl2, -lq[h]));
+                    if ((mask && q0 + c + h < kv_row0 + r) || !key_valid) pe = 0.f;
+                    pu[c + h] = __float_as_uint(pe);
+                }
+            }
+            bwd32_store_p<W>(lane_base + Cfg::kColS, pu);
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_p_ready);
+            // ---- dS^T = P^T o (dP^T - D)   (Eq. 17), in place over dP^T
+            if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+            bwd32_ds_inplace<W>(lane_base + Cfg::kColDP, pu, [&](int c) { return __ldg(dvq + c); });
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+        }
+        // ---------------- epilogue: dV -> sV, dK * scale -> sK, then TMA stores.
+        if (ok) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
+        if (ok) {
+            ptx::tc_fence_after();
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDV, r, 1.f, sV);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sK);
+            ptx::fence_async_smem();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && threadIdx.x == 64) {
+            for (int bx = 0; bx < G::kNBoxK; ++bx) {
+                ptx::tma_store_3d(&tm_dv, sV + bx * kTileRows * G::kRowBK, bx * G::kBoxK, kv_row0, bh);
+                ptx::tma_store_3d(&tm_dk, sK + bx * kTileRows * G::kRowBK, bx * G::kBoxK, kv_row0, bh);
+            }
+            ptx::tma_store_commit();
+            ptx::tma_store_wait_all();
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+    if (threadIdx.x == 0 && abort_flag) atomicCAS(p.status, 0u, kDevStatusTimeout);
+}
+
+// ------------------------------------------------------------------ dQ pass
+
+// One CTA per (query tile i, head); Q_i and dO_i stay resident, the key rows
+// query tile i sees stream through in sub-tiles of W rows.  Per sub-tile the
+// MMA issuer runs S = Q K^T, dP = dO V^T, dQ += dS K, issuing the next S as
+// soon as the warpgroup has read this one and the next dP right after dQ.
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_kk, const __grid_constant__ CUtensorMap tm_kmn,
+                    const __grid_constant__ CUtensorMap tm_vk, const __grid_constant__ CUtensorMap tm_dq,
+                    const BwdParams p) {
+    using Cfg = Bwd32Cfg<D>;
+    using G = typename Cfg::G;
+    constexpr int W = Cfg::kWq;
+    constexpr int ST = Cfg::kStQ;
+    constexpr int TK = Cfg::tile_k(kTileRows);
+    constexpr int SK = Cfg::tile_k(W);
+    constexpr int SB = Cfg::q_stage(W);
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bar_qdo_full, bar_full[ST], bar_empty[ST];
+    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready, bar_dq_done, bar_drain;
+    __shared__ uint32_t tmem_slot;
+    __shared__ volatile uint32_t abort_flag;
+
+    const uint32_t raw = ptx::smem_addr(smem_raw);
+    uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t* sQ = smem;
+    uint8_t* sDO = sQ + TK;
+    uint8_t* sStage = sDO + TK;
+    // Stage s: K (K-major) | V (K-major) | K (MN-major).
+    auto st_kk = [&](int s) { return sStage + s * SB; };
+    auto st_vk = [&](int s) { return sStage + s * SB + SK; };
+    auto st_kmn = [&](int s) { return sStage + s * SB + 2 * SK; };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Work item: causal query tile i sees keys < 128 (i + 1); longest first.
+    const int item = blockIdx.x;
+    const int rank = item / p.BH;
+    const int bh = item - rank * p.BH;
+    const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
+    const int q_row0 = q_tile * kTileRows;
+    const int n_sub = (p.N + W - 1) / W;
+    const int lim = (q_row0 + kTileRows) / W;
+    const int n_kv = p.causal ? (lim < n_sub ? lim : n_sub) : n_sub;
+
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        ptx::mbar_init(&bar_qdo_full, 1);
+        for (int s = 0; s < ST; ++s) {
+            ptx::mbar_init(&bar_full[s], 1);
+            ptx::mbar_init(&bar_empty[s], 1);
+        }
+        ptx::mbar_init(&bar_s_full, 1);
+        ptx::mbar_init(&bar_dp_full, 1);
+        ptx::mbar_init(&bar_s_read, 4);
+        ptx::mbar_init(&bar_ds_ready, 4);
+        ptx::mbar_init(&bar_dq_done, 1);
+        ptx::mbar_init(&bar_drain, 1);
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(&tmem_slot, Cfg::kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint64_t tmo = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::prefetch_tmap(&tm_kk);
+            ptx::prefetch_tmap(&tm_kmn);
+            ptx::prefetch_tmap(&tm_vk);
+            const uint64_t keep = ptx::policy_evict_last();
+            ptx::mbar_arrive_expect_tx(&bar_qdo_full, 2 * TK);
+            for (int b = 0; b < G::kNBoxK; ++b) {
+                ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
+                ptx::tma_load_3d(sDO + b * kTileRows * G::kRowBK, &tm_do, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
+            }
+            int issued = 0;
+            for (int j = 0; j < n_kv; ++j) {
+                const int s = j % ST;
+                if (j >= ST && !ptx::mbar_wait(&bar_empty[s], ((j / ST) & 1) ^ 1, &abort_flag, tmo)) break;
+                const int row0 = j * W;
+                ptx::mbar_arrive_expect_tx(&bar_full[s], SB);
+                for (int b = 0; b < G::kNBoxK; ++b) {
+                    ptx::tma_load_3d_hint(st_kk(s) + b * W * G::kRowBK, &tm_kk, &bar_full[s], b * G::kBoxK, row0, bh, keep);
+                    ptx::tma_load_3d_hint(st_vk(s) + b * W * G::kRowBK, &tm_vk, &bar_full[s], b * G::kBoxK, row0, bh, keep);
+                }
+                for (int b = 0; b < G::kNBoxMN; ++b)
+                    ptx::tma_load_3d_hint(st_kmn(s) + b * W * G::kRowBMN, &tm_kmn, &bar_full[s], b * G::kBoxMN, row0, bh, keep);
+                issued = j + 1;
+            }
+            if (abort_flag) {
+                constexpr uint64_t kDrainNs = 20000000ull;
+                ptx::mbar_wait_drain(&bar_qdo_full, 0, kDrainNs);
+                for (int t = issued - 1; t >= 0 && t >= issued - ST; --t)
+                    ptx::mbar_wait_drain(&bar_full[t % ST], (t / ST) & 1, kDrainNs);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, W, false, false);
+            constexpr uint32_t idesc_dq = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
+            const uint32_t q_addr = ptx::smem_addr(sQ);
+            const uint32_t do_addr = ptx::smem_addr(sDO);
+            // S = Q_i K_j^T   (Eq. 13)
+            auto issue_s = [&](int j) -> bool {
+                const int s = j % ST;
+                if (!ptx::mbar_wait(&bar_full[s], (j / ST) & 1, &abort_flag, tmo)) return false;
+                ptx::tc_fence_after();
+                const uint32_t ka = ptx::smem_addr(st_kk(s));
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk)
+                    ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_s_full);
+                return true;
+            };
+            // dP = dO_i V_j^T   (Eq. 16); the stage is already full.
+            auto issue_dp = [&](int j) {
+                const uint32_t va = ptx::smem_addr(st_vk(j % ST));
+#pragma unroll
+                for (int kk = 0; kk < G::kStepsD; ++kk)
+                    ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_dp_full);
+            };
+            bool ok = ptx::mbar_wait(&bar_qdo_full, 0, &abort_flag, tmo);
+            if (ok) ok = issue_s(0);
+            if (ok) issue_dp(0);
+            for (int j = 0; ok && j < n_kv; ++j) {
+                // Next scores as soon as the warpgroup has read S(j).
+                if (j + 1 < n_kv) {
+                    if (!ptx::mbar_wait(&bar_s_read, j & 1, &abort_flag, tmo)) { ok = false; break; }
+                    if (!issue_s(j + 1)) { ok = false; break; }
+                }
+                // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
+                if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t kmn = ptx::smem_addr(st_kmn(j % ST));
+#pragma unroll
+                for (int kk = 0; kk < W / G::kKStep; ++kk)
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * G::kKStep, desc_mnmajor<G>(kmn, kk, W), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(&bar_empty[j % ST]);
+                if (j + 1 < n_kv) issue_dp(j + 1);
+            }
+            if (ok) {
+                ptx::mma_commit(&bar_dq_done);
+            } else {
+                ptx::mma_commit(&bar_drain);
+                ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+            }
+        }
+    } else {
+        // ------------------------------------------------ P / dS warpgroup
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;               // query row inside the tile
+        const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
+        const float sl2 = p.scale_log2;
+        const size_t vrow = static_cast<size_t>(bh) * p.n_pad + q_row0 + r;
+        const float l2r = p.l2[vrow];                    // L_i * log2(e) (+inf past N)
+        const float dr = p.dvec[vrow];                   // D_i (0 past N)
+        bool ok = true;
+        for (int j = 0; j < n_kv; ++j) {
+            const int k0 = j * W;
+            const bool mask = p.causal && k0 + W - 1 > q_row0;   // some key follows some query
+            const int kv_valid = p.N - k0;                          // key columns < N
+            // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14), kept in registers
+            if (!ptx::mbar_wait(&bar_s_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+            uint32_t pu[W];
+            tmem_ld_cols<W>(lane_base + Cfg::kColS, pu);
+            ptx::tmem_wait_ld();
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_s_read);
+#pragma unroll
+            for (int c = 0; c < W; ++c) {
+                float pe = ptx::ex2_approx(fmaf(__uint_as_float(pu[c]), sl2, -l2r));
+                if ((mask && k0 + c > q_row0 + r) || c >= kv_valid) pe = 0.f;
+                pu[c] = __float_as_uint(pe);
+            }
+            // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
+            if (!ptx::mbar_wait(&bar_dp_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
+            ptx::tc_fence_after();
+            bwd32_ds_inplace<W>(lane_base + Cfg::kColDP, pu, [&](int) { return dr; });
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+        }
+        // ---------------- epilogue: dQ * scale -> sQ -> TMA store.
+        if (ok) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
+        if (ok) {
+            ptx::tc_fence_after();
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDQ, r, p.scale, sQ);
+            ptx::fence_async_smem();
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && threadIdx.x == 64) {
+            for (int bx = 0; bx < G::kNBoxK; ++bx)
+                ptx::tma_store_3d(&tm_dq, sQ + bx * kTileRows * G::kRowBK, bx * G::kBoxK, q_row0, bh);
+            ptx::tma_store_commit();
+            ptx::tma_store_wait_all();
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
+    }
+    if (threadIdx.x == 0 && abort_flag) atomicCAS(p.status, 0u, kDevStatusTimeout);
+}
+
+}  // namespace fa2

@@ -27,6 +27,13 @@
 //             row in TMEM when the running max grows.  After the last tile it
 //             normalises O, stages it in shared memory for a TMA store and
 //             writes L.
+//   warp 6    (fp32 inputs only) operand rounding: rounds every Q, K and V
+//             tile in shared memory to TF32 (round to nearest) once its TMA
+//             copy has landed and only then releases it to the MMA issuer, so
+//             the tensor core reads the operands exactly instead of dropping
+//             their 13 low bits (a biased error); the softmax group rounds P
+//             the same way.  The backward pass rounds its copies identically,
+//             so its recomputed scores equal these.
 // Scores are kept in log2 units (scale * log2(e) folded into one multiply)
 // so every exponential is a single ex2.  The running max used as the
 // exponent's reference is only raised when the row max grows by more than
@@ -54,7 +61,7 @@ struct FwdParams {
 template <int ES, int D>
 struct FwdCfg {
     using G = TileGeom<ES, D>;
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = G::kF32 ? 224 : 192;
     static constexpr int kBudget = 227 * 1024 - 2048;
     static constexpr int kFree = kBudget - G::kTileBytesK;
     // Ring depths for K and V (at most 4 each), as many as fit.
@@ -70,8 +77,24 @@ struct FwdCfg {
     static constexpr uint32_t kOCol = 256;
 };
 
+// Rounds `bytes` bytes of fp32 values in shared memory to TF32 in place (one
+// warp), then makes the writes visible to the tensor core's operand reads.
+__device__ __forceinline__ void round_tf32_smem(uint8_t* base, int bytes, int lane) {
+    float4* p4 = reinterpret_cast<float4*>(base);
+    for (int i = lane; i < bytes / 16; i += 32) {
+        float4 x = p4[i];
+        x.x = __uint_as_float(ptx::to_tf32_rna(x.x));
+        x.y = __uint_as_float(ptx::to_tf32_rna(x.y));
+        x.z = __uint_as_float(ptx::to_tf32_rna(x.z));
+        x.w = __uint_as_float(ptx::to_tf32_rna(x.w));
+        p4[i] = x;
+    }
+    ptx::fence_async_smem();
+    __syncwarp();
+}
+
 template <int ES, int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(FwdCfg<ES, D>::kThreads, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                const FwdParams p) {
@@ -85,8 +108,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint64_t bar_k_full[KST], bar_k_empty[KST];
     __shared__ uint64_t bar_v_full[VST], bar_v_empty[VST];
     __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done, bar_drain;
+    // fp32: tiles released by the rounding warp (the MMA issuer waits on these).
+    __shared__ uint64_t bar_q_ready, bar_k_ready[KST], bar_v_ready[VST];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    uint64_t* const q_go = G::kF32 ? &bar_q_ready : &bar_q_full;
+    uint64_t* const k_go = G::kF32 ? bar_k_ready : bar_k_full;
+    uint64_t* const v_go = G::kF32 ? bar_v_ready : bar_v_full;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -111,6 +139,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int s = 0; s < KST; ++s) { ptx::mbar_init(&bar_k_full[s], 1); ptx::mbar_init(&bar_k_empty[s], 1); }
         for (int s = 0; s < VST; ++s) { ptx::mbar_init(&bar_v_full[s], 1); ptx::mbar_init(&bar_v_empty[s], 1); }
         for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bar_s_full[b], 1); ptx::mbar_init(&bar_p_full[b], 4); }
+        ptx::mbar_init(&bar_q_ready, 1);
+        for (int s = 0; s < KST; ++s) ptx::mbar_init(&bar_k_ready[s], 1);
+        for (int s = 0; s < VST; ++s) ptx::mbar_init(&bar_v_ready[s], 1);
         ptx::mbar_init(&bar_o_done, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::fence_mbar_init();
@@ -167,11 +198,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr = ptx::smem_addr(sQ);
-            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            bool ok = ptx::mbar_wait(q_go, 0, &abort_flag, tmo);
             auto issue_pv = [&](int jj) -> bool {
                 if (!ptx::mbar_wait(&bar_p_full[jj & 1], (jj >> 1) & 1, &abort_flag, tmo)) return false;
                 const int vs = jj % VST;
-                if (!ptx::mbar_wait(&bar_v_full[vs], (jj / VST) & 1, &abort_flag, tmo)) return false;
+                if (!ptx::mbar_wait(&v_go[vs], (jj / VST) & 1, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
                 const uint32_t v_addr = ptx::smem_addr(sV + vs * G::kTileBytesMN);
                 const uint32_t p_tmem = tmem + (jj & 1) * 128;
@@ -189,7 +220,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             };
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int ks = j % KST;
-                if (!ptx::mbar_wait(&bar_k_full[ks], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                if (!ptx::mbar_wait(&k_go[ks], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t k_addr = ptx::smem_addr(sK + ks * G::kTileBytesK);
                 const uint32_t s_tmem = tmem + (j & 1) * 128;
@@ -213,7 +244,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
             }
         }
-    } else {
+    } else if (warp < 6) {
         // ------------------------------------------------ softmax warpgroup
         const int quarter = warp & 3;           // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;      // query row inside the tile
@@ -287,7 +318,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int c0 = 0; c0 < 128; c0 += 32) {
                     uint32_t u[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(s[c0 + c]);
+                    for (int c = 0; c < 32; ++c) u[c] = ptx::to_tf32_rna(s[c0 + c]);
                     ptx::tmem_st32(s_tmem + c0, u);
                 }
             } else {
@@ -354,6 +385,25 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ptx::tma_store_3d(&tm_o, sQ + b * kTileRows * G::kRowBK, b * G::kBoxK, q_row0, bh);
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
+        }
+    } else {
+        // ------------------------------------------------ TF32 rounding (fp32 only)
+        if constexpr (G::kF32) {
+            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            if (ok) {
+                round_tf32_smem(sQ, G::kTileBytesK, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int ks = j % KST;
+                if (!ptx::mbar_wait(&bar_k_full[ks], (j / KST) & 1, &abort_flag, tmo)) break;
+                round_tf32_smem(sK + ks * G::kTileBytesK, G::kTileBytesK, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_k_ready[ks]);
+                const int vs = j % VST;
+                if (!ptx::mbar_wait(&bar_v_full[vs], (j / VST) & 1, &abort_flag, tmo)) break;
+                round_tf32_smem(sV + vs * G::kTileBytesMN, G::kTileBytesMN, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs]);
+            }
         }
     }
 

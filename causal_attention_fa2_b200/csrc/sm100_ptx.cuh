@@ -392,6 +392,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// fp32 -> TF32 (10 explicit mantissa bits), rounded to nearest with ties away
+// from zero; returned as the fp32 bit pattern with its 13 low bits clear, so a
+// TF32 tensor-core operand holding it is read exactly.
+__device__ __forceinline__ uint32_t to_tf32_rna(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

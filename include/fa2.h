@@ -90,9 +90,10 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
 
 /*
  * Bytes of device workspace fa2_backward needs for these sizes: the fp32 D
- * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes
- * (each rounded up to 256 bytes).  Returns 0 for arguments fa2_backward
- * would reject.
+ * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes, and
+ * for FA2_FP32 also copies of q, k, v and dout rounded to TF32 (round to
+ * nearest), 4 * 4 * B * H * N * d bytes (every region rounded up to 256
+ * bytes).  Returns 0 for arguments fa2_backward would reject.
  */
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype);
 
@@ -144,12 +145,13 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
  * workspace fa2_backward asks for.
  *
  * Arguments and results are those of fa2_backward without the workspace: the
- * scratch (the fp32 D and log2-scaled L vectors) lives in a fixed 64 MiB
+ * scratch (the workspace fa2_backward_workspace_bytes sizes) lives in a fixed 64 MiB
  * array that the library places in device memory of every GPU that loads it,
  * held until the process exits.  Problems whose workspace would exceed it
- * (fa2_backward_workspace_bytes(...) > 64 MiB, i.e. B*H*ceil(N/128)*128 above
- * about 8.3 million rows) are rejected with FA2_ERR_SCRATCH_TOO_SMALL before
- * anything is enqueued.  The call allocates nothing: no cudaMalloc,
+ * (fa2_backward_workspace_bytes(...) > 64 MiB: for FA2_BF16, B*H*ceil(N/128)*128
+ * above about 8.3 million rows; for FA2_FP32, whose workspace also holds the
+ * rounded operand copies, B*H*N*d above about 4 million elements) are
+ * rejected with FA2_ERR_SCRATCH_TOO_SMALL before anything is enqueued.  The call allocates nothing: no cudaMalloc,
  * cudaFree, or allocating library routine.
  *
  * The first call on each device looks up the array's device address

@@ -95,12 +95,14 @@ def test_backward_validation(fa2lib):
 @pytest.mark.parametrize("B,H,N,d", [(1, 1, 1, 16), (2, 3, 200, 80), (1, 36, 4096, 128)])
 def test_workspace_size(fa2lib, B, H, N, d):
     """D and log2-scaled L (fp32, padded to whole 128-row tiles), each region
-    rounded up to 256 bytes."""
+    rounded up to 256 bytes; for fp32 inputs also four operand copies."""
     def up(x):
         return (x + 255) // 256 * 256
     n_pad = (N + 127) // 128 * 128
     expect = 2 * up(B * H * n_pad * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
+    # fp32 inputs: plus TF32-rounded copies of q, k, v and dout.
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 1) == expect + 4 * up(B * H * N * d * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, 24, 0) == 0
 
 

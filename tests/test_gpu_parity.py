@@ -57,12 +57,13 @@ def test_bf16_small_full_parity(oracle_mod, B, H, N, d, causal):
 
 @pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
 @pytest.mark.parametrize("B,H,N,d", SMALL)
-def test_fp32_small_forward_parity(oracle_mod, B, H, N, d, causal):
+def test_fp32_small_full_parity(oracle_mod, B, H, N, d, causal):
+    """fp32 inputs (TF32 tensor-core MMAs): forward and backward in full."""
     inp = fa2_inputs.make_inputs(B, H, N, d, "fp32", seed=17 + N + d)
     scale = default_scale(d)
-    got = gpu_fwd_bwd(inp, causal, scale, do_backward=False)
-    ref = _oracle(oracle_mod, inp, causal, scale, backward=False)
-    for name in ("o", "lse"):
+    got = gpu_fwd_bwd(inp, causal, scale)
+    ref = _oracle(oracle_mod, inp, causal, scale)
+    for name in ("o", "lse", "dq", "dk", "dv"):
         assert_close(to64(got[name]), ref[name], "fp32", name)
 
 
@@ -100,13 +101,14 @@ def test_workload_full_heads_parity(oracle_mod, w):
             assert_close(to64(got[name][b, h]), ref, w.dtype, f"{name}[head {hh}]")
 
 
-def test_fp32_workload_forward_full(oracle_mod):
+def test_fp32_workload_full(oracle_mod):
+    """The fp32 model-table workload (B=2, H=4, N=128, d=64), every output in full."""
     w = fa2_inputs.WORKLOADS["fp32-b2h4-n128-d64"]
     inp = fa2_inputs.workload_inputs(w)
-    got = gpu_fwd_bwd(inp, w.causal, w.scale, do_backward=False)
-    ref = _oracle(oracle_mod, inp, w.causal, w.scale, backward=False)
-    assert_close(to64(got["o"]), ref["o"], "fp32", "o")
-    assert_close(to64(got["lse"]), ref["lse"], "fp32", "lse")
+    got = gpu_fwd_bwd(inp, w.causal, w.scale)
+    ref = _oracle(oracle_mod, inp, w.causal, w.scale)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(to64(got[name]), ref[name], "fp32", name)
 
 
 def test_outputs_stay_in_bounds():
@@ -139,10 +141,11 @@ def test_outputs_stay_in_bounds():
         assert torch.isfinite(t.float()).all()
 
 
-def test_forward_and_backward_deterministic():
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_forward_and_backward_deterministic(dtype):
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
-    inp = fa2_inputs.make_inputs(2, 4, 640, 128, "bf16", seed=9)
+    inp = fa2_inputs.make_inputs(2, 4, 640, 128, dtype, seed=9)
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
     o1, l1 = fa2.forward(q, k, v)
     o2, l2 = fa2.forward(q, k, v)
