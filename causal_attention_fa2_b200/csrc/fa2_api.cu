@@ -208,7 +208,8 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     // 1. D and log2-scaled L.
     const long long rows = static_cast<long long>(BH) * ws.n_pad;
     if (!mark(0)) return FA2_ERR_CUDA;
-    fa2_bwd_pre_kernel<T, D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+    constexpr int kPreRows = BwdPreCfg<D>::kRowsPerBlock;
+    fa2_bwd_pre_kernel<D><<<static_cast<unsigned>((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
         static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;

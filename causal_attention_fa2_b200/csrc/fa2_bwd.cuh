@@ -31,6 +31,8 @@
 // memory on the hot path.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include <cstdint>
 
 #include "fa2_traits.cuh"
@@ -68,32 +70,53 @@ inline BwdWorkspace bwd_workspace_layout(int BH, int N, int d, int elem_bytes) {
 
 // ------------------------------------------------------------------ pre-processing
 
-template <typename T, int D>
+// Geometry of the pre-pass: a row of d 16-bit values is read as 16-byte
+// vectors by kTPR threads (d / 8 rounded up to a power of two), so one warp
+// covers 32 / kTPR rows and one 256-thread block 8 * 32 / kTPR rows.
+template <int D>
+struct BwdPreCfg {
+    static constexpr int kVec = 8;                                  // elements per 16-byte load
+    static constexpr int kUsed = (D + kVec - 1) / kVec;            // threads that load
+    static constexpr int kTPR = kUsed <= 2 ? 2 : kUsed <= 4 ? 4 : kUsed <= 8 ? 8 : 16;
+    static constexpr int kRowsPerBlock = 8 * 32 / kTPR;
+};
+
+// D_i = rowsum(O_i o dO_i) and L_i * log2(e) per query row; rows past N (up
+// to the padded length) get D = 0 and L = +inf so they drop out of P and dS.
+template <int D>
 __global__ void __launch_bounds__(256)
-fa2_bwd_pre_kernel(const T* __restrict__ o, const T* __restrict__ dout,
+fa2_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                    const float* __restrict__ lse, float* __restrict__ l2,
                    float* __restrict__ dvec, int N, int n_pad, long long rows_total) {
-    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows_total) return;
+    using C = BwdPreCfg<D>;
+    const int sub = threadIdx.x % C::kTPR;
+    const long long row = static_cast<long long>(blockIdx.x) * C::kRowsPerBlock + threadIdx.x / C::kTPR;
+    const bool live = row < rows_total;
     const long long bh = row / n_pad;
     const int n = static_cast<int>(row - bh * n_pad);
-    if (n >= N) {
-        if (lane == 0) {
-            l2[row] = INFINITY;
-            dvec[row] = 0.f;
-        }
-        return;
-    }
-    const size_t base = (static_cast<size_t>(bh) * N + n) * D;
     float acc = 0.f;
-    for (int e = lane; e < D; e += 32)
-        acc += static_cast<float>(o[base + e]) * static_cast<float>(dout[base + e]);
+    if (live && n < N && sub < C::kUsed) {
+        const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * C::kVec;
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + base));
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + base));
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
+        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-        dvec[row] = acc;
-        l2[row] = lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f;
+        for (int w = 0; w < 4; ++w) {
+            acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
+            acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(bw[w] & 0xffff0000u), acc);
+        }
+    }
+#pragma unroll
+    for (int off = C::kTPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (live && sub == 0) {
+        if (n < N) {
+            dvec[row] = acc;
+            l2[row] = lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f;
+        } else {
+            dvec[row] = 0.f;
+            l2[row] = INFINITY;
+        }
     }
 }
 
