@@ -1,14 +1,15 @@
 """Benchmark: causal FlashAttention-2 forward + backward on B200.
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-fa2_forward (O, L) then fa2_backward (D pre-pass, key/value-tile main pass,
-dQ finalisation), on the 10B-model head shape (B=1, H=36, N=4096, d=128,
-bf16, causal) unless --workload names another.
+fa2_forward (O, L) then fa2_backward (D / L pre-pass, dK/dV pass over key
+tiles, dQ pass over query tiles), on the 10B-model head shape (B=1, H=36,
+N=4096, d=128, bf16, causal) unless --workload names another.
 
 Metric: attention TFLOP/s with causal FLOPs counted (forward 4*d*P_c,
 backward 10*d*P_c, P_c = B*H*N(N+1)/2 unmasked query/key pairs).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa2|reference]
+    python bench.py --table      # per-workload / sweep-point timing table
 
 For N > 1 run under torchrun: each rank runs the same workload on its own
 seeded batch (heads are independent; no collective on the data path), and the
@@ -37,14 +38,16 @@ import fa2_inputs  # noqa: E402
 METRIC = "attention TFLOP/s (causal) fwd and fwd+bwd at 1 B200; % of bf16 tensor peak"
 UNIT = "TFLOP/s"
 SPEC_BF16_TFLOPS = 2250.0      # dense bf16 tensor peak of a B200 (spec sheet)
+SPEC_TF32_TFLOPS = 1100.0      # dense TF32 tensor peak (half the 2.2 PF sparse figure)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each
-# kernel from an ncu capture of the same kernel build; None until one has
-# been taken for the current build.
-FWD_TRAFFIC_BYTES = None
-DKDV_TRAFFIC_BYTES = None
-DQ_TRAFFIC_BYTES = None
+# bf16 d=128 kernel on the 10B head shape, from one ncu capture of the current
+# kernel build; None where no capture of the current build exists.
+FWD_TRAFFIC_BYTES = 211_474_688
+DKDV_TRAFFIC_BYTES = 311_743_488
+DQ_TRAFFIC_BYTES = 313_335_296
+TRAFFIC_WORKLOAD = "10b-b1h36-n4096-d128"
 
 
 def causal_pairs(w) -> float:
@@ -207,6 +210,78 @@ def config_of(w, n):
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
+# --------------------------------------------------------------------- table mode
+
+def alg_bytes(w):
+    """Algorithmic HBM bytes: forward reads Q, K, V and writes O and L; the
+    backward reads Q, K, V, O, dO, L and writes dQ, dK, dV (D and L*log2(e)
+    are workspace, counted as one write and one read each)."""
+    es = 2 if w.dtype == "bf16" else 4
+    t = w.B * w.H * w.N * w.d * es
+    rows = w.B * w.H * w.N * 4
+    return 4 * t + rows, 8 * t + 3 * rows
+
+
+def run_table(args):
+    """Times fa2_forward and fa2_backward on every model-table workload and a
+    selection of sweep points (CUDA events, L2 flushed before each call) and
+    prints one markdown table."""
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    meas = {"bf16": peaks["bf16_tflops"], "fp32": peaks["bf16_tflops"] * SPEC_TF32_TFLOPS / SPEC_BF16_TFLOPS}
+    spec = {"bf16": SPEC_BF16_TFLOPS, "fp32": SPEC_TF32_TFLOPS}
+    points = list(fa2_inputs.WORKLOADS.values())
+    points += [fa2_inputs.sweep_workload(N, d, dt) for dt in ("bf16", "fp32") for d in fa2_inputs.SWEEP_D
+               for N in (128, 512, 1024, 4096, 8192, 16384, 32768)]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    print(f"peaks: bf16 {meas['bf16']:.1f} TFLOP/s ({peak_src}); TF32 {meas['fp32']:.1f} "
+          f"(bf16 x 1100/2250); HBM {peaks['hbm_gbs']:.1f} GB/s")
+    print("| workload | dtype | fwd ms | fwd TFLOP/s | fwd % spec / % meas | fwd GB/s | bwd ms | "
+          "bwd TFLOP/s | bwd % spec / % meas | bwd GB/s |")
+    print("|---|---|---|---|---|---|---|---|---|---|")
+    for w in points:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(w.seed)
+        dt = fa2_inputs.DTYPES[w.dtype]
+        q, k, v, do = (torch.randn((w.B, w.H, w.N, w.d), generator=g).to(dt).to(dev) for _ in range(4))
+        o, lse = fa2.forward(q, k, v, causal=w.causal, scale=w.scale)
+        ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype), dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        f_fwd, f_bwd = flops(w)
+        b_fwd, b_bwd = alg_bytes(w)
+        reps = max(3, min(args.steps, 20))
+        tf, tb = [], []
+        for i in range(reps + 3):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record()
+            fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            e[1].record()
+            flush.zero_()
+            e2 = torch.cuda.Event(enable_timing=True)
+            e2.record()
+            fa2.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws,
+                         dq=dq, dk=dk, dv=dv)
+            e[2].record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                tf.append(e[0].elapsed_time(e[1]))
+                tb.append(e2.elapsed_time(e[2]))
+        mf, mb = sorted(tf)[len(tf) // 2], sorted(tb)[len(tb) // 2]
+        tff, tfb = f_fwd / mf / 1e9, f_bwd / mb / 1e9
+        print(f"| {w.name} | {w.dtype} | {mf:.4f} | {tff:.1f} | {100 * tff / spec[w.dtype]:.1f} / "
+              f"{100 * tff / meas[w.dtype]:.1f} | {b_fwd / mf / 1e6:.0f} | {mb:.4f} | {tfb:.1f} | "
+              f"{100 * tfb / spec[w.dtype]:.1f} / {100 * tfb / meas[w.dtype]:.1f} | {b_bwd / mb / 1e6:.0f} |",
+              flush=True)
+        del q, k, v, do, o, lse, ws, dq, dk, dv
+    status = fa2.last_device_status()
+    if status != 0:
+        raise SystemExit(f"device status after timing: {fa2.status_string(status)}")
+    return 0
+
+
 # --------------------------------------------------------------------- GPU arm
 
 def main():
@@ -217,7 +292,11 @@ def main():
     ap.add_argument("--impl", default="fa2", choices=["fa2", "reference"])
     ap.add_argument("--workload", default="10b-b1h36-n4096-d128")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--table", action="store_true",
+                    help="time every model-table workload and sweep point; print a table")
     args = ap.parse_args()
+    if args.table:
+        return run_table(args)
     w = fa2_inputs.WORKLOADS[args.workload]
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -343,9 +422,18 @@ def main():
         # 8*d*P_c; dQ pass dQ = 2*d*P_c (its recomputed S and dP are not
         # algorithmic work).
         pc4 = f_fwd / 4.0
-        cands = [(avg_fwd, f"fa2_fwd2_kernel<bf16,d={w.d}>", f_fwd, FWD_TRAFFIC_BYTES),
-                 (avg_dkdv, f"fa2_bwd_dkdv_kernel<bf16,d={w.d}>", 8 * pc4, DKDV_TRAFFIC_BYTES),
-                 (avg_dq, f"fa2_bwd_dq_kernel<bf16,d={w.d}>", 2 * pc4, DQ_TRAFFIC_BYTES)]
+        if w.dtype == "bf16":
+            names = (f"fa2_fwd2_kernel<bf16,d={w.d}>", f"fa2_bwd_dkdv_kernel<bf16,d={w.d}>",
+                     f"fa2_bwd_dq_kernel<bf16,d={w.d}>")
+            traffic = ((FWD_TRAFFIC_BYTES, DKDV_TRAFFIC_BYTES, DQ_TRAFFIC_BYTES)
+                       if w.name == TRAFFIC_WORKLOAD else (None, None, None))
+        else:
+            names = (f"fa2_fwd_kernel<fp32,d={w.d}>", f"fa2_bwd32_dkdv_kernel<d={w.d}>",
+                     f"fa2_bwd32_dq_kernel<d={w.d}>")
+            traffic = (None, None, None)
+        cands = [(avg_fwd, names[0], f_fwd, traffic[0]),
+                 (avg_dkdv, names[1], 8 * pc4, traffic[1]),
+                 (avg_dq, names[2], 2 * pc4, traffic[2])]
         kms, kname, kflops, ktraffic = max(cands, key=lambda c: c[0])
         achieved = kflops / (kms * 1e-3) / 1e12
         line = {

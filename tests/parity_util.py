@@ -15,7 +15,8 @@ def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, name: str):
+def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, name: str) -> float:
+    """Per-element tolerance check; returns the largest absolute error."""
     atol, rtol = TOL[dtype]
     assert got.shape == ref.shape, (name, got.shape, ref.shape)
     assert np.isfinite(got).all(), f"{name}: non-finite values in the CUDA result"
@@ -28,6 +29,7 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, name: str):
             f"{name}: {int(bad.sum())} of {err.size} elements out of tolerance "
             f"(atol={atol}, rtol={rtol}); worst at {idx}: got {got[idx]!r} ref {ref[idx]!r}; "
             f"max abs err {err.max():.3e}")
+    return float(err.max()) if err.size else 0.0
 
 
 def gpu_fwd_bwd(inp, causal: bool, scale: float, do_backward: bool = True):

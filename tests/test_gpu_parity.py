@@ -98,7 +98,8 @@ def test_workload_full_heads_parity(oracle_mod, w):
         o, lse = oracle_mod.forward(q, k, v, w.causal, w.scale)
         dq, dk, dv = oracle_mod.backward(q, k, v, do, w.causal, w.scale)
         for name, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-            assert_close(to64(got[name][b, h]), ref, w.dtype, f"{name}[head {hh}]")
+            e = assert_close(to64(got[name][b, h]), ref, w.dtype, f"{name}[head {hh}]")
+            print(f"ERR {w.name} head {hh} {name} max_abs {e:.3e}")
 
 
 def test_fp32_workload_full(oracle_mod):
@@ -108,7 +109,8 @@ def test_fp32_workload_full(oracle_mod):
     got = gpu_fwd_bwd(inp, w.causal, w.scale)
     ref = _oracle(oracle_mod, inp, w.causal, w.scale)
     for name in ("o", "lse", "dq", "dk", "dv"):
-        assert_close(to64(got[name]), ref[name], "fp32", name)
+        e = assert_close(to64(got[name]), ref[name], "fp32", name)
+        print(f"ERR {w.name} all heads {name} max_abs {e:.3e}")
 
 
 def test_outputs_stay_in_bounds():

@@ -32,7 +32,8 @@ def test_sweep_point_full(oracle_mod, N, d, dtype):
     o, lse = oracle_mod.forward(q, k, v, w.causal, w.scale)
     dq, dk, dv = oracle_mod.backward(q, k, v, do, w.causal, w.scale)
     for name, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-        assert_close(to64(got[name]), ref, dtype, name)
+        e = assert_close(to64(got[name]), ref, dtype, name)
+        print(f"ERR {w.name} all heads {name} max_abs {e:.3e}")
 
 
 @pytest.mark.parametrize("N,d,dtype", LONG_POINTS, ids=_ids(LONG_POINTS))
@@ -46,4 +47,5 @@ def test_sweep_point_sampled(oracle_mod, N, d, dtype):
         q, k, v, do = (to64(inp[n][0, h].float()) for n in ("q", "k", "v", "do"))
         ref = oracle_mod.head_sampled(q, k, v, do, w.causal, w.scale, rows, rows)
         for name in ("o", "lse", "dq", "dk", "dv"):
-            assert_close(to64(got[name][0, h][rows]), ref[name], dtype, f"{name}[head {h}]")
+            e = assert_close(to64(got[name][0, h][rows]), ref[name], dtype, f"{name}[head {h}]")
+            print(f"ERR {w.name} head {h} sampled {name} max_abs {e:.3e}")
