@@ -216,7 +216,7 @@ def alg_bytes(w):
     """Algorithmic HBM bytes: forward reads Q, K, V and writes O and L; the
     backward reads Q, K, V, O, dO, L and writes dQ, dK, dV (D and L*log2(e)
     are workspace, counted as one write and one read each)."""
-    es = 2 if w.dtype == "bf16" else 4
+    es = 4 if w.dtype == "fp32" else 2
     t = w.B * w.H * w.N * w.d * es
     rows = w.B * w.H * w.N * 4
     return 4 * t + rows, 8 * t + 3 * rows
@@ -230,9 +230,12 @@ def run_table(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    meas = {"bf16": peaks["bf16_tflops"], "fp32": peaks["bf16_tflops"] * SPEC_TF32_TFLOPS / SPEC_BF16_TFLOPS}
-    spec = {"bf16": SPEC_BF16_TFLOPS, "fp32": SPEC_TF32_TFLOPS}
+    meas = {"bf16": peaks["bf16_tflops"], "fp16": peaks["bf16_tflops"],
+            "fp32": peaks["bf16_tflops"] * SPEC_TF32_TFLOPS / SPEC_BF16_TFLOPS}
+    spec = {"bf16": SPEC_BF16_TFLOPS, "fp16": SPEC_BF16_TFLOPS, "fp32": SPEC_TF32_TFLOPS}
     points = list(fa2_inputs.WORKLOADS.values())
+    w10 = fa2_inputs.WORKLOADS["10b-b1h36-n4096-d128"]
+    points.append(fa2_inputs.Workload("10b-b1h36-n4096-d128-fp16", w10.B, w10.H, w10.N, w10.d, "fp16", w10.seed))
     points += [fa2_inputs.sweep_workload(N, d, dt) for dt in ("bf16", "fp32") for d in fa2_inputs.SWEEP_D
                for N in (128, 512, 1024, 4096, 8192, 16384, 32768)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)

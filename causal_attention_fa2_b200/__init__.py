@@ -21,7 +21,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import _native
-from ._native import (FA2_BF16, FA2_FP32, FA2Error, clear_device_status,  # noqa: F401
+from ._native import (FA2_BF16, FA2_FP16, FA2_FP32, FA2Error, clear_device_status,  # noqa: F401
                       last_device_status, library_path, status_string)
 
 __all__ = [
@@ -31,14 +31,14 @@ __all__ = [
 ]
 
 SUPPORTED_HEAD_DIMS = (16, 32, 64, 80, 128)
-_DTYPES = {torch.bfloat16: FA2_BF16, torch.float32: FA2_FP32}
+_DTYPES = {torch.bfloat16: FA2_BF16, torch.float32: FA2_FP32, torch.float16: FA2_FP16}
 
 
 def _dtype_code(t: torch.Tensor) -> int:
     try:
         return _DTYPES[t.dtype]
     except KeyError:
-        raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+        raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16, torch.float16 or torch.float32")
 
 
 def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
@@ -67,7 +67,7 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
             lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T (+ causal mask)) V and L = logsumexp (fp32).
 
-    q, k, v: contiguous CUDA tensors [B, H, N, d] (bf16 or fp32).
+    q, k, v: contiguous CUDA tensors [B, H, N, d] (bf16, fp16 or fp32).
     Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).
     """
     B, H, N, d = _check_qkv(q, k, v)

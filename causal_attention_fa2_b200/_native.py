@@ -12,6 +12,7 @@ from typing import Optional
 
 FA2_BF16 = 0
 FA2_FP32 = 1
+FA2_FP16 = 2
 
 FA2_OK = 0
 FA2_ERR_DEVICE_TIMEOUT = 8

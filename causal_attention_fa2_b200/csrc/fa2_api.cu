@@ -74,7 +74,7 @@ bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 80
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2_dtype dtype) {
-    if (dtype != FA2_BF16 && dtype != FA2_FP32) return FA2_ERR_UNSUPPORTED_DTYPE;
+    if (dtype != FA2_BF16 && dtype != FA2_FP32 && dtype != FA2_FP16) return FA2_ERR_UNSUPPORTED_DTYPE;
     if (B < 1 || H < 1 || N < 1 || N > kMaxN) return FA2_ERR_BAD_SHAPE;
     if (static_cast<long long>(B) * H > (1ll << 31) - 1) return FA2_ERR_BAD_SHAPE;
     const long long tiles = (N + kTileRows - 1) / kTileRows;
@@ -89,7 +89,7 @@ fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2
 // of box_cols x 128 rows x 1 head.
 fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int N, int BH,
                     int box_cols, int row_bytes, bool mn_major_f32, int box_rows = kTileRows) {
-    const int es = dtype == FA2_BF16 ? 2 : 4;
+    const int es = dtype == FA2_FP32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                           static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es,
@@ -101,8 +101,9 @@ fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int
                             : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
                                                : CU_TENSOR_MAP_SWIZZLE_32B;
     CUresult r = g_encode(m,
-                          dtype == FA2_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          dtype == FA2_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                          : dtype == FA2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                           3, const_cast<void*>(ptr), dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -137,7 +138,7 @@ constexpr bool use_two_tile_forward() {
     return ES == 2 && Fwd2Cfg<ES, D>::kFits;
 }
 
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int H, int N, int causal, float scale, fa2_dtype dtype,
                           cudaStream_t stream, uint32_t* status) {
@@ -160,8 +161,8 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.timeout_ns = kDefaultTimeoutNs;
     if constexpr (use_two_tile_forward<ES, D>()) {
         // Two query tiles per CTA (softmax of one overlaps the MMAs of the other).
-        using Cfg2 = Fwd2Cfg<ES, D>;
-        auto kern = fa2_fwd2_kernel<ES, D>;
+        using Cfg2 = Fwd2Cfg<ES, D, F16>;
+        auto kern = fa2_fwd2_kernel<ES, D, F16>;
         if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
         const unsigned pairs = static_cast<unsigned>((p.n_tiles + 1) / 2);
         kern<<<pairs * static_cast<unsigned>(BH), Cfg2::kThreads, Cfg2::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
@@ -174,29 +175,29 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
 
-template <int ES>
+template <int ES, bool F16 = false>
 fa2_status dispatch_forward(int d, const void* q, const void* k, const void* v, void* o,
                             float* lse, int B, int H, int N, int causal, float scale,
                             fa2_dtype dtype, cudaStream_t stream, uint32_t* status) {
     switch (d) {
-        case 16: return launch_forward<ES, 16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
-        case 32: return launch_forward<ES, 32>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
-        case 64: return launch_forward<ES, 64>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
-        case 80: return launch_forward<ES, 80>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
-        case 128: return launch_forward<ES, 128>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 16: return launch_forward<ES, 16, F16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 32: return launch_forward<ES, 32, F16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 64: return launch_forward<ES, 64, F16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 80: return launch_forward<ES, 80, F16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
+        case 128: return launch_forward<ES, 128, F16>(q, k, v, o, lse, B, H, N, causal, scale, dtype, stream, status);
         default: return FA2_ERR_UNSUPPORTED_HEAD_DIM;
     }
 }
 
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 fa2_status launch_backward_t(const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
                              int B, int H, int N, int causal, float scale, fa2_dtype dtype,
                              uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                              uint32_t* status, unsigned long long timeout_ns,
                              void* const* events) {
-    using T = typename std::conditional<ES == 2, __nv_bfloat16, float>::type;
-    using Cfg = BwdCfg<ES, D>;
+    using T = typename std::conditional<ES == 2, uint16_t, float>::type;
+    using Cfg = BwdCfg<ES, D, F16>;
     auto mark = [&](int i) -> bool {
         if (!events || !events[i]) return true;
         return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
@@ -209,7 +210,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     const long long rows = static_cast<long long>(BH) * ws.n_pad;
     if (!mark(0)) return FA2_ERR_CUDA;
     constexpr int kPreRows = BwdPreCfg<D>::kRowsPerBlock;
-    fa2_bwd_pre_kernel<D><<<static_cast<unsigned>((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
+    fa2_bwd_pre_kernel<D, F16><<<static_cast<unsigned>((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
         static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
@@ -235,14 +236,14 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
     // 2. dK, dV: key/value-tile-outer pass.
     {
-        auto kern = fa2_bwd_dkdv_kernel<ES, D>;
+        auto kern = fa2_bwd_dkdv_kernel<ES, D, F16>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     }
     // 3. dQ: query-tile-outer pass.
     {
-        auto kern = fa2_bwd_dq_kernel<ES, D>;
+        auto kern = fa2_bwd_dq_kernel<ES, D, F16>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
@@ -342,6 +343,10 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
         if (dtype == FA2_FP32)                                                                \
             return launch_backward32_t<DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal, \
                                            scale, ws_base, ws, stream, status, timeout_ns, events); \
+        if (dtype == FA2_FP16)                                                                \
+            return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N,   \
+                                                  causal, scale, dtype, ws_base, ws, stream,    \
+                                                  status, timeout_ns, events);                  \
         return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, causal,   \
                                         scale, dtype, ws_base, ws, stream, status, timeout_ns, events);
     switch (d) {
@@ -377,6 +382,8 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == FA2_BF16)
         return dispatch_forward<2>(d, q, k, v, o, lse, B, H, N, causal, scale, dtype, s, status);
+    if (dtype == FA2_FP16)
+        return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, N, causal, scale, dtype, s, status);
     return dispatch_forward<4>(d, q, k, v, o, lse, B, H, N, causal, scale, dtype, s, status);
 }
 
@@ -445,7 +452,7 @@ const char* fa2_status_string(fa2_status status) {
         case FA2_ERR_NULL_PTR: return "FA2_ERR_NULL_PTR: a required pointer is NULL";
         case FA2_ERR_BAD_SHAPE: return "FA2_ERR_BAD_SHAPE: B, H or N out of range";
         case FA2_ERR_UNSUPPORTED_HEAD_DIM: return "FA2_ERR_UNSUPPORTED_HEAD_DIM: d must be 16, 32, 64, 80 or 128";
-        case FA2_ERR_UNSUPPORTED_DTYPE: return "FA2_ERR_UNSUPPORTED_DTYPE: dtype must be FA2_BF16 or FA2_FP32";
+        case FA2_ERR_UNSUPPORTED_DTYPE: return "FA2_ERR_UNSUPPORTED_DTYPE: dtype must be FA2_BF16, FA2_FP32 or FA2_FP16";
         case FA2_ERR_MISALIGNED: return "FA2_ERR_MISALIGNED: tensors need 16-byte, lse 4-byte, workspace 256-byte alignment";
         case FA2_ERR_WORKSPACE_TOO_SMALL: return "FA2_ERR_WORKSPACE_TOO_SMALL: see fa2_backward_workspace_bytes";
         case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call or kernel launch failed";

@@ -83,9 +83,10 @@ struct BwdPreCfg {
 
 // D_i = rowsum(O_i o dO_i) and L_i * log2(e) per query row; rows past N (up
 // to the padded length) get D = 0 and L = +inf so they drop out of P and dS.
-template <int D>
+// O and dO are 16-bit (bf16, or fp16 when F16), read as raw 16-bit pairs.
+template <int D, bool F16 = false>
 __global__ void __launch_bounds__(256)
-fa2_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                    const float* __restrict__ lse, float* __restrict__ l2,
                    float* __restrict__ dvec, int N, int n_pad, long long rows_total) {
     using C = BwdPreCfg<D>;
@@ -103,8 +104,11 @@ fa2_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __r
         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(bw[w] << 16), acc);
-            acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(bw[w] & 0xffff0000u), acc);
+            float a0, a1, b0, b1;
+            TileGeom<2, D, F16>::unpack2(aw[w], a0, a1);
+            TileGeom<2, D, F16>::unpack2(bw[w], b0, b1);
+            acc = fmaf(a0, b0, acc);
+            acc = fmaf(a1, b1, acc);
         }
     }
 #pragma unroll
@@ -132,9 +136,9 @@ struct BwdParams {
     unsigned long long timeout_ns;
 };
 
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 struct BwdCfg {
-    using G = TileGeom<ES, D>;
+    using G = TileGeom<ES, D, F16>;
     static_assert(ES == 2, "the backward kernels are written for 16-bit inputs");
     static constexpr int kThreads = 320;   // 10 warps
     static constexpr int kTile = G::kTileBytesK;
@@ -156,13 +160,13 @@ struct BwdCfg {
 //   dV += P^T(i) dO(i)      (A = P^T from TMEM)     ; S^T(i+1) = K Q(i+1)^T
 //   dK += dS^T(i) Q(i)      (A = dS^T from TMEM)    ; dP^T(i+1) = V dO(i+1)^T
 // while the groups compute P^T(i+1) and dS^T(i+1).
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const BwdParams p) {
-    using Cfg = BwdCfg<ES, D>;
+    using Cfg = BwdCfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int RS = Cfg::kRing;
     constexpr int TB = Cfg::kTile;
@@ -381,8 +385,8 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         if ((diag && r > qc0 + c + h) || !key_valid) pe = 0.f;
                         pv[h] = pe;
                     }
-                    pk[c >> 1] = ptx::pack_bf16x2(pv[0], pv[1]);
-                    pk[(c >> 1) + 1] = ptx::pack_bf16x2(pv[2], pv[3]);
+                    pk[c >> 1] = G::pack2(pv[0], pv[1]);
+                    pk[(c >> 1) + 1] = G::pack2(pv[2], pv[3]);
                 }
             }
             if (!ptx::mbar_wait(&bar_s_read, it & 1, &abort_flag, tmo)) { ok = false; break; }
@@ -411,10 +415,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
 #pragma unroll
                     for (int h = 0; h < 4; h += 2) {
-                        const uint32_t pw = pk[(c + h) >> 1];
-                        const float p0 = __uint_as_float(pw << 16);
-                        const float p1 = __uint_as_float(pw & 0xffff0000u);
-                        dk[(c + h) >> 1] = ptx::pack_bf16x2(p0 * (__uint_as_float(ud[c + h]) - dq4[h]),
+                        float p0, p1;
+                        G::unpack2(pk[(c + h) >> 1], p0, p1);
+                        dk[(c + h) >> 1] = G::pack2(p0 * (__uint_as_float(ud[c + h]) - dq4[h]),
                                                             p1 * (__uint_as_float(ud[c + h + 1]) - dq4[h + 1]));
                     }
                 }
@@ -446,10 +449,10 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     if (cc < D) {
                         const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
                         uint4 w;
-                        w.x = ptx::pack_bf16x2(f[0] * mul, f[1] * mul);
-                        w.y = ptx::pack_bf16x2(f[2] * mul, f[3] * mul);
-                        w.z = ptx::pack_bf16x2(f[4] * mul, f[5] * mul);
-                        w.w = ptx::pack_bf16x2(f[6] * mul, f[7] * mul);
+                        w.x = G::pack2(f[0] * mul, f[1] * mul);
+                        w.y = G::pack2(f[2] * mul, f[3] * mul);
+                        w.z = G::pack2(f[4] * mul, f[5] * mul);
+                        w.w = G::pack2(f[6] * mul, f[7] * mul);
                         *reinterpret_cast<uint4*>(out_stage + kmajor_chunk_offset<G>(r, cc)) = w;
                     }
                 }
@@ -484,12 +487,12 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 //   S(j) = Q K_j^T ; dP(j) = dO V_j^T ; dQ += dS(j) K_j   (A = dS from TMEM)
 // issuing S(j+1) as soon as both groups have read S(j), and dP(j+1) right
 // after dQ(j), so the groups' exponentials overlap the tensor core.
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-    using Cfg = BwdCfg<ES, D>;
+    using Cfg = BwdCfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int RS = Cfg::kRing;
     constexpr int TB = Cfg::kTile;
@@ -676,7 +679,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         if ((diag && kc0 + c + h > r) || c + h >= kv_valid) pe = 0.f;
                         pv[h] = pe;
                     }
-                    pk[c >> 1] = ptx::pack_bf16x2(pv[0], pv[1]);
+                    pk[c >> 1] = G::pack2(pv[0], pv[1]);
                 }
             }
             // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
@@ -693,10 +696,9 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (lane == 0) ptx::mbar_arrive(&bar_dp_read);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    const uint32_t pw = pk[c >> 1];
-                    const float p0 = __uint_as_float(pw << 16);
-                    const float p1 = __uint_as_float(pw & 0xffff0000u);
-                    dk[c >> 1] = ptx::pack_bf16x2(p0 * (__uint_as_float(ud[c]) - dr),
+                    float p0, p1;
+                    G::unpack2(pk[c >> 1], p0, p1);
+                    dk[c >> 1] = G::pack2(p0 * (__uint_as_float(ud[c]) - dr),
                                                   p1 * (__uint_as_float(ud[c + 1]) - dr));
                 }
             }
@@ -725,10 +727,10 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
                             const float s = p.scale;
                             uint4 w;
-                            w.x = ptx::pack_bf16x2(f[0] * s, f[1] * s);
-                            w.y = ptx::pack_bf16x2(f[2] * s, f[3] * s);
-                            w.z = ptx::pack_bf16x2(f[4] * s, f[5] * s);
-                            w.w = ptx::pack_bf16x2(f[6] * s, f[7] * s);
+                            w.x = G::pack2(f[0] * s, f[1] * s);
+                            w.y = G::pack2(f[2] * s, f[3] * s);
+                            w.z = G::pack2(f[4] * s, f[5] * s);
+                            w.w = G::pack2(f[6] * s, f[7] * s);
                             *reinterpret_cast<uint4*>(sQ + kmajor_chunk_offset<G>(r, cc)) = w;
                         }
                     }

@@ -36,9 +36,9 @@
 
 namespace fa2 {
 
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 struct Fwd2Cfg {
-    using G = TileGeom<ES, D>;
+    using G = TileGeom<ES, D, F16>;
     static constexpr int kThreads = 320;
     static constexpr int kBudget = 227 * 1024 - 2048;
     static constexpr int kQBytes = 2 * G::kTileBytesK;
@@ -56,14 +56,14 @@ struct Fwd2Cfg {
 
 // One softmax warpgroup: processes query tile `t` (0 = A, 1 = B) for key
 // tiles 0 .. n_kv-1, then writes its O tile and L rows.
-template <int ES, int D>
+template <int ES, int D, bool F16>
 __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_tile, int n_kv,
                                              int bh, uint32_t tmem, uint8_t* sQt,
                                              uint64_t* bar_s_full, uint64_t* bar_p_full,
                                              uint64_t* bar_o_done,
                                              volatile uint32_t* abort_flag,
                                              const CUtensorMap* tm_o) {
-    using Cfg = Fwd2Cfg<ES, D>;
+    using Cfg = Fwd2Cfg<ES, D, F16>;
     using G = typename Cfg::G;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -154,7 +154,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
             } else {
                 uint32_t u[16];
 #pragma unroll
-                for (int c = 0; c < 16; ++c) u[c] = ptx::pack_bf16x2(s[c0 + 2 * c], s[c0 + 2 * c + 1]);
+                for (int c = 0; c < 16; ++c) u[c] = G::pack2(s[c0 + 2 * c], s[c0 + 2 * c + 1]);
                 ptx::tmem_st16(s_tmem + c0 / 2, u);
             }
         }
@@ -194,10 +194,10 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
                     if (col < D) {
                         uint4 w;
                         const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
-                        w.x = ptx::pack_bf16x2(f[0] * inv_l, f[1] * inv_l);
-                        w.y = ptx::pack_bf16x2(f[2] * inv_l, f[3] * inv_l);
-                        w.z = ptx::pack_bf16x2(f[4] * inv_l, f[5] * inv_l);
-                        w.w = ptx::pack_bf16x2(f[6] * inv_l, f[7] * inv_l);
+                        w.x = G::pack2(f[0] * inv_l, f[1] * inv_l);
+                        w.y = G::pack2(f[2] * inv_l, f[3] * inv_l);
+                        w.z = G::pack2(f[4] * inv_l, f[5] * inv_l);
+                        w.w = G::pack2(f[6] * inv_l, f[7] * inv_l);
                         *reinterpret_cast<uint4*>(sQt + kmajor_chunk_offset<G>(r, col)) = w;
                     }
                 }
@@ -221,12 +221,12 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
     }
 }
 
-template <int ES, int D>
+template <int ES, int D, bool F16 = false>
 __global__ void __launch_bounds__(320, 1)
 fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const FwdParams p) {
-    using Cfg = Fwd2Cfg<ES, D>;
+    using Cfg = Fwd2Cfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int ST = Cfg::kStages;
     static_assert(ST >= 1, "two query tiles and one K/V stage do not fit in shared memory");
@@ -409,7 +409,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ------------------------------------------------ softmax warpgroups
         const int t = (warp - 2) >> 2;       // 0: warps 2-5 (tile A), 1: warps 6-9 (tile B)
         if (n_kv_t[t] > 0) {
-            fwd2_softmax<ES, D>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
+            fwd2_softmax<ES, D, F16>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
                                 &bar_p_full[t], &bar_o_done[t], &abort_flag, &tm_o);
         }
     }

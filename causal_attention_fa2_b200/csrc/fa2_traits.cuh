@@ -30,11 +30,14 @@ constexpr int kTileRows = 128;  // B_q = B_k = 128 rows per tile
 // Device status codes the kernels record (same values as fa2_status).
 constexpr uint32_t kDevStatusTimeout = 8;
 
-template <int ES, int D>
+// ES = element bytes (2 or 4); for 2-byte inputs F16 selects fp16 over bf16.
+template <int ES, int D, bool F16 = false>
 struct TileGeom {
+    static_assert(!(F16 && ES != 2), "fp16 inputs are 2-byte elements");
     static constexpr int kES = ES;
     static constexpr int kD = D;
     static constexpr bool kF32 = (ES == 4);
+    static constexpr bool kF16 = F16;
     // K-major staging.
     static constexpr int kBoxK = (D * ES >= 128) ? (128 / ES) : D;
     static constexpr int kRowBK = kBoxK * ES;
@@ -53,7 +56,17 @@ struct TileGeom {
     static constexpr int kStepsD = (D + kKStep - 1) / kKStep;    // MMAs to contract over d
     static constexpr int kStepsRows = kTileRows / kKStep;        // MMAs to contract over 128 rows
     static constexpr int kNOut = (D + 15) / 16 * 16;              // MMA N when d is the output dim
-    static constexpr uint32_t kFmt = kF32 ? ptx::kFmtTF32 : ptx::kFmtBF16;
+    static constexpr uint32_t kFmt = kF32 ? ptx::kFmtTF32 : (F16 ? ptx::kFmtF16 : ptx::kFmtBF16);
+    // Two fp32 values rounded (nearest even) to the 16-bit input type, packed
+    // with the first in the low half; and the reverse, exact.
+    static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+        if constexpr (F16) return ptx::pack_f16x2(lo, hi);
+        else return ptx::pack_bf16x2(lo, hi);
+    }
+    static __device__ __forceinline__ void unpack2(uint32_t w, float& lo, float& hi) {
+        if constexpr (F16) ptx::unpack_f16x2(w, lo, hi);
+        else ptx::unpack_bf16x2(w, lo, hi);
+    }
     static constexpr int kPCols = kF32 ? 128 : 64;                // TMEM columns of a 128-wide P row
 };
 

@@ -401,6 +401,24 @@ __device__ __forceinline__ uint32_t to_tf32_rna(float x) {
     return r;
 }
 
+// Two fp32 values rounded to nearest-even fp16, packed (lo in the low half).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// The two halves of a packed 16-bit pair widened to fp32 (exact).
+__device__ __forceinline__ void unpack_bf16x2(uint32_t w, float& lo, float& hi) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ void unpack_f16x2(uint32_t w, float& lo, float& hi) {
+    unsigned short a = static_cast<unsigned short>(w & 0xffffu), b = static_cast<unsigned short>(w >> 16);
+    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(a));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(b));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

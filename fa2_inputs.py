@@ -21,7 +21,7 @@ from typing import Dict, List
 
 import torch
 
-DTYPES = {"bf16": torch.bfloat16, "fp32": torch.float32}
+DTYPES = {"bf16": torch.bfloat16, "fp32": torch.float32, "fp16": torch.float16}
 
 
 @dataclasses.dataclass(frozen=True)

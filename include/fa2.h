@@ -49,10 +49,13 @@ extern "C" {
 #endif
 
 /* Element type of q, k, v, o, dout, dq, dk, dv.  Accumulation is always fp32.
- * FA2_FP32 inputs are consumed by the tensor cores as TF32. */
+ * FA2_FP32 inputs are consumed by the tensor cores as TF32 (rounded to
+ * nearest); FA2_BF16 and FA2_FP16 inputs directly, with P and dS rounded to
+ * the input type before their MMAs. */
 typedef enum {
     FA2_BF16 = 0,
-    FA2_FP32 = 1
+    FA2_FP32 = 1,
+    FA2_FP16 = 2
 } fa2_dtype;
 
 typedef enum {

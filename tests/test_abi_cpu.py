@@ -70,7 +70,7 @@ def test_forward_validation(fa2lib):
     assert fwd(L, N=(1 << 24) + 1) == 2
     for d in (0, 8, 48, 96, 256):
         assert fwd(L, d=d) == 3                    # FA2_ERR_UNSUPPORTED_HEAD_DIM
-    assert fwd(L, dtype=2) == 4                    # FA2_ERR_UNSUPPORTED_DTYPE
+    assert fwd(L, dtype=3) == 4                    # FA2_ERR_UNSUPPORTED_DTYPE
     assert fwd(L, q=BAD) == 5                      # FA2_ERR_MISALIGNED
     assert fwd(L, o=P + 8) == 5
     assert fwd(L, lse=P + 2) == 5
@@ -101,6 +101,7 @@ def test_workspace_size(fa2lib, B, H, N, d):
     n_pad = (N + 127) // 128 * 128
     expect = 2 * up(B * H * n_pad * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 2) == expect      # fp16
     # fp32 inputs: plus TF32-rounded copies of q, k, v and dout.
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 1) == expect + 4 * up(B * H * N * d * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, 24, 0) == 0

@@ -67,6 +67,33 @@ def test_fp32_small_full_parity(oracle_mod, B, H, N, d, causal):
         assert_close(to64(got[name]), ref[name], "fp32", name)
 
 
+@pytest.mark.parametrize("causal", [True, False], ids=["causal", "full"])
+@pytest.mark.parametrize("B,H,N,d", SMALL)
+def test_fp16_small_full_parity(oracle_mod, B, H, N, d, causal):
+    """fp16 inputs (kind::f16 MMAs with fp16 operands): forward and backward in full."""
+    inp = fa2_inputs.make_inputs(B, H, N, d, "fp16", seed=23 + N + d)
+    scale = default_scale(d)
+    got = gpu_fwd_bwd(inp, causal, scale)
+    ref = _oracle(oracle_mod, inp, causal, scale)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(to64(got[name]), ref[name], "fp16", name)
+
+
+def test_fp16_10b_shape_heads(oracle_mod):
+    """The 10B head shape (B=1, H=36, N=4096, d=128) with fp16 inputs; first and
+    last head compared in full."""
+    w = fa2_inputs.WORKLOADS["10b-b1h36-n4096-d128"]
+    inp = fa2_inputs.make_inputs(w.B, w.H, w.N, w.d, "fp16", seed=w.seed)
+    got = gpu_fwd_bwd(inp, w.causal, w.scale)
+    for hh in (0, w.H - 1):
+        q, k, v, do = (to64(inp[n][0, hh].float()) for n in ("q", "k", "v", "do"))
+        o, lse = oracle_mod.forward(q, k, v, w.causal, w.scale)
+        dq, dk, dv = oracle_mod.backward(q, k, v, do, w.causal, w.scale)
+        for name, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            e = assert_close(to64(got[name][0, hh]), ref, "fp16", f"{name}[head {hh}]")
+            print(f"ERR fp16-10b head {hh} {name} max_abs {e:.3e}")
+
+
 @pytest.mark.parametrize("scale", [0.09, 0.14])
 def test_nondefault_scale(oracle_mod, scale):
     """A scale other than 1/sqrt(d) must enter S, dQ and dK.  (Much sharper
