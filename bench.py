@@ -236,6 +236,10 @@ def run_table(args):
     points = list(fa2_inputs.WORKLOADS.values())
     w10 = fa2_inputs.WORKLOADS["10b-b1h36-n4096-d128"]
     points.append(fa2_inputs.Workload("10b-b1h36-n4096-d128-fp16", w10.B, w10.H, w10.N, w10.d, "fp16", w10.seed))
+    # Grouped-query points: (workload, key/value heads).
+    gqa = {"10b-b1h36-n4096-d128-gqa-kv4": 4, "10b-b1h36-n4096-d128-mqa": 1}
+    for name in gqa:
+        points.append(fa2_inputs.Workload(name, w10.B, w10.H, w10.N, w10.d, "bf16", w10.seed))
     points += [fa2_inputs.sweep_workload(N, d, dt) for dt in ("bf16", "fp32") for d in fa2_inputs.SWEEP_D
                for N in (128, 512, 1024, 4096, 8192, 16384, 32768)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -248,7 +252,9 @@ def run_table(args):
         g = torch.Generator(device="cpu")
         g.manual_seed(w.seed)
         dt = fa2_inputs.DTYPES[w.dtype]
-        q, k, v, do = (torch.randn((w.B, w.H, w.N, w.d), generator=g).to(dt).to(dev) for _ in range(4))
+        h_kv = gqa.get(w.name, w.H)
+        q, k, v, do = (torch.randn((w.B, h, w.N, w.d), generator=g).to(dt).to(dev)
+                       for h in (w.H, h_kv, h_kv, w.H))
         o, lse = fa2.forward(q, k, v, causal=w.causal, scale=w.scale)
         ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype), dtype=torch.uint8, device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)

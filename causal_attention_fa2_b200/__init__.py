@@ -42,10 +42,15 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
-    if q.dim() != 4:
-        raise ValueError("expected q, k, v of shape [B, H, N, d]")
-    if k.shape != q.shape or v.shape != q.shape:
-        raise ValueError(f"q, k, v shapes must match, got {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
+    """q [B, H, N, d]; k, v [B, H_kv, N, d] with H a multiple of H_kv (H_kv < H:
+    grouped-query attention).  Returns (B, H, H_kv, N, d)."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("expected q, k, v of shape [B, H, N, d] (k, v: [B, H_kv, N, d])")
+    B, H, N, d = q.shape
+    if (k.shape != v.shape or k.shape[0] != B or k.shape[2:] != q.shape[2:]
+            or k.shape[1] < 1 or H % k.shape[1]):
+        raise ValueError(f"q, k, v shapes do not fit [B, H, N, d] / [B, H_kv, N, d] with H a multiple "
+                         f"of H_kv: {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -55,7 +60,7 @@ def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
             raise ValueError(f"{name} must be contiguous [B, H, N, d]")
     if k.device != q.device or v.device != q.device:
         raise ValueError("q, k, v must be on one device")
-    return tuple(q.shape)
+    return B, H, k.shape[1], N, d
 
 
 def _stream_handle(device: torch.device) -> int:
@@ -67,10 +72,12 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
             lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T (+ causal mask)) V and L = logsumexp (fp32).
 
-    q, k, v: contiguous CUDA tensors [B, H, N, d] (bf16, fp16 or fp32).
+    q: contiguous CUDA tensor [B, H, N, d] (bf16, fp16 or fp32); k, v:
+    [B, H_kv, N, d] with H a multiple of H_kv (grouped-query attention when
+    H_kv < H: query head h uses key/value head h // (H // H_kv)).
     Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).
     """
-    B, H, N, d = _check_qkv(q, k, v)
+    B, H, H_kv, N, d = _check_qkv(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -78,10 +85,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
-        _native.check(_native.lib().fa2_forward(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-            B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
-            _stream_handle(q.device)))
+        if H_kv == H:
+            _native.check(_native.lib().fa2_forward(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
+                _stream_handle(q.device)))
+        else:
+            _native.check(_native.lib().fa2_forward_gqa(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, H, H_kv, N, d, int(bool(causal)), float(scale), _dtype_code(q),
+                _stream_handle(q.device)))
     return out, lse
 
 
@@ -102,7 +115,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     objects the library records at its kernel boundaries (before the D/L
     pre-pass, after it, after the main pass, after the dQ finalisation).
     """
-    B, H, N, d = _check_qkv(q, k, v)
+    B, H, H_kv, N, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
         if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
@@ -120,7 +133,17 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     if events is not None:
         if len(events) != 4:
             raise ValueError("events must hold four torch.cuda.Event objects")
+        if H_kv != H:
+            raise ValueError("events are supported for H_kv == H only")
         ev_arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    if H_kv != H:
+        with torch.cuda.device(q.device):
+            _native.check(_native.lib().fa2_backward_gqa(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d,
+                int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
+                workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
+        return dq, dk, dv
     with torch.cuda.device(q.device):
         _native.check(_native.lib().fa2_backward_timed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),

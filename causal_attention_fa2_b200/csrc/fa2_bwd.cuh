@@ -131,6 +131,7 @@ struct BwdParams {
     const float* dvec;     // [BH][n_pad]  D, 0 past N
     uint32_t* status;
     int N, BH, n_tiles, n_pad, causal;
+    int H, H_kv, group, BH_kv;   // query heads, key/value heads, H / H_kv, B * H_kv
     float scale_log2;      // scale * log2(e)
     float scale;
     unsigned long long timeout_ns;
@@ -193,14 +194,20 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: with the causal mask, key tile j is seen by query tiles j..T-1,
-    // so small j carries the most work and is issued first.
+    // Work item: (key tile j, key/value head).  Key tile j is seen by query
+    // tiles j..T-1 (causal) of each of the `group` query heads sharing this
+    // key/value head, whose dK and dV sum over all of them; small j carries
+    // the most work and is issued first.
     const int item = blockIdx.x;
-    const int kv_tile = item / p.BH;
-    const int bh = item - kv_tile * p.BH;
+    const int kv_tile = item / p.BH_kv;
+    const int bh = item - kv_tile * p.BH_kv;            // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
-    const int n_q = p.n_tiles - i_begin;
+    const int n_q = p.n_tiles - i_begin;                // query tiles per query head
+    const int n_it = n_q * p.group;                     // (query head, query tile) steps
     const int kv_row0 = kv_tile * kTileRows;
+    // Step it: query tile i_begin + it % n_q of the it / n_q-th query head of the group.
+    auto q_tile_of = [&](int it) { return i_begin + it % n_q; };
+    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -242,19 +249,20 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
             }
             int q_issued = 0, do_issued = 0;
-            for (int it = 0; it < n_q; ++it) {
-                const int row0 = (i_begin + it) * kTileRows;
+            for (int it = 0; it < n_it; ++it) {
+                const int row0 = q_tile_of(it) * kTileRows;
+                const int qh = q_head_of(it);
                 const int s = it % RS;
                 const uint32_t ph = ((it / RS) & 1) ^ 1;
                 if (it >= RS && !ptx::mbar_wait(&bar_q_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_q_full[s], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(sQr + s * TB + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full[s], b * G::kBoxK, row0, bh);
+                    ptx::tma_load_3d(sQr + s * TB + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full[s], b * G::kBoxK, row0, qh);
                 q_issued = it + 1;
                 if (it >= RS && !ptx::mbar_wait(&bar_do_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_do_full[s], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(sDOr + s * TB + b * kTileRows * G::kRowBK, &tm_do, &bar_do_full[s], b * G::kBoxK, row0, bh);
+                    ptx::tma_load_3d(sDOr + s * TB + b * kTileRows * G::kRowBK, &tm_do, &bar_do_full[s], b * G::kBoxK, row0, qh);
                 do_issued = it + 1;
             }
             if (abort_flag) {
@@ -299,7 +307,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             };
             bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
             if (ok) ok = issue_s(0) && issue_dp(0);
-            for (int it = 0; ok && it < n_q; ++it) {
+            for (int it = 0; ok && it < n_it; ++it) {
                 // dV_j += P^T dO_i   (Eq. 15); P^T read from the score columns.
                 if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
@@ -308,7 +316,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
                     ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8, desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_do_empty[it % RS]);
-                if (it + 1 < n_q && !issue_s(it + 1)) { ok = false; break; }
+                if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
                 if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
@@ -317,7 +325,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
                     ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * 8, desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_q_empty[it % RS]);
-                if (it + 1 < n_q && !issue_dp(it + 1)) { ok = false; break; }
+                if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
             }
             if (ok) {
                 ptx::mma_commit(&bar_dkv_full);
@@ -336,16 +344,19 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool key_valid = kv_row0 + r < p.N;
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
-        const size_t vec_base = static_cast<size_t>(bh) * p.n_pad + qc0;
+        // Offset of step it's L / D values for this group's 64 query columns.
+        auto vec_base = [&](int it) {
+            return static_cast<size_t>(q_head_of(it)) * p.n_pad + static_cast<size_t>(q_tile_of(it)) * kTileRows + qc0;
+        };
         float nl2[2], nd[2];
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-            nl2[m] = p.l2[vec_base + static_cast<size_t>(i_begin) * kTileRows + lane + 32 * m];
-            nd[m] = p.dvec[vec_base + static_cast<size_t>(i_begin) * kTileRows + lane + 32 * m];
+            nl2[m] = p.l2[vec_base(0) + lane + 32 * m];
+            nd[m] = p.dvec[vec_base(0) + lane + 32 * m];
         }
         bool ok = true;
-        for (int it = 0; it < n_q; ++it) {
-            const int i = i_begin + it;
+        for (int it = 0; it < n_it; ++it) {
+            const int i = q_tile_of(it);
             const int b = it & 1;
 #pragma unroll
             for (int m = 0; m < 2; ++m) {
@@ -353,11 +364,12 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 sDv[wi][b][lane + 32 * m] = nd[m];
             }
             __syncwarp();
-            if (it + 1 < n_q) {
+            if (it + 1 < n_it) {
+                const size_t nb = vec_base(it + 1);
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
-                    nl2[m] = p.l2[vec_base + static_cast<size_t>(i + 1) * kTileRows + lane + 32 * m];
-                    nd[m] = p.dvec[vec_base + static_cast<size_t>(i + 1) * kTileRows + lane + 32 * m];
+                    nl2[m] = p.l2[nb + lane + 32 * m];
+                    nd[m] = p.dvec[nb + lane + 32 * m];
                 }
             }
             const bool diag = p.causal && (i == kv_tile);
@@ -522,6 +534,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
     const int n_kv = p.causal ? (q_tile + 1) : p.n_tiles;
     const int q_row0 = q_tile * kTileRows;
+    const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -569,12 +582,12 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (j >= RS && !ptx::mbar_wait(&bar_k_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_k_full[s], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sKr + s * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh, keep);
+                    ptx::tma_load_3d_hint(sKr + s * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
                 k_issued = j + 1;
                 if (j >= RS && !ptx::mbar_wait(&bar_v_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[s], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sVr + s * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[s], b * G::kBoxK, j * kTileRows, bh, keep);
+                    ptx::tma_load_3d_hint(sVr + s * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
                 v_issued = j + 1;
             }
             if (abort_flag) {

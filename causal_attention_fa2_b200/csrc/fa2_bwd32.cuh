@@ -79,17 +79,15 @@ struct Bwd32Cfg {
 
 // ------------------------------------------------------------------ pre-processing
 
-// One warp per query row (8 rows per block): TF32-rounded copies of the q, k,
-// v and dout rows, D_i = sum_t round(dO_it) O_it, and L_i * log2(e); rows past
-// N (up to the padded length) get D = 0 and L = +inf.
+// One warp per query row (8 rows per block): TF32-rounded copies of the q and
+// dout rows, D_i = sum_t round(dO_it) O_it, and L_i * log2(e); rows past N (up
+// to the padded length) get D = 0 and L = +inf.
 template <int D>
 __global__ void __launch_bounds__(256)
-fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ k,
-                     const float* __restrict__ v, const float* __restrict__ o,
+fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ o,
                      const float* __restrict__ dout, const float* __restrict__ lse,
-                     float* __restrict__ qr, float* __restrict__ kr, float* __restrict__ vr,
-                     float* __restrict__ dor, float* __restrict__ l2, float* __restrict__ dvec,
-                     int N, int n_pad, long long rows_total) {
+                     float* __restrict__ qr, float* __restrict__ dor, float* __restrict__ l2,
+                     float* __restrict__ dvec, int N, int n_pad, long long rows_total) {
     const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows_total) return;
@@ -108,8 +106,6 @@ fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ k,
         const float g = __uint_as_float(ptx::to_tf32_rna(dout[base + e]));
         dor[base + e] = g;
         qr[base + e] = __uint_as_float(ptx::to_tf32_rna(q[base + e]));
-        kr[base + e] = __uint_as_float(ptx::to_tf32_rna(k[base + e]));
-        vr[base + e] = __uint_as_float(ptx::to_tf32_rna(v[base + e]));
         acc += o[base + e] * g;
     }
 #pragma unroll
@@ -117,6 +113,20 @@ fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ k,
     if (lane == 0) {
         dvec[row] = acc;
         l2[row] = lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f;
+    }
+}
+
+// TF32-rounded copy of an fp32 tensor (k or v: [B * H_kv][N][d]), n4 float4s.
+__global__ void __launch_bounds__(256)
+fa2_round_tf32_kernel(const float4* __restrict__ in, float4* __restrict__ out, size_t n4) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float4 x = in[i];
+        x.x = __uint_as_float(ptx::to_tf32_rna(x.x));
+        x.y = __uint_as_float(ptx::to_tf32_rna(x.y));
+        x.z = __uint_as_float(ptx::to_tf32_rna(x.z));
+        x.w = __uint_as_float(ptx::to_tf32_rna(x.w));
+        out[i] = x;
     }
 }
 
@@ -242,15 +252,20 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: with the causal mask, key tile j is seen by query rows >= 128 j,
-    // so small j carries the most work and is issued first.
+    // Work item: (key tile j, key/value head).  Key tile j is seen by query
+    // rows >= 128 j (causal) of each of the `group` query heads sharing this
+    // key/value head, whose dK and dV sum over all of them; small j carries
+    // the most work and is issued first.
     const int item = blockIdx.x;
-    const int kv_tile = item / p.BH;
-    const int bh = item - kv_tile * p.BH;
+    const int kv_tile = item / p.BH_kv;
+    const int bh = item - kv_tile * p.BH_kv;            // key/value head
     const int kv_row0 = kv_tile * kTileRows;
     const int n_sub = (p.N + W - 1) / W;
     const int sub_begin = p.causal ? kv_row0 / W : 0;
-    const int n_q = n_sub - sub_begin;
+    const int n_q = n_sub - sub_begin;                  // sub-tiles per query head
+    const int n_it = n_q * p.group;                     // (query head, sub-tile) steps
+    auto q_row_of = [&](int it) { return (sub_begin + it % n_q) * W; };
+    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -290,18 +305,19 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
             }
             int issued = 0;
-            for (int it = 0; it < n_q; ++it) {
+            for (int it = 0; it < n_it; ++it) {
                 const int s = it % ST;
                 if (it >= ST && !ptx::mbar_wait(&bar_empty[s], ((it / ST) & 1) ^ 1, &abort_flag, tmo)) break;
-                const int row0 = (sub_begin + it) * W;
+                const int row0 = q_row_of(it);
+                const int qh = q_head_of(it);
                 ptx::mbar_arrive_expect_tx(&bar_full[s], SB);
                 for (int b = 0; b < G::kNBoxK; ++b) {
-                    ptx::tma_load_3d(st_qk(s) + b * W * G::kRowBK, &tm_qk, &bar_full[s], b * G::kBoxK, row0, bh);
-                    ptx::tma_load_3d(st_dok(s) + b * W * G::kRowBK, &tm_dok, &bar_full[s], b * G::kBoxK, row0, bh);
+                    ptx::tma_load_3d(st_qk(s) + b * W * G::kRowBK, &tm_qk, &bar_full[s], b * G::kBoxK, row0, qh);
+                    ptx::tma_load_3d(st_dok(s) + b * W * G::kRowBK, &tm_dok, &bar_full[s], b * G::kBoxK, row0, qh);
                 }
                 for (int b = 0; b < G::kNBoxMN; ++b) {
-                    ptx::tma_load_3d(st_qmn(s) + b * W * G::kRowBMN, &tm_qmn, &bar_full[s], b * G::kBoxMN, row0, bh);
-                    ptx::tma_load_3d(st_domn(s) + b * W * G::kRowBMN, &tm_domn, &bar_full[s], b * G::kBoxMN, row0, bh);
+                    ptx::tma_load_3d(st_qmn(s) + b * W * G::kRowBMN, &tm_qmn, &bar_full[s], b * G::kBoxMN, row0, qh);
+                    ptx::tma_load_3d(st_domn(s) + b * W * G::kRowBMN, &tm_domn, &bar_full[s], b * G::kBoxMN, row0, qh);
                 }
                 issued = it + 1;
             }
@@ -342,7 +358,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
             if (ok) ok = issue_s(0);
             if (ok) issue_dp(0);
-            for (int it = 0; ok && it < n_q; ++it) {
+            for (int it = 0; ok && it < n_it; ++it) {
                 const int s = it % ST;
                 // dV_j += P^T dO_i   (Eq. 15); P^T read from the score columns.
                 if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
@@ -351,7 +367,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
                     ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-                if (it + 1 < n_q && !issue_s(it + 1)) { ok = false; break; }
+                if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
                 if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
@@ -360,7 +376,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
                     ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_empty[s]);
-                if (it + 1 < n_q) issue_dp(it + 1);
+                if (it + 1 < n_it) issue_dp(it + 1);
             }
             if (ok) {
                 ptx::mma_commit(&bar_dkv_full);
@@ -377,10 +393,11 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int it = 0; it < n_q; ++it) {
-            const int q0 = (sub_begin + it) * W;
-            const float* l2q = p.l2 + static_cast<size_t>(bh) * p.n_pad + q0;
-            const float* dvq = p.dvec + static_cast<size_t>(bh) * p.n_pad + q0;
+        for (int it = 0; it < n_it; ++it) {
+            const int q0 = q_row_of(it);
+            const size_t qv = static_cast<size_t>(q_head_of(it)) * p.n_pad + q0;
+            const float* l2q = p.l2 + qv;
+            const float* dvq = p.dvec + qv;
             // Some query of this sub-tile precedes some key of the tile.
             const bool mask = p.causal && q0 < kv_row0 + kTileRows - 1;
             // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14), in place
@@ -489,6 +506,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int n_sub = (p.N + W - 1) / W;
     const int lim = (q_row0 + kTileRows) / W;
     const int n_kv = p.causal ? (lim < n_sub ? lim : n_sub) : n_sub;
+    const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -534,11 +552,11 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int row0 = j * W;
                 ptx::mbar_arrive_expect_tx(&bar_full[s], SB);
                 for (int b = 0; b < G::kNBoxK; ++b) {
-                    ptx::tma_load_3d_hint(st_kk(s) + b * W * G::kRowBK, &tm_kk, &bar_full[s], b * G::kBoxK, row0, bh, keep);
-                    ptx::tma_load_3d_hint(st_vk(s) + b * W * G::kRowBK, &tm_vk, &bar_full[s], b * G::kBoxK, row0, bh, keep);
+                    ptx::tma_load_3d_hint(st_kk(s) + b * W * G::kRowBK, &tm_kk, &bar_full[s], b * G::kBoxK, row0, bh_kv, keep);
+                    ptx::tma_load_3d_hint(st_vk(s) + b * W * G::kRowBK, &tm_vk, &bar_full[s], b * G::kBoxK, row0, bh_kv, keep);
                 }
                 for (int b = 0; b < G::kNBoxMN; ++b)
-                    ptx::tma_load_3d_hint(st_kmn(s) + b * W * G::kRowBMN, &tm_kmn, &bar_full[s], b * G::kBoxMN, row0, bh, keep);
+                    ptx::tma_load_3d_hint(st_kmn(s) + b * W * G::kRowBMN, &tm_kmn, &bar_full[s], b * G::kBoxMN, row0, bh_kv, keep);
                 issued = j + 1;
             }
             if (abort_flag) {

@@ -53,6 +53,7 @@ struct FwdParams {
     int N;                 // sequence length (queries = keys)
     int BH;                // batch * heads
     int n_tiles;           // ceil(N / 128)
+    int H, H_kv, group;    // query heads, key/value heads, H / H_kv
     int causal;
     float scale_log2;      // scale * log2(e)
     unsigned long long timeout_ns;
@@ -132,6 +133,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int q_tile = p.causal ? (p.n_tiles - 1 - tile_rank) : tile_rank;
     const int n_kv = p.causal ? (q_tile + 1) : p.n_tiles;
     const int q_row0 = q_tile * kTileRows;
+    const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -172,14 +174,14 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 uint8_t* dk = sK + ks * G::kTileBytesK;
                 ptx::mbar_arrive_expect_tx(&bar_k_full[ks], G::kTileBytesK);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, j * kTileRows, bh);
+                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, j * kTileRows, bh_kv);
                 k_issued = j + 1;
                 const int vs = j % VST;
                 if (j >= VST && !ptx::mbar_wait(&bar_v_empty[vs], ((j / VST) & 1) ^ 1, &abort_flag, tmo)) break;
                 uint8_t* dv = sV + vs * G::kTileBytesMN;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[vs], G::kTileBytesMN);
                 for (int b = 0; b < G::kNBoxMN; ++b)
-                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, j * kTileRows, bh);
+                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, j * kTileRows, bh_kv);
                 v_issued = j + 1;
             }
             if (abort_flag) {

@@ -259,6 +259,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int n_kv_t[2] = {p.causal ? tile[0] + 1 : p.n_tiles,
                            has_b ? (p.causal ? tile[1] + 1 : p.n_tiles) : 0};
     const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
+    const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -307,13 +308,13 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mbar_arrive_expect_tx(&bar_k_full[s], G::kTileBytesK);
                 for (int b = 0; b < G::kNBoxK; ++b)
                     ptx::tma_load_3d_hint(sK + s * G::kTileBytesK + b * kTileRows * G::kRowBK, &tm_k,
-                                          &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh, keep);
+                                          &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
                 k_issued = j + 1;
                 if (j >= ST && !ptx::mbar_wait(&bar_v_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[s], G::kTileBytesMN);
                 for (int b = 0; b < G::kNBoxMN; ++b)
                     ptx::tma_load_3d_hint(sV + s * G::kTileBytesMN + b * kTileRows * G::kRowBMN, &tm_v,
-                                          &bar_v_full[s], b * G::kBoxMN, j * kTileRows, bh, keep);
+                                          &bar_v_full[s], b * G::kBoxMN, j * kTileRows, bh_kv, keep);
                 v_issued = j + 1;
             }
             if (abort_flag) {

@@ -27,6 +27,14 @@ namespace fa2 {
 
 constexpr int kTileRows = 128;  // B_q = B_k = 128 rows per tile
 
+// Grouped-query attention: query heads h = g * group .. g * group + group - 1
+// of a batch share key/value head g.  `bh` indexes [B * H] query heads; the
+// result indexes [B * H_kv] key/value heads (H_kv = H / group; group = 1 is
+// plain multi-head attention).
+__host__ __device__ inline int kv_head_of(int bh, int H, int H_kv, int group) {
+    return (bh / H) * H_kv + (bh % H) / group;
+}
+
 // Device status codes the kernels record (same values as fa2_status).
 constexpr uint32_t kDevStatusTimeout = 8;
 

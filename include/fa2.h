@@ -92,6 +92,19 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
                        fa2_dtype dtype, fa2_stream_t stream);
 
 /*
+ * Grouped-query attention (the "LLM FLOPs Computation" page, section
+ * Extension: GQA): H query heads share H_kv key/value heads, query head h of a
+ * batch using key/value head h / (H / H_kv); H_kv = H is fa2_forward and
+ * H_kv = 1 is multi-query attention.
+ *   q, o   [B, H, N, d];  k, v  [B, H_kv, N, d];  lse [B, H, N] float32
+ * H must be a multiple of H_kv (else FA2_ERR_BAD_SHAPE).  Other arguments,
+ * results and errors are those of fa2_forward.
+ */
+fa2_status fa2_forward_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int H, int H_kv, int N, int d, int causal, float scale,
+                           fa2_dtype dtype, fa2_stream_t stream);
+
+/*
  * Bytes of device workspace fa2_backward needs for these sizes: the fp32 D
  * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes, and
  * for FA2_FP32 also copies of q, k, v and dout rounded to TF32 (round to
@@ -118,6 +131,19 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
                         int B, int H, int N, int d, int causal, float scale, fa2_dtype dtype,
                         void* workspace, size_t workspace_bytes, fa2_stream_t stream);
+
+/*
+ * Backward pass of fa2_forward_gqa: dq [B, H, N, d]; dk, dv [B, H_kv, N, d],
+ * each key/value head's gradient being the sum over the H / H_kv query heads
+ * that share it (accumulated in one thread block, so still deterministic).
+ * The workspace is fa2_backward_workspace_bytes(B, H, N, d, dtype) (query
+ * heads).  Other arguments, results and errors are those of fa2_backward.
+ */
+fa2_status fa2_backward_gqa(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                            int B, int H, int H_kv, int N, int d, int causal, float scale,
+                            fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                            fa2_stream_t stream);
 
 /*
  * fa2_backward plus timing hooks, for profiling: identical arguments and

@@ -118,3 +118,20 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa2.forward(x, x, x)
+
+
+def test_gqa_head_validation(fa2lib):
+    """fa2_forward_gqa / fa2_backward_gqa: H must be a positive multiple of H_kv."""
+    L = fa2lib
+
+    def fwd_gqa(H, H_kv):
+        return L.fa2_forward_gqa(P, P, P, P, P, 1, H, H_kv, 128, 64, 1, 0.125, 0, None)
+
+    def bwd_gqa(H, H_kv):
+        return L.fa2_backward_gqa(P, P, P, P, P, P, P, P, P, 1, H, H_kv, 128, 64, 1, 0.125, 0,
+                                  P, 1 << 30, None)
+
+    for H, H_kv in ((4, 3), (4, 0), (4, 8), (6, -2)):
+        assert fwd_gqa(H, H_kv) == 2, (H, H_kv)     # FA2_ERR_BAD_SHAPE
+        assert bwd_gqa(H, H_kv) == 2, (H, H_kv)
+    assert fwd_gqa(0, 1) == 2
