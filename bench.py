@@ -256,7 +256,7 @@ def run_table(args):
         q, k, v, do = (torch.randn((w.B, h, w.N, w.d), generator=g).to(dt).to(dev)
                        for h in (w.H, h_kv, h_kv, w.H))
         o, lse = fa2.forward(q, k, v, causal=w.causal, scale=w.scale)
-        ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype), dtype=torch.uint8, device=dev)
+        ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype, h_kv), dtype=torch.uint8, device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         f_fwd, f_bwd = flops(w)
         b_fwd, b_bwd = alg_bytes(w)

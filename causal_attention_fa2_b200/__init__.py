@@ -42,14 +42,15 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
-    """q [B, H, N, d]; k, v [B, H_kv, N, d] with H a multiple of H_kv (H_kv < H:
-    grouped-query attention).  Returns (B, H, H_kv, N, d)."""
+    """q [B, H, N, d]; k, v [B, H_kv, Nk, d] with H a multiple of H_kv (H_kv < H:
+    grouped-query attention; Nk != N: different key length).  Returns
+    (B, H, H_kv, N, Nk, d)."""
     if q.dim() != 4 or k.dim() != 4:
-        raise ValueError("expected q, k, v of shape [B, H, N, d] (k, v: [B, H_kv, N, d])")
+        raise ValueError("expected q of shape [B, H, N, d] and k, v of shape [B, H_kv, Nk, d]")
     B, H, N, d = q.shape
-    if (k.shape != v.shape or k.shape[0] != B or k.shape[2:] != q.shape[2:]
+    if (k.shape != v.shape or k.shape[0] != B or k.shape[3] != d
             or k.shape[1] < 1 or H % k.shape[1]):
-        raise ValueError(f"q, k, v shapes do not fit [B, H, N, d] / [B, H_kv, N, d] with H a multiple "
+        raise ValueError(f"q, k, v shapes do not fit [B, H, N, d] / [B, H_kv, Nk, d] with H a multiple "
                          f"of H_kv: {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)}")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
@@ -60,7 +61,7 @@ def _check_qkv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor):
             raise ValueError(f"{name} must be contiguous [B, H, N, d]")
     if k.device != q.device or v.device != q.device:
         raise ValueError("q, k, v must be on one device")
-    return B, H, k.shape[1], N, d
+    return B, H, k.shape[1], N, k.shape[2], d
 
 
 def _stream_handle(device: torch.device) -> int:
@@ -73,11 +74,12 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
     """O = softmax(scale * Q K^T (+ causal mask)) V and L = logsumexp (fp32).
 
     q: contiguous CUDA tensor [B, H, N, d] (bf16, fp16 or fp32); k, v:
-    [B, H_kv, N, d] with H a multiple of H_kv (grouped-query attention when
-    H_kv < H: query head h uses key/value head h // (H // H_kv)).
+    [B, H_kv, Nk, d] with H a multiple of H_kv (grouped-query attention when
+    H_kv < H: query head h uses key/value head h // (H // H_kv)); with
+    causal, key j is visible to query i iff j <= i.
     Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).
     """
-    B, H, H_kv, N, d = _check_qkv(q, k, v)
+    B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
@@ -85,21 +87,25 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     with torch.cuda.device(q.device):
-        if H_kv == H:
+        if H_kv == H and Nk == N:
             _native.check(_native.lib().fa2_forward(
                 q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                 B, H, N, d, int(bool(causal)), float(scale), _dtype_code(q),
                 _stream_handle(q.device)))
         else:
-            _native.check(_native.lib().fa2_forward_gqa(
+            _native.check(_native.lib().fa2_forward_ex(
                 q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                B, H, H_kv, N, d, int(bool(causal)), float(scale), _dtype_code(q),
+                B, H, H_kv, N, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
                 _stream_handle(q.device)))
     return out, lse
 
 
-def backward_workspace_bytes(B: int, H: int, N: int, d: int, dtype: torch.dtype) -> int:
-    return int(_native.lib().fa2_backward_workspace_bytes(B, H, N, d, _DTYPES[dtype]))
+def backward_workspace_bytes(B: int, H: int, N: int, d: int, dtype: torch.dtype,
+                             H_kv: Optional[int] = None, Nk: Optional[int] = None) -> int:
+    """Workspace bytes of backward(); H_kv and Nk default to H and N."""
+    H_kv = H if H_kv is None else H_kv
+    Nk = N if Nk is None else Nk
+    return int(_native.lib().fa2_backward_workspace_bytes_ex(B, H, H_kv, N, Nk, d, _DTYPES[dtype]))
 
 
 def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
@@ -115,7 +121,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     objects the library records at its kernel boundaries (before the D/L
     pre-pass, after it, after the main pass, after the dQ finalisation).
     """
-    B, H, H_kv, N, d = _check_qkv(q, k, v)
+    B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
         if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
@@ -123,7 +129,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    need = backward_workspace_bytes(B, H, N, d, q.dtype)
+    need = backward_workspace_bytes(B, H, N, d, q.dtype, H_kv, Nk)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     dq = torch.empty_like(q) if dq is None else dq
@@ -133,14 +139,14 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     if events is not None:
         if len(events) != 4:
             raise ValueError("events must hold four torch.cuda.Event objects")
-        if H_kv != H:
-            raise ValueError("events are supported for H_kv == H only")
+        if H_kv != H or Nk != N:
+            raise ValueError("events are supported for H_kv == H and Nk == N only")
         ev_arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
-    if H_kv != H:
+    if H_kv != H or Nk != N:
         with torch.cuda.device(q.device):
-            _native.check(_native.lib().fa2_backward_gqa(
+            _native.check(_native.lib().fa2_backward_ex(
                 q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, d,
+                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, Nk, d,
                 int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
                 workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
         return dq, dk, dv

@@ -26,12 +26,13 @@ _lock = threading.Lock()
 SIGNATURES = {
     "fa2_forward": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5
                     + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
-    "fa2_forward_gqa": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 6
-                        + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
+    "fa2_forward_ex": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7
+                       + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "fa2_backward_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 5),
-    "fa2_backward_gqa": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 6
-                         + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
-                            ctypes.c_void_p]),
+    "fa2_backward_workspace_bytes_ex": (ctypes.c_size_t, [ctypes.c_int] * 7),
+    "fa2_backward_ex": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7
+                        + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                           ctypes.c_void_p]),
     "fa2_backward": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                      + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                         ctypes.c_void_p]),

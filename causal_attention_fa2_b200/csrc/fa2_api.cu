@@ -140,7 +140,7 @@ constexpr bool use_two_tile_forward() {
 
 template <int ES, int D, bool F16 = false>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                          int H, int H_kv, int N, int causal, float scale, fa2_dtype dtype,
+                          int H, int H_kv, int N, int Nk, int causal, float scale, fa2_dtype dtype,
                           cudaStream_t stream, uint32_t* status) {
     using Cfg = FwdCfg<ES, D>;
     const int BH = B * H;
@@ -148,18 +148,20 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     CUtensorMap mq, mk, mv, mo;
     fa2_status st;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
-    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH_kv)) != FA2_OK) return st;
-    if ((st = make_maps_mnmajor<ES, D>(&mv, v, dtype, N, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, Nk, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_mnmajor<ES, D>(&mv, v, dtype, Nk, BH_kv)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mo, o, dtype, N, BH)) != FA2_OK) return st;
     FwdParams p;
     p.lse = lse;
     p.status = status;
     p.N = N;
+    p.Nk = Nk;
     p.BH = BH;
     p.H = H;
     p.H_kv = H_kv;
     p.group = H / H_kv;
     p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.n_tiles_k = (Nk + kTileRows - 1) / kTileRows;
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
@@ -181,14 +183,14 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
 
 template <int ES, bool F16 = false>
 fa2_status dispatch_forward(int d, const void* q, const void* k, const void* v, void* o,
-                            float* lse, int B, int H, int H_kv, int N, int causal, float scale,
+                            float* lse, int B, int H, int H_kv, int N, int Nk, int causal, float scale,
                             fa2_dtype dtype, cudaStream_t stream, uint32_t* status) {
     switch (d) {
-        case 16: return launch_forward<ES, 16, F16>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, stream, status);
-        case 32: return launch_forward<ES, 32, F16>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, stream, status);
-        case 64: return launch_forward<ES, 64, F16>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, stream, status);
-        case 80: return launch_forward<ES, 80, F16>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, stream, status);
-        case 128: return launch_forward<ES, 128, F16>(q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, stream, status);
+        case 16: return launch_forward<ES, 16, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
+        case 32: return launch_forward<ES, 32, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
+        case 64: return launch_forward<ES, 64, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
+        case 80: return launch_forward<ES, 80, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
+        case 128: return launch_forward<ES, 128, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
         default: return FA2_ERR_UNSUPPORTED_HEAD_DIM;
     }
 }
@@ -196,7 +198,7 @@ fa2_status dispatch_forward(int d, const void* q, const void* k, const void* v, 
 template <int ES, int D, bool F16 = false>
 fa2_status launch_backward_t(const void* q, const void* k, const void* v, const void* o,
                              const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                             int B, int H, int H_kv, int N, int causal, float scale, fa2_dtype dtype,
+                             int B, int H, int H_kv, int N, int Nk, int causal, float scale, fa2_dtype dtype,
                              uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                              uint32_t* status, unsigned long long timeout_ns,
                              void* const* events) {
@@ -220,30 +222,32 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
     const int BH_kv = B * H_kv;
-    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, N, BH_kv)) != FA2_OK) return st;
-    if ((st = make_maps_kmajor<ES, D>(&mv, v, dtype, N, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, Nk, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mv, v, dtype, Nk, BH_kv)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdo, dout, dtype, N, BH)) != FA2_OK) return st;
-    if ((st = make_maps_kmajor<ES, D>(&mdk, dk, dtype, N, BH_kv)) != FA2_OK) return st;
-    if ((st = make_maps_kmajor<ES, D>(&mdv, dv, dtype, N, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdk, dk, dtype, Nk, BH_kv)) != FA2_OK) return st;
+    if ((st = make_maps_kmajor<ES, D>(&mdv, dv, dtype, Nk, BH_kv)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdq, dq, dtype, N, BH)) != FA2_OK) return st;
     BwdParams p;
     p.l2 = l2;
     p.dvec = dvec;
     p.status = status;
     p.N = N;
+    p.Nk = Nk;
     p.BH = BH;
     p.H = H;
     p.H_kv = H_kv;
     p.group = H / H_kv;
     p.BH_kv = B * H_kv;
     p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.n_tiles_k = (Nk + kTileRows - 1) / kTileRows;
     p.n_pad = ws.n_pad;
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
-    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(p.BH_kv);
+    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
     // 2. dK, dV: key/value-tile-outer pass.
     {
@@ -267,7 +271,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
 template <int D>
 fa2_status launch_backward32_t(const void* q, const void* k, const void* v, const void* o,
                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                               int B, int H, int H_kv, int N, int causal, float scale, uint8_t* ws_base,
+                               int B, int H, int H_kv, int N, int Nk, int causal, float scale, uint8_t* ws_base,
                                const BwdWorkspace& ws, cudaStream_t stream, uint32_t* status,
                                unsigned long long timeout_ns, void* const* events) {
     using Cfg = Bwd32Cfg<D>;
@@ -291,7 +295,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     fa2_bwd32_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
         static_cast<const float*>(q), static_cast<const float*>(o), static_cast<const float*>(dout),
         lse, qr, dor, l2, dvec, N, ws.n_pad, rows);
-    const size_t kv4 = static_cast<size_t>(B) * H_kv * N * D / 4;   // D is a multiple of 4
+    const size_t kv4 = static_cast<size_t>(B) * H_kv * Nk * D / 4;  // D is a multiple of 4
     const unsigned round_grid = static_cast<unsigned>((kv4 + 255) / 256 < 4096 ? (kv4 + 255) / 256 : 4096);
     fa2_round_tf32_kernel<<<round_grid, 256, 0, stream>>>(static_cast<const float4*>(k), reinterpret_cast<float4*>(kr), kv4);
     fa2_round_tf32_kernel<<<round_grid, 256, 0, stream>>>(static_cast<const float4*>(v), reinterpret_cast<float4*>(vr), kv4);
@@ -302,38 +306,41 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     dout = dor;
     // q, dout, dq have B*H heads; k, v, dk, dv B*H_kv.
     const int BH_kv = B * H_kv;
-    auto kmap = [&](CUtensorMap* m, const void* ptr, int box_rows, int heads) {
-        return make_map(m, ptr, dt, D, N, heads, G::kBoxK, G::kRowBK, false, box_rows);
+    // Query-side tensors (q, dout, dq): B*H heads of N rows; key-side (k, v, dk, dv): B*H_kv of Nk.
+    auto kmap = [&](CUtensorMap* m, const void* ptr, int box_rows, int heads, int rows) {
+        return make_map(m, ptr, dt, D, rows, heads, G::kBoxK, G::kRowBK, false, box_rows);
     };
-    auto mnmap = [&](CUtensorMap* m, const void* ptr, int box_rows, int heads) {
-        return make_map(m, ptr, dt, D, N, heads, G::kBoxMN, G::kRowBMN, true, box_rows);
+    auto mnmap = [&](CUtensorMap* m, const void* ptr, int box_rows, int heads, int rows) {
+        return make_map(m, ptr, dt, D, rows, heads, G::kBoxMN, G::kRowBMN, true, box_rows);
     };
     BwdParams p;
     p.l2 = l2;
     p.dvec = dvec;
     p.status = status;
     p.N = N;
+    p.Nk = Nk;
     p.BH = BH;
     p.H = H;
     p.H_kv = H_kv;
     p.group = H / H_kv;
     p.BH_kv = BH_kv;
     p.n_tiles = (N + kTileRows - 1) / kTileRows;
+    p.n_tiles_k = (Nk + kTileRows - 1) / kTileRows;
     p.n_pad = ws.n_pad;
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
-    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(p.BH_kv);
+    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
     {
         constexpr int W = Cfg::kWkv;
         CUtensorMap mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv;
-        if ((st = kmap(&mqk, q, W, BH)) != FA2_OK || (st = mnmap(&mqmn, q, W, BH)) != FA2_OK ||
-            (st = kmap(&mk, k, kTileRows, BH_kv)) != FA2_OK || (st = kmap(&mv, v, kTileRows, BH_kv)) != FA2_OK ||
-            (st = kmap(&mdok, dout, W, BH)) != FA2_OK || (st = mnmap(&mdomn, dout, W, BH)) != FA2_OK ||
-            (st = kmap(&mdk, dk, kTileRows, BH_kv)) != FA2_OK || (st = kmap(&mdv, dv, kTileRows, BH_kv)) != FA2_OK)
+        if ((st = kmap(&mqk, q, W, BH, N)) != FA2_OK || (st = mnmap(&mqmn, q, W, BH, N)) != FA2_OK ||
+            (st = kmap(&mk, k, kTileRows, BH_kv, Nk)) != FA2_OK || (st = kmap(&mv, v, kTileRows, BH_kv, Nk)) != FA2_OK ||
+            (st = kmap(&mdok, dout, W, BH, N)) != FA2_OK || (st = mnmap(&mdomn, dout, W, BH, N)) != FA2_OK ||
+            (st = kmap(&mdk, dk, kTileRows, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdv, dv, kTileRows, BH_kv, Nk)) != FA2_OK)
             return st;
         auto kern = fa2_bwd32_dkdv_kernel<D>;
         if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
@@ -343,9 +350,9 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     {
         constexpr int W = Cfg::kWq;
         CUtensorMap mq, mdo, mkk, mkmn, mvk, mdq;
-        if ((st = kmap(&mq, q, kTileRows, BH)) != FA2_OK || (st = kmap(&mdo, dout, kTileRows, BH)) != FA2_OK ||
-            (st = kmap(&mkk, k, W, BH_kv)) != FA2_OK || (st = mnmap(&mkmn, k, W, BH_kv)) != FA2_OK ||
-            (st = kmap(&mvk, v, W, BH_kv)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows, BH)) != FA2_OK)
+        if ((st = kmap(&mq, q, kTileRows, BH, N)) != FA2_OK || (st = kmap(&mdo, dout, kTileRows, BH, N)) != FA2_OK ||
+            (st = kmap(&mkk, k, W, BH_kv, Nk)) != FA2_OK || (st = mnmap(&mkmn, k, W, BH_kv, Nk)) != FA2_OK ||
+            (st = kmap(&mvk, v, W, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows, BH, N)) != FA2_OK)
             return st;
         auto kern = fa2_bwd32_dq_kernel<D>;
         if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
@@ -357,19 +364,19 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
 
 fa2_status launch_backward(const void* q, const void* k, const void* v, const void* o,
                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                           int H, int H_kv, int N, int d, int causal, float scale, fa2_dtype dtype,
+                           int H, int H_kv, int N, int Nk, int d, int causal, float scale, fa2_dtype dtype,
                            uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                            uint32_t* status, unsigned long long timeout_ns, void* const* events) {
 #define FA2_BWD_CASE(DD)                                                                      \
     case DD:                                                                                  \
         if (dtype == FA2_FP32)                                                                \
-            return launch_backward32_t<DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, causal, \
+            return launch_backward32_t<DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, causal, \
                                            scale, ws_base, ws, stream, status, timeout_ns, events); \
         if (dtype == FA2_FP16)                                                                \
-            return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, \
+            return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, \
                                                   causal, scale, dtype, ws_base, ws, stream,    \
                                                   status, timeout_ns, events);                  \
-        return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, causal, \
+        return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, causal, \
                                         scale, dtype, ws_base, ws, stream, status, timeout_ns, events);
     switch (d) {
         FA2_BWD_CASE(16)
@@ -394,12 +401,21 @@ fa2_status check_heads(int H, int H_kv) {
     return (H_kv >= 1 && H_kv <= H && H % H_kv == 0) ? FA2_OK : FA2_ERR_BAD_SHAPE;
 }
 
+// Key/value length: the same bounds as the query length.
+fa2_status check_keys(int B, int H_kv, int Nk) {
+    if (Nk < 1 || Nk > kMaxN) return FA2_ERR_BAD_SHAPE;
+    const long long tiles = (Nk + kTileRows - 1) / kTileRows;
+    if (tiles * B * H_kv > (1ll << 31) - 1) return FA2_ERR_BAD_SHAPE;
+    return FA2_OK;
+}
+
 fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                        int H, int H_kv, int N, int d, int causal, float scale, fa2_dtype dtype,
-                        fa2_stream_t stream) {
+                        int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                        fa2_dtype dtype, fa2_stream_t stream) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
+    if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
@@ -409,33 +425,34 @@ fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, fl
     if ((st = init_device(&dev, &status)) != FA2_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == FA2_BF16)
-        return dispatch_forward<2>(d, q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, s, status);
+        return dispatch_forward<2>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
     if (dtype == FA2_FP16)
-        return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, s, status);
-    return dispatch_forward<4>(d, q, k, v, o, lse, B, H, H_kv, N, causal, scale, dtype, s, status);
+        return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
+    return dispatch_forward<4>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
 }
 
 fa2_status backward_impl(const void* q, const void* k, const void* v, const void* o,
                          const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                         int H, int H_kv, int N, int d, int causal, float scale, fa2_dtype dtype,
-                         void* workspace, size_t workspace_bytes, fa2_stream_t stream,
-                         void* const* events) {
+                         int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                         fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                         fa2_stream_t stream, void* const* events) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
+    if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4) || !aligned(workspace, 256))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H_kv, Nk, d, dtype == FA2_FP32 ? 4 : 2);
     if (workspace_bytes < ws.total) return FA2_ERR_WORKSPACE_TOO_SMALL;
     int dev;
     uint32_t* status;
     if ((st = init_device(&dev, &status)) != FA2_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, causal, scale,
+    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                            dtype, static_cast<uint8_t*>(workspace), ws, s, status,
                            kDefaultTimeoutNs, events);
 }
@@ -448,18 +465,26 @@ extern "C" {
 fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                        int H, int N, int d, int causal, float scale, fa2_dtype dtype,
                        fa2_stream_t stream) {
-    return forward_impl(q, k, v, o, lse, B, H, H, N, d, causal, scale, dtype, stream);
+    return forward_impl(q, k, v, o, lse, B, H, H, N, N, d, causal, scale, dtype, stream);
 }
 
-fa2_status fa2_forward_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
-                           int B, int H, int H_kv, int N, int d, int causal, float scale,
-                           fa2_dtype dtype, fa2_stream_t stream) {
-    return forward_impl(q, k, v, o, lse, B, H, H_kv, N, d, causal, scale, dtype, stream);
+fa2_status fa2_forward_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                          int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                          fa2_dtype dtype, fa2_stream_t stream) {
+    return forward_impl(q, k, v, o, lse, B, H, H_kv, N, Nk, d, causal, scale, dtype, stream);
 }
 
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype) {
     if (check_common(B, H, N, d, 0, 1.f, dtype) != FA2_OK) return 0;
-    return bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2).total;
+    return bwd_workspace_layout(B * H, N, B * H, N, d, dtype == FA2_FP32 ? 4 : 2).total;
+}
+
+size_t fa2_backward_workspace_bytes_ex(int B, int H, int H_kv, int N, int Nk, int d,
+                                       fa2_dtype dtype) {
+    if (check_common(B, H, N, d, 0, 1.f, dtype) != FA2_OK || check_heads(H, H_kv) != FA2_OK ||
+        check_keys(B, H_kv, Nk) != FA2_OK)
+        return 0;
+    return bwd_workspace_layout(B * H, N, B * H_kv, Nk, d, dtype == FA2_FP32 ? 4 : 2).total;
 }
 
 fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const void* o,
@@ -467,7 +492,7 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
                               int B, int H, int N, int d, int causal, float scale,
                               fa2_dtype dtype, void* workspace, size_t workspace_bytes,
                               fa2_stream_t stream, void* const* events) {
-    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, causal, scale, dtype,
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, N, d, causal, scale, dtype,
                          workspace, workspace_bytes, stream, events);
 }
 
@@ -475,16 +500,16 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                         int H, int N, int d, int causal, float scale, fa2_dtype dtype,
                         void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
-    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, causal, scale, dtype,
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, N, d, causal, scale, dtype,
                          workspace, workspace_bytes, stream, nullptr);
 }
 
-fa2_status fa2_backward_gqa(const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                            int B, int H, int H_kv, int N, int d, int causal, float scale,
-                            fa2_dtype dtype, void* workspace, size_t workspace_bytes,
-                            fa2_stream_t stream) {
-    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, d, causal, scale,
+fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                           int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                           fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                           fa2_stream_t stream) {
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                          dtype, workspace, workspace_bytes, stream, nullptr);
 }
 
@@ -573,14 +598,14 @@ extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const v
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
     if (ws.total > kNoAllocScratchBytes) return FA2_ERR_SCRATCH_TOO_SMALL;
     int dev;
     uint32_t* status;
     if ((st = init_device(&dev, &status)) != FA2_OK) return st;
     unsigned char* scratch = nullptr;
     if ((st = noalloc_scratch(dev, &scratch)) != FA2_OK) return st;
-    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, d, causal, scale, dtype,
+    return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, N, d, causal, scale, dtype,
                            scratch, ws, reinterpret_cast<cudaStream_t>(stream), status,
                            kDefaultTimeoutNs, nullptr);
 }

@@ -40,8 +40,9 @@
 namespace fa2 {
 
 // Workspace carved out of the caller's buffer (every region 256-byte aligned):
-// L*log2(e) and D, fp32, [BH][n_pad]; for 4-byte inputs also copies of q, k,
-// v and dout rounded to TF32, [BH][N][d] each (offsets 0 when absent).
+// L*log2(e) and D, fp32, [BH][n_pad]; for 4-byte inputs also copies of q and
+// dout ([BH][N][d]) and of k and v ([BH_kv][Nk][d]) rounded to TF32 (offsets 0
+// when absent).
 struct BwdWorkspace {
     size_t l2_off, d_off, q_off, k_off, v_off, do_off, total;
     int n_pad;
@@ -49,7 +50,7 @@ struct BwdWorkspace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-inline BwdWorkspace bwd_workspace_layout(int BH, int N, int d, int elem_bytes) {
+inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d, int elem_bytes) {
     BwdWorkspace w;
     w.n_pad = (N + kTileRows - 1) / kTileRows * kTileRows;
     const size_t vec = align256(static_cast<size_t>(BH) * w.n_pad * sizeof(float));
@@ -58,12 +59,13 @@ inline BwdWorkspace bwd_workspace_layout(int BH, int N, int d, int elem_bytes) {
     w.total = 2 * vec;
     w.q_off = w.k_off = w.v_off = w.do_off = 0;
     if (elem_bytes == 4) {
-        const size_t t = align256(static_cast<size_t>(BH) * N * d * sizeof(float));
+        const size_t tq = align256(static_cast<size_t>(BH) * N * d * sizeof(float));
+        const size_t tk = align256(static_cast<size_t>(BH_kv) * Nk * d * sizeof(float));
         w.q_off = w.total;
-        w.k_off = w.q_off + t;
-        w.v_off = w.k_off + t;
-        w.do_off = w.v_off + t;
-        w.total = w.do_off + t;
+        w.k_off = w.q_off + tq;
+        w.v_off = w.k_off + tk;
+        w.do_off = w.v_off + tk;
+        w.total = w.do_off + tq;
     }
     return w;
 }
@@ -130,7 +132,8 @@ struct BwdParams {
     const float* l2;       // [BH][n_pad]  L * log2(e), +inf past N
     const float* dvec;     // [BH][n_pad]  D, 0 past N
     uint32_t* status;
-    int N, BH, n_tiles, n_pad, causal;
+    int N, BH, n_tiles, n_pad, causal;   // query length, B * H, query tiles, padded rows
+    int Nk, n_tiles_k;                   // key/value length and tiles
     int H, H_kv, group, BH_kv;   // query heads, key/value heads, H / H_kv, B * H_kv
     float scale_log2;      // scale * log2(e)
     float scale;
@@ -202,7 +205,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int kv_tile = item / p.BH_kv;
     const int bh = item - kv_tile * p.BH_kv;            // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
-    const int n_q = p.n_tiles - i_begin;                // query tiles per query head
+    // Query tiles per query head; none when no query reaches this key tile
+    // (causal, keys longer than queries): then dK = dV = 0 is written.
+    const int n_q = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;
     const int n_it = n_q * p.group;                     // (query head, query tile) steps
     const int kv_row0 = kv_tile * kTileRows;
     // Step it: query tile i_begin + it % n_q of the it / n_q-th query head of the group.
@@ -240,7 +245,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && n_it > 0) {
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_do);
             ptx::mbar_arrive_expect_tx(&bar_kv_full, 2 * TB);
@@ -276,7 +281,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && n_it > 0) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_kv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t k_addr = ptx::smem_addr(sK);
@@ -341,18 +346,20 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // key row inside the tile
         const int qc0 = 64 * g;
-        const bool key_valid = kv_row0 + r < p.N;
+        const bool key_valid = kv_row0 + r < p.Nk;
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
         // Offset of step it's L / D values for this group's 64 query columns.
         auto vec_base = [&](int it) {
             return static_cast<size_t>(q_head_of(it)) * p.n_pad + static_cast<size_t>(q_tile_of(it)) * kTileRows + qc0;
         };
-        float nl2[2], nd[2];
+        float nl2[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
+        if (n_it > 0) {
 #pragma unroll
-        for (int m = 0; m < 2; ++m) {
-            nl2[m] = p.l2[vec_base(0) + lane + 32 * m];
-            nd[m] = p.dvec[vec_base(0) + lane + 32 * m];
+            for (int m = 0; m < 2; ++m) {
+                nl2[m] = p.l2[vec_base(0) + lane + 32 * m];
+                nd[m] = p.dvec[vec_base(0) + lane + 32 * m];
+            }
         }
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
@@ -443,8 +450,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
         }
-        // ---------------- epilogue: dV (group 0) / dK (group 1) -> shared memory -> TMA store.
-        if (ok) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
+        // ---------------- epilogue: dV (group 0) / dK (group 1) -> shared memory -> TMA store
+        // (zeros when no query reaches this key tile).
+        if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
         uint8_t* out_stage = g == 0 ? sV : sK;
         if (ok) {
             ptx::tc_fence_after();
@@ -452,9 +460,11 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float mul = g == 0 ? 1.f : p.scale;
 #pragma unroll
             for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
-                uint32_t u[16];
-                ptx::tmem_ld16(lane_base + col + c0, u);
-                ptx::tmem_wait_ld();
+                uint32_t u[16] = {};
+                if (n_it > 0) {
+                    ptx::tmem_ld16(lane_base + col + c0, u);
+                    ptx::tmem_wait_ld();
+                }
 #pragma unroll
                 for (int h8 = 0; h8 < 2; ++h8) {
                     const int cc = c0 + 8 * h8;
@@ -532,7 +542,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int rank = item / p.BH;
     const int bh = item - rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
-    const int n_kv = p.causal ? (q_tile + 1) : p.n_tiles;
+    // Key tiles this query tile sees (causal: key index <= query index).
+    const int n_kv = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
     const int q_row0 = q_tile * kTileRows;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
@@ -670,7 +681,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
             const bool diag = p.causal && (j == q_tile);
-            const int kv_valid = p.N - j * kTileRows - kc0;   // this group's key columns < N
+            const int kv_valid = p.Nk - j * kTileRows - kc0;  // this group's key columns < Nk
             // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14)
             if (!ptx::mbar_wait(&bar_s_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();

@@ -187,14 +187,18 @@ __device__ __forceinline__ void bwd32_ds_inplace(uint32_t dp_col, const uint32_t
 }
 
 // 128 x D fp32 accumulator in TMEM (this thread's row r) times `mul` -> the
-// K-major staging layout of an fp32 tile in shared memory.
+// K-major staging layout of an fp32 tile in shared memory; zeros instead when
+// `zero` (nothing was accumulated).
 template <class G>
-__device__ __forceinline__ void bwd32_stage_rows(uint32_t acc_col, int r, float mul, uint8_t* stage) {
+__device__ __forceinline__ void bwd32_stage_rows(uint32_t acc_col, int r, float mul, uint8_t* stage,
+                                                 bool zero = false) {
 #pragma unroll
     for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
-        uint32_t u[16];
-        ptx::tmem_ld16(acc_col + c0, u);
-        ptx::tmem_wait_ld();
+        uint32_t u[16] = {};
+        if (!zero) {
+            ptx::tmem_ld16(acc_col + c0, u);
+            ptx::tmem_wait_ld();
+        }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
             const int col = c0 + 4 * q4;
@@ -260,9 +264,11 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     const int kv_tile = item / p.BH_kv;
     const int bh = item - kv_tile * p.BH_kv;            // key/value head
     const int kv_row0 = kv_tile * kTileRows;
-    const int n_sub = (p.N + W - 1) / W;
+    const int n_sub = (p.N + W - 1) / W;                // query sub-tiles
     const int sub_begin = p.causal ? kv_row0 / W : 0;
-    const int n_q = n_sub - sub_begin;                  // sub-tiles per query head
+    // Sub-tiles per query head; none when no query reaches this key tile
+    // (causal, keys longer than queries): then dK = dV = 0 is written.
+    const int n_q = n_sub > sub_begin ? n_sub - sub_begin : 0;
     const int n_it = n_q * p.group;                     // (query head, sub-tile) steps
     auto q_row_of = [&](int it) { return (sub_begin + it % n_q) * W; };
     auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
@@ -294,7 +300,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && n_it > 0) {
             ptx::prefetch_tmap(&tm_qk);
             ptx::prefetch_tmap(&tm_qmn);
             ptx::prefetch_tmap(&tm_dok);
@@ -330,7 +336,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && n_it > 0) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, W, false, false);
             constexpr uint32_t idesc_kv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t k_addr = ptx::smem_addr(sK);
@@ -389,7 +395,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         // ------------------------------------------------ P / dS warpgroup
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // key row inside the tile
-        const bool key_valid = kv_row0 + r < p.N;
+        const bool key_valid = kv_row0 + r < p.Nk;
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
         bool ok = true;
@@ -431,11 +437,11 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
         }
         // ---------------- epilogue: dV -> sV, dK * scale -> sK, then TMA stores.
-        if (ok) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
+        if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDV, r, 1.f, sV);
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sK);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDV, r, 1.f, sV, n_it == 0);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sK, n_it == 0);
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -503,7 +509,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int bh = item - rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
     const int q_row0 = q_tile * kTileRows;
-    const int n_sub = (p.N + W - 1) / W;
+    const int n_sub = (p.Nk + W - 1) / W;               // key sub-tiles
     const int lim = (q_row0 + kTileRows) / W;
     const int n_kv = p.causal ? (lim < n_sub ? lim : n_sub) : n_sub;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
@@ -632,7 +638,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int j = 0; j < n_kv; ++j) {
             const int k0 = j * W;
             const bool mask = p.causal && k0 + W - 1 > q_row0;   // some key follows some query
-            const int kv_valid = p.N - k0;                          // key columns < N
+            const int kv_valid = p.Nk - k0;                         // key columns < Nk
             // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14), kept in registers
             if (!ptx::mbar_wait(&bar_s_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();

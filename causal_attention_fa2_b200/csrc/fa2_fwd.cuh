@@ -50,9 +50,11 @@ namespace fa2 {
 struct FwdParams {
     float* lse;            // [BH][N] natural-log logsumexp
     uint32_t* status;      // device status word
-    int N;                 // sequence length (queries = keys)
+    int N;                 // query sequence length
+    int Nk;                // key/value sequence length
     int BH;                // batch * heads
-    int n_tiles;           // ceil(N / 128)
+    int n_tiles;           // ceil(N / 128): query tiles
+    int n_tiles_k;         // ceil(Nk / 128): key tiles
     int H, H_kv, group;    // query heads, key/value heads, H / H_kv
     int causal;
     float scale_log2;      // scale * log2(e)
@@ -131,7 +133,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int tile_rank = item / p.BH;
     const int bh = item - tile_rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - tile_rank) : tile_rank;
-    const int n_kv = p.causal ? (q_tile + 1) : p.n_tiles;
+    // Key tiles this query tile sees (causal: key index <= query index).
+    const int n_kv = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
     const int q_row0 = q_tile * kTileRows;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
@@ -273,7 +276,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             // Mask: causal diagonal tile (key > query), or keys past N.
             const bool diag = p.causal && (j == q_tile);
-            const int kv_valid = p.N - j * kTileRows;
+            const int kv_valid = p.Nk - j * kTileRows;
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 128; ++c) {

@@ -92,7 +92,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
                 for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(u[c]);
             }
         }
-        const int kv_valid = p.N - j * kTileRows;
+        const int kv_valid = p.Nk - j * kTileRows;
         if (p.causal && j == q_tile) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
@@ -256,8 +256,9 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int pair = p.causal ? (n_pairs - 1 - rank) : rank;
     const int tile[2] = {2 * pair, 2 * pair + 1};
     const bool has_b = tile[1] < p.n_tiles;
-    const int n_kv_t[2] = {p.causal ? tile[0] + 1 : p.n_tiles,
-                           has_b ? (p.causal ? tile[1] + 1 : p.n_tiles) : 0};
+    // Key tiles each query tile sees (causal: key index <= query index).
+    const int n_kv_t[2] = {p.causal ? min(tile[0] + 1, p.n_tiles_k) : p.n_tiles_k,
+                           has_b ? (p.causal ? min(tile[1] + 1, p.n_tiles_k) : p.n_tiles_k) : 0};
     const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 

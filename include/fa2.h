@@ -92,17 +92,24 @@ fa2_status fa2_forward(const void* q, const void* k, const void* v, void* o, flo
                        fa2_dtype dtype, fa2_stream_t stream);
 
 /*
- * Grouped-query attention (the "LLM FLOPs Computation" page, section
- * Extension: GQA): H query heads share H_kv key/value heads, query head h of a
- * batch using key/value head h / (H / H_kv); H_kv = H is fa2_forward and
- * H_kv = 1 is multi-query attention.
- *   q, o   [B, H, N, d];  k, v  [B, H_kv, N, d];  lse [B, H, N] float32
- * H must be a multiple of H_kv (else FA2_ERR_BAD_SHAPE).  Other arguments,
- * results and errors are those of fa2_forward.
+ * The general forward: grouped-query attention and different query and key
+ * lengths.
+ *   - H query heads share H_kv key/value heads (the "LLM FLOPs Computation"
+ *     page, section Extension: GQA): query head h of a batch uses key/value
+ *     head h / (H / H_kv); H_kv = H is multi-head, H_kv = 1 multi-query
+ *     attention.  H must be a multiple of H_kv.
+ *   - N query rows attend to Nk key/value rows (the handout's Algorithm 1
+ *     takes N_q and N_k separately, section 4.2.2).  With causal = 1 key j is
+ *     visible to query i iff j <= i (the same index comparison as for
+ *     N_q = N_k), so keys at or past N are seen by no query.
+ *   q, o   [B, H, N, d];  k, v  [B, H_kv, Nk, d];  lse [B, H, N] float32
+ * fa2_forward(...) is fa2_forward_ex(..., H_kv = H, N, Nk = N, ...).  Shapes
+ * out of range (H not a multiple of H_kv, Nk < 1 or > 2^24) give
+ * FA2_ERR_BAD_SHAPE; otherwise as fa2_forward.
  */
-fa2_status fa2_forward_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
-                           int B, int H, int H_kv, int N, int d, int causal, float scale,
-                           fa2_dtype dtype, fa2_stream_t stream);
+fa2_status fa2_forward_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                          int B, int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                          fa2_dtype dtype, fa2_stream_t stream);
 
 /*
  * Bytes of device workspace fa2_backward needs for these sizes: the fp32 D
@@ -112,6 +119,14 @@ fa2_status fa2_forward_gqa(const void* q, const void* k, const void* v, void* o,
  * bytes).  Returns 0 for arguments fa2_backward would reject.
  */
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype);
+
+/*
+ * Workspace of fa2_backward_ex: as fa2_backward_workspace_bytes, except that
+ * the FA2_FP32 copies of k and v have B * H_kv * Nk * d elements.  Returns 0
+ * for arguments fa2_backward_ex would reject.
+ */
+size_t fa2_backward_workspace_bytes_ex(int B, int H, int H_kv, int N, int Nk, int d,
+                                       fa2_dtype dtype);
 
 /*
  * Backward pass with recomputation (handout section 4.2.2, Eqs. 13-19;
@@ -133,17 +148,18 @@ fa2_status fa2_backward(const void* q, const void* k, const void* v, const void*
                         void* workspace, size_t workspace_bytes, fa2_stream_t stream);
 
 /*
- * Backward pass of fa2_forward_gqa: dq [B, H, N, d]; dk, dv [B, H_kv, N, d],
+ * Backward pass of fa2_forward_ex: dq [B, H, N, d]; dk, dv [B, H_kv, Nk, d],
  * each key/value head's gradient being the sum over the H / H_kv query heads
- * that share it (accumulated in one thread block, so still deterministic).
- * The workspace is fa2_backward_workspace_bytes(B, H, N, d, dtype) (query
- * heads).  Other arguments, results and errors are those of fa2_backward.
+ * that share it (accumulated in one thread block, so still deterministic);
+ * key rows no query sees get zero gradients.  The workspace is
+ * fa2_backward_workspace_bytes_ex(B, H, H_kv, N, Nk, d, dtype) bytes.  Other
+ * arguments, results and errors are those of fa2_backward.
  */
-fa2_status fa2_backward_gqa(const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                            int B, int H, int H_kv, int N, int d, int causal, float scale,
-                            fa2_dtype dtype, void* workspace, size_t workspace_bytes,
-                            fa2_stream_t stream);
+fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const void* o,
+                           const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                           int B, int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                           fa2_dtype dtype, void* workspace, size_t workspace_bytes,
+                           fa2_stream_t stream);
 
 /*
  * fa2_backward plus timing hooks, for profiling: identical arguments and

@@ -102,6 +102,13 @@ def test_workspace_size(fa2lib, B, H, N, d):
     expect = 2 * up(B * H * n_pad * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 2) == expect      # fp16
+    for dt in (0, 1, 2):
+        assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, H, N, N, d, dt) == \
+            fa2lib.fa2_backward_workspace_bytes(B, H, N, d, dt)
+    # fp32 with other key/value shapes: the k and v copies follow H_kv and Nk.
+    nk, hkv = N + 77, 1
+    assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, hkv, N, nk, d, 1) == \
+        expect + 2 * up(B * H * N * d * 4) + 2 * up(B * hkv * nk * d * 4)
     # fp32 inputs: plus TF32-rounded copies of q, k, v and dout.
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 1) == expect + 4 * up(B * H * N * d * 4)
     assert fa2lib.fa2_backward_workspace_bytes(B, H, N, 24, 0) == 0
@@ -120,18 +127,22 @@ def test_binding_rejects_cpu_tensors():
         fa2.forward(x, x, x)
 
 
-def test_gqa_head_validation(fa2lib):
-    """fa2_forward_gqa / fa2_backward_gqa: H must be a positive multiple of H_kv."""
+def test_ex_shape_validation(fa2lib):
+    """fa2_forward_ex / fa2_backward_ex: H must be a positive multiple of H_kv,
+    and the key length is bounded like the query length."""
     L = fa2lib
 
-    def fwd_gqa(H, H_kv):
-        return L.fa2_forward_gqa(P, P, P, P, P, 1, H, H_kv, 128, 64, 1, 0.125, 0, None)
+    def fwd_ex(H, H_kv, Nk=128):
+        return L.fa2_forward_ex(P, P, P, P, P, 1, H, H_kv, 128, Nk, 64, 1, 0.125, 0, None)
 
-    def bwd_gqa(H, H_kv):
-        return L.fa2_backward_gqa(P, P, P, P, P, P, P, P, P, 1, H, H_kv, 128, 64, 1, 0.125, 0,
-                                  P, 1 << 30, None)
+    def bwd_ex(H, H_kv, Nk=128):
+        return L.fa2_backward_ex(P, P, P, P, P, P, P, P, P, 1, H, H_kv, 128, Nk, 64, 1, 0.125, 0,
+                                 P, 1 << 30, None)
 
     for H, H_kv in ((4, 3), (4, 0), (4, 8), (6, -2)):
-        assert fwd_gqa(H, H_kv) == 2, (H, H_kv)     # FA2_ERR_BAD_SHAPE
-        assert bwd_gqa(H, H_kv) == 2, (H, H_kv)
-    assert fwd_gqa(0, 1) == 2
+        assert fwd_ex(H, H_kv) == 2, (H, H_kv)      # FA2_ERR_BAD_SHAPE
+        assert bwd_ex(H, H_kv) == 2, (H, H_kv)
+    assert fwd_ex(0, 1) == 2
+    for Nk in (0, -5, (1 << 24) + 1):
+        assert fwd_ex(4, 2, Nk) == 2, Nk
+        assert bwd_ex(4, 2, Nk) == 2, Nk

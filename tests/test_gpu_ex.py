@@ -1,10 +1,12 @@
-"""Grouped-query and multi-query attention (H query heads sharing H_kv key/value
-heads; query head h uses key/value head h // (H // H_kv)).
+"""fa2_forward_ex / fa2_backward_ex: grouped-query and multi-query attention
+(H query heads sharing H_kv key/value heads; query head h uses key/value head
+h // (H // H_kv)) and query / key lengths N != Nk (causal: key j visible to
+query i iff j <= i).
 
-Reference: the oracle run per query head with that head's shared K and V;
-dK and dV of a key/value head are the sums of the per-query-head oracle
-gradients over the query heads sharing it (the chain rule through the
-broadcast of K and V to the query heads)."""
+Reference: the oracle run per query head with that head's shared K and V
+(the oracle takes separate query and key lengths); dK and dV of a key/value
+head are the sums of the per-query-head oracle gradients over the query
+heads sharing it (the chain rule through the broadcast of K and V)."""
 import ctypes
 
 import numpy as np
@@ -17,34 +19,42 @@ from parity_util import assert_close, default_scale, to64
 pytestmark = pytest.mark.gpu
 
 CASES = [
-    # (B, H, H_kv, N, d, dtype, causal)
-    (1, 4, 2, 300, 64, "bf16", True),
-    (2, 6, 1, 256, 128, "bf16", True),      # multi-query
-    (1, 8, 4, 1000, 80, "bf16", True),
-    (1, 4, 2, 384, 128, "bf16", False),
-    (1, 4, 1, 200, 32, "fp16", True),
-    (1, 4, 2, 200, 64, "fp32", True),
-    (1, 6, 3, 160, 16, "fp32", False),
+    # (B, H, H_kv, N, Nk, d, dtype, causal)
+    (1, 4, 2, 300, 300, 64, "bf16", True),
+    (2, 6, 1, 256, 256, 128, "bf16", True),      # multi-query
+    (1, 8, 4, 1000, 1000, 80, "bf16", True),
+    (1, 4, 2, 384, 384, 128, "bf16", False),
+    (1, 4, 1, 200, 200, 32, "fp16", True),
+    (1, 4, 2, 200, 200, 64, "fp32", True),
+    (1, 6, 3, 160, 160, 16, "fp32", False),
+    # different query and key lengths
+    (1, 2, 2, 200, 333, 64, "bf16", True),       # keys past the last query: zero dK, dV
+    (1, 2, 2, 300, 129, 128, "bf16", True),
+    (2, 2, 2, 128, 1000, 64, "bf16", False),
+    (1, 4, 2, 513, 64, 80, "bf16", True),
+    (1, 2, 1, 170, 390, 32, "fp16", True),
+    (1, 2, 2, 150, 400, 64, "fp32", True),
+    (1, 2, 2, 260, 100, 128, "fp32", False),
 ]
 
 
-def _inputs(B, H, H_kv, N, d, dtype, seed):
+def _inputs(B, H, H_kv, N, Nk, d, dtype, seed):
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     dt = fa2_inputs.DTYPES[dtype]
     q = torch.randn((B, H, N, d), generator=g).to(dt)
-    k = torch.randn((B, H_kv, N, d), generator=g).to(dt)
-    v = torch.randn((B, H_kv, N, d), generator=g).to(dt)
+    k = torch.randn((B, H_kv, Nk, d), generator=g).to(dt)
+    v = torch.randn((B, H_kv, Nk, d), generator=g).to(dt)
     do = torch.randn((B, H, N, d), generator=g).to(dt)
     return q, k, v, do
 
 
 def _reference(oracle_mod, q, k, v, do, causal, scale):
     B, H, N, d = q.shape
-    H_kv = k.shape[1]
+    H_kv, Nk = k.shape[1], k.shape[2]
     grp = H // H_kv
     ref = {n: np.zeros(s) for n, s in (("o", (B, H, N, d)), ("lse", (B, H, N)), ("dq", (B, H, N, d)),
-                                         ("dk", (B, H_kv, N, d)), ("dv", (B, H_kv, N, d)))}
+                                         ("dk", (B, H_kv, Nk, d)), ("dv", (B, H_kv, Nk, d)))}
     for b in range(B):
         for h in range(H):
             hk = h // grp
@@ -57,15 +67,15 @@ def _reference(oracle_mod, q, k, v, do, causal, scale):
     return ref
 
 
-@pytest.mark.parametrize("B,H,H_kv,N,d,dtype,causal", CASES)
-def test_gqa_parity(oracle_mod, B, H, H_kv, N, d, dtype, causal):
+@pytest.mark.parametrize("B,H,H_kv,N,Nk,d,dtype,causal", CASES)
+def test_ex_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal):
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
     # (With seed 31 + N + d + H_kv the multi-query bf16 case had one dQ element
     # of query row 1 at 1.6x the bound: with two visible keys each dS_1j is
     # large and its bf16 rounding before the dQ MMA shows; recorded in the
     # design notes as a property of the 16-bit dS, not of the head mapping.)
-    q, k, v, do = _inputs(B, H, H_kv, N, d, dtype, seed=131 + N + d + H_kv)
+    q, k, v, do = _inputs(B, H, H_kv, N, Nk, d, dtype, seed=131 + N + d + H_kv + Nk)
     scale = default_scale(d)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o, lse = fa2.forward(qd, kd, vd, causal=causal, scale=scale)
@@ -73,6 +83,9 @@ def test_gqa_parity(oracle_mod, B, H, H_kv, N, d, dtype, causal):
     torch.cuda.synchronize()
     assert dk.shape == k.shape and dv.shape == v.shape
     ref = _reference(oracle_mod, q, k, v, do, causal, scale)
+    if causal and Nk > N:
+        # No query reaches keys N .. Nk-1: their gradients are exactly zero.
+        assert not dk[:, :, N:].any() and not dv[:, :, N:].any()
     # dK and dV add up `group` per-head gradients; the tolerance is the
     # per-element one of a single gradient, scaled by the group size.
     for name, got in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
@@ -89,9 +102,9 @@ def test_gqa_parity(oracle_mod, B, H, H_kv, N, d, dtype, causal):
 TOLS = {"bf16": 1e-2, "fp16": 1e-2, "fp32": 2e-3}
 
 
-def test_gqa_with_all_heads_is_mha_bitwise():
-    """fa2_forward_gqa / fa2_backward_gqa with H_kv = H give the bits of
-    fa2_forward / fa2_backward."""
+def test_ex_with_mha_shapes_is_bitwise_mha():
+    """fa2_forward_ex / fa2_backward_ex with H_kv = H and Nk = N give the bits
+    of fa2_forward / fa2_backward."""
     import causal_attention_fa2_b200 as fa2
     from causal_attention_fa2_b200 import _native
     lib = _native.lib()
@@ -104,13 +117,13 @@ def test_gqa_with_all_heads_is_mha_bitwise():
     ref = fa2.backward(q, k, v, o, lse, do, causal=True, scale=scale)
     o2, lse2 = torch.empty_like(o), torch.empty_like(lse)
     s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    assert lib.fa2_forward_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), lse2.data_ptr(),
-                               B, H, H, N, d, 1, scale, 0, s) == 0
+    assert lib.fa2_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), lse2.data_ptr(),
+                              B, H, H, N, N, d, 1, scale, 0, s) == 0
     ws = torch.empty(fa2.backward_workspace_bytes(B, H, N, d, q.dtype), dtype=torch.uint8, device=dev)
     g = [torch.empty_like(q) for _ in range(3)]
-    assert lib.fa2_backward_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                do.data_ptr(), g[0].data_ptr(), g[1].data_ptr(), g[2].data_ptr(),
-                                B, H, H, N, d, 1, scale, 0, ws.data_ptr(), ws.numel(), s) == 0
+    assert lib.fa2_backward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                               do.data_ptr(), g[0].data_ptr(), g[1].data_ptr(), g[2].data_ptr(),
+                               B, H, H, N, N, d, 1, scale, 0, ws.data_ptr(), ws.numel(), s) == 0
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
     assert all(torch.equal(a, b) for a, b in zip(ref, g))
@@ -119,7 +132,7 @@ def test_gqa_with_all_heads_is_mha_bitwise():
 def test_gqa_backward_deterministic():
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
-    q, k, v, do = (t.to(dev) for t in _inputs(2, 8, 2, 512, 128, "bf16", seed=5))
+    q, k, v, do = (t.to(dev) for t in _inputs(2, 8, 2, 512, 700, 128, "bf16", seed=5))
     o, lse = fa2.forward(q, k, v)
     g1 = fa2.backward(q, k, v, o, lse, do)
     g2 = fa2.backward(q, k, v, o, lse, do)
