@@ -259,8 +259,8 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     // 3. dQ: query-tile-outer pass.
     {
         auto kern = fa2_bwd_dq_kernel<ES, D, F16>;
-        if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+        if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
     }
     return FA2_OK;

@@ -144,7 +144,10 @@ template <int ES, int D, bool F16 = false>
 struct BwdCfg {
     using G = TileGeom<ES, D, F16>;
     static_assert(ES == 2, "the backward kernels are written for 16-bit inputs");
-    static constexpr int kThreads = 320;   // 10 warps
+    // Warp 0 TMA producer, warp 1 MMA issuer, warps 2-9 the two elementwise
+    // groups; the dQ pass adds warp 10 as a second MMA issuer.
+    static constexpr int kThreads = 320;
+    static constexpr int kThreadsDq = 352;
     static constexpr int kTile = G::kTileBytesK;
     // 227 KB minus the alignment pad and the static shared memory.
     static constexpr int kBudget = 227 * 1024 - 1024 - 9 * 1024;
@@ -153,6 +156,14 @@ struct BwdCfg {
     static constexpr int kRing = kRing0 > 3 ? 3 : kRing0;
     static_assert(kRing >= 2, "shared memory too small for the streaming rings");
     static constexpr int kSmemBytes = 1024 + 2 * kTile + 2 * kRing * kTile;
+    // dQ pass (static shared memory under 1 KB): Q, dO resident, K and V
+    // streamed.  K_j stays until dQ += dS K_j has read it, two MMA groups
+    // after S(j), so K takes the deeper ring.
+    static constexpr int kDqStream = (227 * 1024 - 1024 - 1024) / kTile - 2;
+    static constexpr int kRingK = kDqStream - 2 > 3 ? 3 : kDqStream - 2;
+    static constexpr int kRingV = kDqStream - kRingK > 3 ? 3 : kDqStream - kRingK;
+    static_assert(kRingK >= 2 && kRingV >= 2, "shared memory too small for the dQ rings");
+    static constexpr int kDqSmemBytes = 1024 + (2 + kRingK + kRingV) * kTile;
     static constexpr uint32_t kTmemCols = 512;
     // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
@@ -289,8 +300,12 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             auto q_addr = [&](int it) { return ptx::smem_addr(sQr + (it % RS) * TB); };
             auto do_addr = [&](int it) { return ptx::smem_addr(sDOr + (it % RS) * TB); };
             // S^T = K_j Q_i^T   (Eq. 13, transposed: rows are keys)
+            // Q_i / dO_i of step i >= 1 have landed once the groups report P^T / dS^T
+            // of step i-1 (one thread checks them before arriving), so only step 0
+            // waits on the loads here: each such wait stalls this thread behind its
+            // pending MMAs.
             auto issue_s = [&](int it) -> bool {
-                if (!ptx::mbar_wait(&bar_q_full[it % RS], (it / RS) & 1, &abort_flag, tmo)) return false;
+                if (it == 0 && !ptx::mbar_wait(&bar_q_full[0], 0, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
                 const uint32_t qa = q_addr(it);
 #pragma unroll
@@ -301,7 +316,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             };
             // dP^T = V_j dO_i^T   (Eq. 16, transposed)
             auto issue_dp = [&](int it) -> bool {
-                if (!ptx::mbar_wait(&bar_do_full[it % RS], (it / RS) & 1, &abort_flag, tmo)) return false;
+                if (it == 0 && !ptx::mbar_wait(&bar_do_full[0], 0, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
                 const uint32_t da = do_addr(it);
 #pragma unroll
@@ -415,7 +430,13 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_p_ready);
+            if (lane == 0) {
+                // The issuer's S^T(it+1) follows this barrier: check Q_{it+1} first.
+                if (wi == 0 && it + 1 < n_it)
+                    ok = ptx::mbar_wait(&bar_q_full[(it + 1) % RS], ((it + 1) / RS) & 1, &abort_flag, tmo);
+                if (ok) ptx::mbar_arrive(&bar_p_ready);
+            }
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
             // ---- dS^T = P^T o (dP^T - D)   (Eq. 17)
             if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -448,7 +469,13 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+            if (lane == 0) {
+                // The issuer's dP^T(it+1) follows this barrier: check dO_{it+1} first.
+                if (wi == 0 && it + 1 < n_it)
+                    ok = ptx::mbar_wait(&bar_do_full[(it + 1) % RS], ((it + 1) / RS) & 1, &abort_flag, tmo);
+                if (ok) ptx::mbar_arrive(&bar_ds_ready);
+            }
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
         }
         // ---------------- epilogue: dV (group 0) / dK (group 1) -> shared memory -> TMA store
         // (zeros when no query reaches this key tile).
@@ -505,25 +532,29 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
 // ------------------------------------------------------------------ dQ pass
 
-// One CTA per (query tile i, head).  Per key tile j the MMA issuer runs
+// One CTA per (query tile i, head).  Per key tile j the tensor core runs
 //   S(j) = Q K_j^T ; dP(j) = dO V_j^T ; dQ += dS(j) K_j   (A = dS from TMEM)
-// issuing S(j+1) as soon as both groups have read S(j), and dP(j+1) right
-// after dQ(j), so the groups' exponentials overlap the tensor core.
+// from two issuing threads: S(j+1) as soon as both groups have read S(j),
+// and dP(j+1) right after dQ(j), so the groups' exponentials overlap the
+// tensor core.  A thread that waits on an mbarrier after committing MMAs
+// stalls until those MMAs are done; with two issuers the other one's MMAs
+// keep the tensor core busy meanwhile.
 template <int ES, int D, bool F16 = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using Cfg = BwdCfg<ES, D, F16>;
     using G = typename Cfg::G;
-    constexpr int RS = Cfg::kRing;
+    constexpr int RK = Cfg::kRingK;
+    constexpr int RV = Cfg::kRingV;
     constexpr int TB = Cfg::kTile;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_qdo_full;
-    __shared__ uint64_t bar_k_full[RS], bar_k_empty[RS], bar_v_full[RS], bar_v_empty[RS];
+    __shared__ uint64_t bar_k_full[RK], bar_k_empty[RK], bar_v_full[RV], bar_v_empty[RV];
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_dp_read, bar_ds_ready;
-    __shared__ uint64_t bar_dq_done, bar_drain;
+    __shared__ uint64_t bar_dq_done, bar_drain[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
 
@@ -532,7 +563,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint8_t* sQ = smem;
     uint8_t* sDO = sQ + TB;
     uint8_t* sKr = sDO + TB;
-    uint8_t* sVr = sKr + RS * TB;
+    uint8_t* sVr = sKr + RK * TB;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -550,9 +581,11 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (threadIdx.x == 0) {
         abort_flag = 0u;
         ptx::mbar_init(&bar_qdo_full, 1);
-        for (int s = 0; s < RS; ++s) {
+        for (int s = 0; s < RK; ++s) {
             ptx::mbar_init(&bar_k_full[s], 1);
-            ptx::mbar_init(&bar_k_empty[s], 1);
+            ptx::mbar_init(&bar_k_empty[s], 2);         // released by S(j) and dQ(j)
+        }
+        for (int s = 0; s < RV; ++s) {
             ptx::mbar_init(&bar_v_full[s], 1);
             ptx::mbar_init(&bar_v_empty[s], 1);
         }
@@ -562,7 +595,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ptx::mbar_init(&bar_dp_read, 8);
         ptx::mbar_init(&bar_ds_ready, 8);
         ptx::mbar_init(&bar_dq_done, 1);
-        ptx::mbar_init(&bar_drain, 1);
+        ptx::mbar_init(&bar_drain[0], 1);
+        ptx::mbar_init(&bar_drain[1], 1);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -588,83 +622,88 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < n_kv; ++j) {
-                const int s = j % RS;
-                const uint32_t ph = ((j / RS) & 1) ^ 1;
-                if (j >= RS && !ptx::mbar_wait(&bar_k_empty[s], ph, &abort_flag, tmo)) break;
-                ptx::mbar_arrive_expect_tx(&bar_k_full[s], TB);
+                const int sk = j % RK;
+                if (j >= RK && !ptx::mbar_wait(&bar_k_empty[sk], ((j / RK) & 1) ^ 1, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_k_full[sk], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sKr + s * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
+                    ptx::tma_load_3d_hint(sKr + sk * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[sk], b * G::kBoxK, j * kTileRows, bh_kv, keep);
                 k_issued = j + 1;
-                if (j >= RS && !ptx::mbar_wait(&bar_v_empty[s], ph, &abort_flag, tmo)) break;
-                ptx::mbar_arrive_expect_tx(&bar_v_full[s], TB);
+                const int sv = j % RV;
+                if (j >= RV && !ptx::mbar_wait(&bar_v_empty[sv], ((j / RV) & 1) ^ 1, &abort_flag, tmo)) break;
+                ptx::mbar_arrive_expect_tx(&bar_v_full[sv], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sVr + s * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
+                    ptx::tma_load_3d_hint(sVr + sv * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[sv], b * G::kBoxK, j * kTileRows, bh_kv, keep);
                 v_issued = j + 1;
             }
             if (abort_flag) {
                 constexpr uint64_t kDrainNs = 20000000ull;
                 ptx::mbar_wait_drain(&bar_qdo_full, 0, kDrainNs);
-                for (int t = k_issued - 1; t >= 0 && t >= k_issued - RS; --t)
-                    ptx::mbar_wait_drain(&bar_k_full[t % RS], (t / RS) & 1, kDrainNs);
-                for (int t = v_issued - 1; t >= 0 && t >= v_issued - RS; --t)
-                    ptx::mbar_wait_drain(&bar_v_full[t % RS], (t / RS) & 1, kDrainNs);
+                for (int t = k_issued - 1; t >= 0 && t >= k_issued - RK; --t)
+                    ptx::mbar_wait_drain(&bar_k_full[t % RK], (t / RK) & 1, kDrainNs);
+                for (int t = v_issued - 1; t >= 0 && t >= v_issued - RV; --t)
+                    ptx::mbar_wait_drain(&bar_v_full[t % RV], (t / RV) & 1, kDrainNs);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 10) {
+        // ------------------------------------------------ MMA issuers
+        // Issuer 0 (warp 1): S(j) for every key tile, each as soon as both
+        // groups have read S(j-1).  Issuer 1 (warp 10): dP(0); per key tile j
+        // dQ += dS(j) K_j, then dP(j+1) (it overwrites dS(j)).  A wait stalls
+        // only the thread whose MMAs precede it, so one issuer's MMAs keep the
+        // tensor core busy while the other waits.  K_j's slot is released by
+        // both S(j) and dQ(j); V_j's by dP(j).
+        const int role = warp == 1 ? 0 : 1;
         if (lane == 0) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_dq = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr = ptx::smem_addr(sQ);
             const uint32_t do_addr = ptx::smem_addr(sDO);
-            auto k_addr = [&](int j) { return ptx::smem_addr(sKr + (j % RS) * TB); };
-            auto v_addr = [&](int j) { return ptx::smem_addr(sVr + (j % RS) * TB); };
-            // S = Q_i K_j^T   (Eq. 13)
-            auto issue_s = [&](int j) -> bool {
-                if (!ptx::mbar_wait(&bar_k_full[j % RS], (j / RS) & 1, &abort_flag, tmo)) return false;
-                ptx::tc_fence_after();
-                const uint32_t ka = k_addr(j);
-#pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_f16_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk), idesc_s, kk > 0 ? 1u : 0u);
-                ptx::mma_commit(&bar_s_full);
-                return true;
-            };
-            // dP = dO_i V_j^T   (Eq. 16)
-            auto issue_dp = [&](int j) -> bool {
-                if (!ptx::mbar_wait(&bar_v_full[j % RS], (j / RS) & 1, &abort_flag, tmo)) return false;
-                ptx::tc_fence_after();
-                const uint32_t va = v_addr(j);
-#pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_f16_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk), idesc_s, kk > 0 ? 1u : 0u);
-                ptx::mma_commit(&bar_dp_full);
-                ptx::mma_commit(&bar_v_empty[j % RS]);
-                return true;
-            };
+            auto k_addr = [&](int j) { return ptx::smem_addr(sKr + (j % RK) * TB); };
+            auto v_addr = [&](int j) { return ptx::smem_addr(sVr + (j % RV) * TB); };
+            auto wait_k = [&](int j) { return ptx::mbar_wait(&bar_k_full[j % RK], (j / RK) & 1, &abort_flag, tmo); };
             bool ok = ptx::mbar_wait(&bar_qdo_full, 0, &abort_flag, tmo);
-            if (ok) ok = issue_s(0) && issue_dp(0);
-            for (int j = 0; ok && j < n_kv; ++j) {
-                // Next scores as soon as both groups have read S(j).
-                if (j + 1 < n_kv) {
-                    if (!ptx::mbar_wait(&bar_s_read, j & 1, &abort_flag, tmo)) { ok = false; break; }
-                    if (!issue_s(j + 1)) { ok = false; break; }
-                }
-                // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
-                if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo)) { ok = false; break; }
-                ptx::tc_fence_after();
-                const uint32_t ka = k_addr(j);
+            if (role == 0) {
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    // S = Q_i K_j^T   (Eq. 13), into the score columns once S(j-1) is read.
+                    if (j > 0 && !ptx::mbar_wait(&bar_s_read, (j - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
+                    if (!wait_k(j)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t ka = k_addr(j);
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * 8, desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar_k_empty[j % RS]);
-                if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
-            }
-            if (ok) {
-                ptx::mma_commit(&bar_dq_done);
+                    for (int kk = 0; kk < G::kStepsD; ++kk)
+                        ptx::mma_f16_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk), idesc_s, kk > 0 ? 1u : 0u);
+                    ptx::mma_commit(&bar_s_full);
+                    ptx::mma_commit(&bar_k_empty[j % RK]);
+                }
             } else {
-                ptx::mma_commit(&bar_drain);
-                ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+                // dP = dO_i V_j^T   (Eq. 16)
+                auto issue_dp = [&](int j) -> bool {
+                    if (!ptx::mbar_wait(&bar_v_full[j % RV], (j / RV) & 1, &abort_flag, tmo)) return false;
+                    const uint32_t va = v_addr(j);
+#pragma unroll
+                    for (int kk = 0; kk < G::kStepsD; ++kk)
+                        ptx::mma_f16_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk), idesc_s, kk > 0 ? 1u : 0u);
+                    ptx::mma_commit(&bar_dp_full);
+                    ptx::mma_commit(&bar_v_empty[j % RV]);
+                    return true;
+                };
+                if (ok) ok = issue_dp(0);
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
+                    if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo) || !wait_k(j)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t ka = k_addr(j);
+#pragma unroll
+                    for (int kk = 0; kk < G::kStepsRows; ++kk)
+                        ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * 8, desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(&bar_k_empty[j % RK]);
+                    if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
+                }
+                if (ok) ptx::mma_commit(&bar_dq_done);
+            }
+            if (!ok) {
+                ptx::mma_commit(&bar_drain[role]);
+                ptx::mbar_wait_drain(&bar_drain[role], 0, 20000000ull);
             }
         }
     } else {
