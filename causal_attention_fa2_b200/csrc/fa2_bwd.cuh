@@ -408,19 +408,29 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&bar_s_read);
+                const float2 sl2v = make_float2(sl2, sl2);
+                if (diag || !key_valid) {
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
-                    const float4 lv = *reinterpret_cast<const float4*>(&sL2[wi][b][c]);
-                    const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
-                    float pv[4];
+                    for (int c = 0; c < 64; c += 4) {
+                        const float4 lv = *reinterpret_cast<const float4*>(&sL2[wi][b][c]);
+                        const float2 a0 = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, make_float2(-lv.x, -lv.y));
+                        const float2 a1 = ptx::fma2(make_float2(__uint_as_float(us[c + 2]), __uint_as_float(us[c + 3])), sl2v, make_float2(-lv.z, -lv.w));
+                        float pv[4] = {ptx::ex2_approx(a0.x), ptx::ex2_approx(a0.y), ptx::ex2_approx(a1.x), ptx::ex2_approx(a1.y)};
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        float pe = ptx::ex2_approx(fmaf(__uint_as_float(us[c + h]), sl2, -lq[h]));
-                        if ((diag && r > qc0 + c + h) || !key_valid) pe = 0.f;
-                        pv[h] = pe;
+                        for (int h = 0; h < 4; ++h)
+                            if ((diag && r > qc0 + c + h) || !key_valid) pv[h] = 0.f;
+                        pk[c >> 1] = G::pack2(pv[0], pv[1]);
+                        pk[(c >> 1) + 1] = G::pack2(pv[2], pv[3]);
                     }
-                    pk[c >> 1] = G::pack2(pv[0], pv[1]);
-                    pk[(c >> 1) + 1] = G::pack2(pv[2], pv[3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        const float4 lv = *reinterpret_cast<const float4*>(&sL2[wi][b][c]);
+                        const float2 a0 = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, make_float2(-lv.x, -lv.y));
+                        const float2 a1 = ptx::fma2(make_float2(__uint_as_float(us[c + 2]), __uint_as_float(us[c + 3])), sl2v, make_float2(-lv.z, -lv.w));
+                        pk[c >> 1] = G::pack2(ptx::ex2_approx(a0.x), ptx::ex2_approx(a0.y));
+                        pk[(c >> 1) + 1] = G::pack2(ptx::ex2_approx(a1.x), ptx::ex2_approx(a1.y));
+                    }
                 }
             }
             if (!ptx::mbar_wait(&bar_s_read, it & 1, &abort_flag, tmo)) { ok = false; break; }
@@ -452,13 +462,13 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) {
                     const float4 dv4 = *reinterpret_cast<const float4*>(&sDv[wi][b][c]);
-                    const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+                    const float2 nd[2] = {make_float2(-dv4.x, -dv4.y), make_float2(-dv4.z, -dv4.w)};
 #pragma unroll
                     for (int h = 0; h < 4; h += 2) {
-                        float p0, p1;
-                        G::unpack2(pk[(c + h) >> 1], p0, p1);
-                        dk[(c + h) >> 1] = G::pack2(p0 * (__uint_as_float(ud[c + h]) - dq4[h]),
-                                                            p1 * (__uint_as_float(ud[c + h + 1]) - dq4[h + 1]));
+                        float2 pp;
+                        G::unpack2(pk[(c + h) >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c + h]), __uint_as_float(ud[c + h + 1])), nd[h >> 1]));
+                        dk[(c + h) >> 1] = G::pack2(ds.x, ds.y);
                     }
                 }
             }
@@ -733,16 +743,22 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&bar_s_read);
+                const float2 sl2v = make_float2(sl2, sl2), nl2v = make_float2(-l2r, -l2r);
+                if (diag || kv_valid < 64) {
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    float pv[2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        float pe = ptx::ex2_approx(fmaf(__uint_as_float(us[c + h]), sl2, -l2r));
-                        if ((diag && kc0 + c + h > r) || c + h >= kv_valid) pe = 0.f;
-                        pv[h] = pe;
+                    for (int c = 0; c < 64; c += 2) {
+                        const float2 a = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, nl2v);
+                        float p0 = ptx::ex2_approx(a.x), p1 = ptx::ex2_approx(a.y);
+                        if ((diag && kc0 + c > r) || c >= kv_valid) p0 = 0.f;
+                        if ((diag && kc0 + c + 1 > r) || c + 1 >= kv_valid) p1 = 0.f;
+                        pk[c >> 1] = G::pack2(p0, p1);
                     }
-                    pk[c >> 1] = G::pack2(pv[0], pv[1]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const float2 a = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, nl2v);
+                        pk[c >> 1] = G::pack2(ptx::ex2_approx(a.x), ptx::ex2_approx(a.y));
+                    }
                 }
             }
             // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
@@ -757,12 +773,13 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&bar_dp_read);
+                const float2 ndv = make_float2(-dr, -dr);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    float p0, p1;
-                    G::unpack2(pk[c >> 1], p0, p1);
-                    dk[c >> 1] = G::pack2(p0 * (__uint_as_float(ud[c]) - dr),
-                                                  p1 * (__uint_as_float(ud[c + 1]) - dr));
+                    float2 pp;
+                    G::unpack2(pk[c >> 1], pp.x, pp.y);
+                    const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])), ndv));
+                    dk[c >> 1] = G::pack2(ds.x, ds.y);
                 }
             }
             if (!ptx::mbar_wait(&bar_dp_read, j & 1, &abort_flag, tmo)) { ok = false; break; }

@@ -83,14 +83,13 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
         ptx::tc_fence_after();
         float s[128];
         {
-            uint32_t u[32];
+            uint32_t u[128];
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-                ptx::tmem_ld32(s_tmem + c0, u);
-                ptx::tmem_wait_ld();
+            for (int c0 = 0; c0 < 128; c0 += 32)
+                ptx::tmem_ld32(s_tmem + c0, *reinterpret_cast<uint32_t(*)[32]>(u + c0));
+            ptx::tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; ++c) s[c0 + c] = __uint_as_float(u[c]);
-            }
+            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(u[c]);
         }
         const int kv_valid = p.Nk - j * kTileRows;
         if (p.causal && j == q_tile) {
@@ -103,15 +102,13 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
             for (int c = 0; c < 128; ++c)
                 if (c >= kv_valid) s[c] = -INFINITY;
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        float mx0 = s[0], mx1 = s[1];
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-            mx0 = fmaxf(mx0, s[c]);
-            mx1 = fmaxf(mx1, s[c + 1]);
-            mx2 = fmaxf(mx2, s[c + 2]);
-            mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 2; c < 126; c += 4) {
+            mx0 = ptx::max3(mx0, s[c], s[c + 1]);
+            mx1 = ptx::max3(mx1, s[c + 2], s[c + 3]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float mx = ptx::max3(mx0, mx1, fmaxf(s[126], s[127]));
         const float m_new = fmaxf(m_raw, mx);
         const bool raise = (m_new - m_raw) * sl2 > 8.f;   // true on the first tile
         float alpha = 1.f;
@@ -135,16 +132,17 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
         }
         l *= alpha;
         const float neg = -m_raw * sl2;
-        float rs0 = 0.f, rs1 = 0.f;
+        const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg, neg);
+        float2 rs = make_float2(0.f, 0.f);      // even / odd column sums
         // Exponentiate 32 columns at a time and store them as P right away.
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-                s[c0 + c] = ptx::ex2_approx(fmaf(s[c0 + c], sl2, neg));
-                s[c0 + c + 1] = ptx::ex2_approx(fmaf(s[c0 + c + 1], sl2, neg));
-                rs0 += s[c0 + c];
-                rs1 += s[c0 + c + 1];
+                const float2 a = ptx::fma2(make_float2(s[c0 + c], s[c0 + c + 1]), sl2v, negv);
+                s[c0 + c] = ptx::ex2_approx(a.x);
+                s[c0 + c + 1] = ptx::ex2_approx(a.y);
+                rs = ptx::add2(rs, make_float2(s[c0 + c], s[c0 + c + 1]));
             }
             if constexpr (G::kF32) {
                 uint32_t u[32];
@@ -158,7 +156,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
                 ptx::tmem_st16(s_tmem + c0 / 2, u);
             }
         }
-        l += rs0 + rs1;
+        l += rs.x + rs.y;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
