@@ -169,6 +169,14 @@ struct BwdCfg {
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
 };
 
+// TMEM column, relative to the score (or dP) block, of k-step kk of the
+// 16-bit P (or dS) A operand.  The group that owns columns [64g, 64g + 64)
+// writes its 64 values, packed two per column, to the first 32 of them, so
+// k-steps 4g .. 4g+3 read there and neither group waits for the other.
+__host__ __device__ constexpr uint32_t a_col(int kk) {
+    return static_cast<uint32_t>((kk / 4) * 64 + (kk % 4) * 8);
+}
+
 // ------------------------------------------------------------------ dK / dV pass
 
 // Per query tile i the MMA issuer runs
@@ -189,7 +197,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full;
     __shared__ uint64_t bar_q_full[RS], bar_q_empty[RS], bar_do_full[RS], bar_do_empty[RS];
-    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_dp_read, bar_p_ready, bar_ds_ready;
+    __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready;
     __shared__ uint64_t bar_dkv_full, bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
@@ -236,8 +244,6 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         ptx::mbar_init(&bar_s_full, 1);
         ptx::mbar_init(&bar_dp_full, 1);
-        ptx::mbar_init(&bar_s_read, 8);
-        ptx::mbar_init(&bar_dp_read, 8);
         ptx::mbar_init(&bar_p_ready, 8);
         ptx::mbar_init(&bar_ds_ready, 8);
         ptx::mbar_init(&bar_dkv_full, 1);
@@ -334,7 +340,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t da = do_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * 8, desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + a_col(kk), desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_do_empty[it % RS]);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
@@ -343,7 +349,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t qa = q_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * 8, desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_q_empty[it % RS]);
                 if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
             }
@@ -404,10 +410,6 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tmem_ld32(lane_base + Cfg::kColS + qc0, *reinterpret_cast<uint32_t(*)[32]>(us));
                 ptx::tmem_ld32(lane_base + Cfg::kColS + qc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(us + 32));
                 ptx::tmem_wait_ld();
-                // Both groups must have read S^T before either writes P^T over it.
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bar_s_read);
                 const float2 sl2v = make_float2(sl2, sl2);
                 if (diag || !key_valid) {
 #pragma unroll
@@ -433,10 +435,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             }
-            if (!ptx::mbar_wait(&bar_s_read, it & 1, &abort_flag, tmo)) { ok = false; break; }
-            ptx::tc_fence_after();
-            // P^T -> TMEM score columns [32g, 32g + 32), A operand of dV += P^T dO.
-            ptx::tmem_st32(lane_base + Cfg::kColS + qc0 / 2, pk);
+            // P^T -> this group's own score columns [64g, 64g + 32) (already read,
+            // so no wait on the other group), A operand of dV += P^T dO.
+            ptx::tmem_st32(lane_base + Cfg::kColS + qc0, pk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -456,9 +457,6 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0, *reinterpret_cast<uint32_t(*)[32]>(ud));
                 ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ud + 32));
                 ptx::tmem_wait_ld();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bar_dp_read);
 #pragma unroll
                 for (int c = 0; c < 64; c += 4) {
                     const float4 dv4 = *reinterpret_cast<const float4*>(&sDv[wi][b][c]);
@@ -472,10 +470,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             }
-            if (!ptx::mbar_wait(&bar_dp_read, it & 1, &abort_flag, tmo)) { ok = false; break; }
-            ptx::tc_fence_after();
-            // dS^T -> TMEM dP^T columns [128 + 32g, ...), A operand of dK += dS^T Q.
-            ptx::tmem_st32(lane_base + Cfg::kColDP + qc0 / 2, dk);
+            // dS^T -> this group's own dP^T columns [128 + 64g, ... + 32), A operand
+            // of dK += dS^T Q.
+            ptx::tmem_st32(lane_base + Cfg::kColDP + qc0, dk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -563,7 +560,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_qdo_full;
     __shared__ uint64_t bar_k_full[RK], bar_k_empty[RK], bar_v_full[RV], bar_v_empty[RV];
-    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_dp_read, bar_ds_ready;
+    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready;
     __shared__ uint64_t bar_dq_done, bar_drain[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
@@ -602,7 +599,6 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ptx::mbar_init(&bar_s_full, 1);
         ptx::mbar_init(&bar_dp_full, 1);
         ptx::mbar_init(&bar_s_read, 8);
-        ptx::mbar_init(&bar_dp_read, 8);
         ptx::mbar_init(&bar_ds_ready, 8);
         ptx::mbar_init(&bar_dq_done, 1);
         ptx::mbar_init(&bar_drain[0], 1);
@@ -705,7 +701,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t ka = k_addr(j);
 #pragma unroll
                     for (int kk = 0; kk < G::kStepsRows; ++kk)
-                        ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * 8, desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                        ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
                     ptx::mma_commit(&bar_k_empty[j % RK]);
                     if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
                 }
@@ -770,9 +766,6 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0, *reinterpret_cast<uint32_t(*)[32]>(ud));
                 ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ud + 32));
                 ptx::tmem_wait_ld();
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bar_dp_read);
                 const float2 ndv = make_float2(-dr, -dr);
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
@@ -782,9 +775,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     dk[c >> 1] = G::pack2(ds.x, ds.y);
                 }
             }
-            if (!ptx::mbar_wait(&bar_dp_read, j & 1, &abort_flag, tmo)) { ok = false; break; }
-            ptx::tc_fence_after();
-            ptx::tmem_st32(lane_base + Cfg::kColDP + kc0 / 2, dk);
+            // dS -> this group's own dP columns [128 + 64g, ... + 32), already read.
+            ptx::tmem_st32(lane_base + Cfg::kColDP + kc0, dk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
