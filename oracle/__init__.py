@@ -56,6 +56,15 @@ def _bind(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_backward.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
                                     ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                     ctypes.c_long, ctypes.c_int, ctypes.c_double]
+    _up = ctypes.POINTER(ctypes.c_ubyte)
+    lib.oracle_forward_bs.restype = ctypes.c_int
+    lib.oracle_forward_bs.argtypes = [_dp, _dp, _dp, _dp, _dp, ctypes.c_long, ctypes.c_long,
+                                      ctypes.c_long, ctypes.c_long, ctypes.c_int, ctypes.c_double,
+                                      _up, ctypes.c_long, ctypes.c_long]
+    lib.oracle_backward_bs.restype = ctypes.c_int
+    lib.oracle_backward_bs.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_long,
+                                       ctypes.c_long, ctypes.c_long, ctypes.c_long, ctypes.c_int,
+                                       ctypes.c_double, _up, ctypes.c_long, ctypes.c_long]
     lib.oracle_head_sampled.restype = ctypes.c_int
     lib.oracle_head_sampled.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_long, ctypes.c_long,
                                         ctypes.c_long, ctypes.c_int, ctypes.c_double,
@@ -146,6 +155,64 @@ def backward(q, k, v, dout, causal: bool, scale: float, return_stats: bool = Fal
     if return_stats:
         return out + (stats.reshape(*lead, nq, 2),)
     return out
+
+
+def _mask_arg(block_mask, nq: int, nk: int, block_q: int, block_k: int):
+    m = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    want = ((nq + block_q - 1) // block_q, (nk + block_k - 1) // block_k)
+    if m.shape != want:
+        raise ValueError(f"block_mask must have shape {want}, got {m.shape}")
+    return m
+
+
+def forward_block_sparse(q, k, v, causal: bool, scale: float, block_mask,
+                         block_q: int = 128, block_k: int = 128):
+    """Block-sparse O and L: key j is visible to query i iff
+    block_mask[i // block_q, j // block_k] is set (and j <= i under causal).
+    Rows that see no key get O = 0 and L = -inf.  Shapes as in forward()."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    qh, lead = _heads_view(q)
+    kh, _ = _heads_view(k)
+    vh, _ = _heads_view(v)
+    heads, nq, d = qh.shape
+    nk = kh.shape[1]
+    if kh.shape != (heads, nk, d) or vh.shape != kh.shape:
+        raise ValueError("q, k, v shapes disagree")
+    m = _mask_arg(block_mask, nq, nk, block_q, block_k)
+    o = np.empty_like(qh)
+    lse = np.empty((heads, nq), dtype=np.float64)
+    rc = _load().oracle_forward_bs(_ptr(qh), _ptr(kh), _ptr(vh), _ptr(o), _ptr(lse), heads, nq, nk,
+                                   d, int(bool(causal)), float(scale),
+                                   m.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)),
+                                   block_q, block_k)
+    if rc != 0:
+        raise RuntimeError(f"oracle_forward_bs failed with code {rc}")
+    return o.reshape(*lead, nq, d), lse.reshape(*lead, nq)
+
+
+def backward_block_sparse(q, k, v, dout, causal: bool, scale: float, block_mask,
+                          block_q: int = 128, block_k: int = 128):
+    """dQ, dK, dV of the block-sparse attention (see forward_block_sparse)."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    qh, lead = _heads_view(q)
+    kh, _ = _heads_view(k)
+    vh, _ = _heads_view(v)
+    doh, _ = _heads_view(dout)
+    heads, nq, d = qh.shape
+    nk = kh.shape[1]
+    if kh.shape != (heads, nk, d) or vh.shape != kh.shape or doh.shape != qh.shape:
+        raise ValueError("q, k, v, dout shapes disagree")
+    m = _mask_arg(block_mask, nq, nk, block_q, block_k)
+    dq = np.empty_like(qh)
+    dk = np.empty_like(kh)
+    dv = np.empty_like(vh)
+    rc = _load().oracle_backward_bs(_ptr(qh), _ptr(kh), _ptr(vh), _ptr(doh), _ptr(dq), _ptr(dk),
+                                    _ptr(dv), heads, nq, nk, d, int(bool(causal)), float(scale),
+                                    m.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)),
+                                    block_q, block_k)
+    if rc != 0:
+        raise RuntimeError(f"oracle_backward_bs failed with code {rc}")
+    return dq.reshape(*lead, nq, d), dk.reshape(*lead, nk, d), dv.reshape(*lead, nk, d)
 
 
 def head_sampled(q, k, v, dout, causal: bool, scale: float, qrows, krows,

@@ -245,6 +245,180 @@ int oracle_backward(const double* q, const double* k, const double* v, const dou
 }
 
 /*
+ * Block-sparse attention ("Notes on flashattention" post, section
+ * "Block-sparse Flashattention", with its Proposition 4): a block mask M over
+ * (query block, key block) pairs of bq x bk rows; key j is visible to query i
+ * iff M[i / bq][j / bk] != 0 and, with causal, j <= i.  Masked scores take no
+ * part in the softmax: the page's algorithm skips the zero blocks entirely,
+ * which is what excluding them computes (the page's "(S o 1_M)_kl = 0 where
+ * M_kl = 0" is read as "excluded from the softmax", the only reading under
+ * which skipping those blocks gives the same P).  A query row that sees no key
+ * has O_i = 0 and L_i = -inf, dQ_i = 0, and adds nothing to dK or dV.
+ * mask is [ceil(nq / bq)][ceil(nk / bk)] bytes, row-major.
+ */
+static int visible_bs(long i, long j, int causal, const unsigned char* mask, long nbk,
+                      long bq, long bk) {
+    if (causal && j > i) return 0;
+    return mask[(i / bq) * nbk + (j / bk)] != 0;
+}
+
+static int check_mask(const unsigned char* mask, long bq, long bk) {
+    return mask != NULL && bq >= 1 && bk >= 1;
+}
+
+/* Scores of row i over its visible keys: idx[0..n) the key indices in
+ * increasing order, s[0..n) the scores; returns n. */
+static long row_scores_bs(const double* qi, const double* kh, long i, long nk, long d,
+                          int causal, double scale, const unsigned char* mask, long nbk,
+                          long bq, long bk, long* idx, double* s) {
+    long n = 0;
+    for (long j = 0; j < nk; ++j) {
+        if (!visible_bs(i, j, causal, mask, nbk, bq, bk)) continue;
+        idx[n] = j;
+        s[n] = scale * dot(qi, kh + j * d, d);
+        ++n;
+    }
+    return n;
+}
+
+int oracle_forward_bs(const double* q, const double* k, const double* v,
+                      double* o, double* lse,
+                      long heads, long nq, long nk, long d, int causal, double scale,
+                      const unsigned char* mask, long bq, long bk) {
+    if (!q || !k || !v || !o || !lse || !check_dims(heads, nq, nk, d) || !check_mask(mask, bq, bk))
+        return ORACLE_BAD_ARG;
+    const long nbk = (nk + bk - 1) / bk;
+    int err = ORACLE_OK;
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+        long* idx = (long*)malloc(sizeof(long) * (size_t)nk);
+        if (!s || !idx) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (long h = 0; h < heads; ++h) {
+            for (long i = 0; i < nq; ++i) {
+                if (!s || !idx) continue;
+                const double* vh = v + h * nk * d;
+                long n = row_scores_bs(q + (h * nq + i) * d, k + h * nk * d, i, nk, d, causal,
+                                       scale, mask, nbk, bq, bk, idx, s);
+                double* oi = o + (h * nq + i) * d;
+                for (long t = 0; t < d; ++t) oi[t] = 0.0;
+                if (n == 0) {
+                    lse[h * nq + i] = -INFINITY;
+                    continue;
+                }
+                double L = row_logsumexp(s, n);
+                for (long r = 0; r < n; ++r) {
+                    double p = exp(s[r] - L);
+                    const double* vj = vh + idx[r] * d;
+                    for (long t = 0; t < d; ++t) oi[t] += p * vj[t];
+                }
+                lse[h * nq + i] = L;
+            }
+        }
+        free(s);
+        free(idx);
+    }
+    return err;
+}
+
+int oracle_backward_bs(const double* q, const double* k, const double* v, const double* dout,
+                       double* dq, double* dk, double* dv,
+                       long heads, long nq, long nk, long d, int causal, double scale,
+                       const unsigned char* mask, long bq, long bk) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv || !check_dims(heads, nq, nk, d) ||
+        !check_mask(mask, bq, bk))
+        return ORACLE_BAD_ARG;
+    const long nbk = (nk + bk - 1) / bk;
+    double* L = (double*)malloc(sizeof(double) * (size_t)(heads * nq));
+    double* c = (double*)malloc(sizeof(double) * (size_t)(heads * nq));
+    if (!L || !c) { free(L); free(c); return ORACLE_NO_MEMORY; }
+    int err = ORACLE_OK;
+    /* Per row: L_i, c_i = sum_j P_ij dP_ij (Eq. 9's scalar) and dQ_i (Eq. 10). */
+#pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (size_t)nk);
+        double* dp = (double*)malloc(sizeof(double) * (size_t)nk);
+        long* idx = (long*)malloc(sizeof(long) * (size_t)nk);
+        if (!s || !dp || !idx) {
+#pragma omp atomic write
+            err = ORACLE_NO_MEMORY;
+        }
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (long h = 0; h < heads; ++h) {
+            for (long i = 0; i < nq; ++i) {
+                if (!s || !dp || !idx) continue;
+                const double* kh = k + h * nk * d;
+                const double* vh = v + h * nk * d;
+                const double* doi = dout + (h * nq + i) * d;
+                double* dqi = dq + (h * nq + i) * d;
+                for (long t = 0; t < d; ++t) dqi[t] = 0.0;
+                long n = row_scores_bs(q + (h * nq + i) * d, kh, i, nk, d, causal, scale,
+                                       mask, nbk, bq, bk, idx, s);
+                if (n == 0) {
+                    L[h * nq + i] = -INFINITY;
+                    c[h * nq + i] = 0.0;
+                    continue;
+                }
+                double Li = row_logsumexp(s, n);
+                double ci = 0.0;
+                for (long r = 0; r < n; ++r) {
+                    s[r] = exp(s[r] - Li);                       /* P_ij */
+                    dp[r] = dot(doi, vh + idx[r] * d, d);        /* dP_ij (Eq. 8) */
+                    ci += s[r] * dp[r];
+                }
+                for (long r = 0; r < n; ++r) {
+                    double ds = s[r] * dp[r] - s[r] * ci;
+                    const double* kj = kh + idx[r] * d;
+                    for (long t = 0; t < d; ++t) dqi[t] += ds * kj[t];
+                }
+                for (long t = 0; t < d; ++t) dqi[t] *= scale;
+                L[h * nq + i] = Li;
+                c[h * nq + i] = ci;
+            }
+        }
+        free(s);
+        free(dp);
+        free(idx);
+    }
+    /* Per key: dV_j = sum_i P_ij dO_i (Eq. 7), dK_j = scale sum_i dS_ij q_i (Eq. 11)
+     * over the query rows that see key j. */
+    if (err == ORACLE_OK) {
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+        for (long h = 0; h < heads; ++h) {
+            for (long j = 0; j < nk; ++j) {
+                const double* qh = q + h * nq * d;
+                const double* doh = dout + h * nq * d;
+                const double* kj = k + (h * nk + j) * d;
+                const double* vj = v + (h * nk + j) * d;
+                double* dkj = dk + (h * nk + j) * d;
+                double* dvj = dv + (h * nk + j) * d;
+                for (long t = 0; t < d; ++t) { dkj[t] = 0.0; dvj[t] = 0.0; }
+                for (long i = 0; i < nq; ++i) {
+                    if (!visible_bs(i, j, causal, mask, nbk, bq, bk)) continue;
+                    const double* qi = qh + i * d;
+                    const double* doi = doh + i * d;
+                    double p = exp(scale * dot(qi, kj, d) - L[h * nq + i]);
+                    double dpv = dot(doi, vj, d);
+                    double ds = p * dpv - p * c[h * nq + i];
+                    for (long t = 0; t < d; ++t) {
+                        dvj[t] += p * doi[t];
+                        dkj[t] += ds * qi[t];
+                    }
+                }
+                for (long t = 0; t < d; ++t) dkj[t] *= scale;
+            }
+        }
+    }
+    free(L);
+    free(c);
+    return err;
+}
+
+/*
  * Sampled outputs of ONE head (q, dout: [nq][d]; k, v: [nk][d]) for checking
  * sizes where the full outputs would take too long to compare:
  *   o_rows/lse_rows/dq_rows for the query rows listed in qrows,
