@@ -31,6 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import fa2_inputs  # noqa: E402
@@ -57,6 +58,19 @@ def causal_pairs(w) -> float:
 def flops(w):
     pc = causal_pairs(w)
     return 4.0 * w.d * pc, 10.0 * w.d * pc
+
+
+def block_sparse_pairs(mask, causal: bool, block: int = 128) -> int:
+    """(query, key) pairs one head computes under a block mask of full
+    block x block tiles: a full block off the diagonal, the lower triangle with
+    the diagonal on it under the causal rule."""
+    total = 0
+    for i in range(mask.shape[0]):
+        for j in range(mask.shape[1]):
+            if not mask[i, j] or (causal and j > i):
+                continue
+            total += block * (block + 1) // 2 if (causal and i == j) else block * block
+    return total
 
 
 def load_peaks():
@@ -240,6 +254,18 @@ def run_table(args):
     gqa = {"10b-b1h36-n4096-d128-gqa-kv4": 4, "10b-b1h36-n4096-d128-mqa": 1}
     for name in gqa:
         points.append(fa2_inputs.Workload(name, w10.B, w10.H, w10.N, w10.d, "bf16", w10.seed))
+    # Block-sparse points: block masks over the 32 x 32 tiles of 128 rows
+    # (a band of 4 tiles: each query tile sees itself and the 3 before it;
+    # and a seeded random mask of density 1/2 that keeps the diagonal).
+    nt = w10.N // 128
+    band = np.zeros((nt, nt), dtype=np.uint8)
+    for i in range(nt):
+        band[i, max(0, i - 3):i + 1] = 1
+    rnd = (np.random.default_rng(7).random((nt, nt)) < 0.5).astype(np.uint8)
+    np.fill_diagonal(rnd, 1)
+    sparse = {"10b-b1h36-n4096-d128-band4": band, "10b-b1h36-n4096-d128-bs50": rnd}
+    for name in sparse:
+        points.append(fa2_inputs.Workload(name, w10.B, w10.H, w10.N, w10.d, "bf16", w10.seed))
     points += [fa2_inputs.sweep_workload(N, d, dt) for dt in ("bf16", "fp32") for d in fa2_inputs.SWEEP_D
                for N in (128, 512, 1024, 4096, 8192, 16384, 32768)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -255,10 +281,16 @@ def run_table(args):
         h_kv = gqa.get(w.name, w.H)
         q, k, v, do = (torch.randn((w.B, h, w.N, w.d), generator=g).to(dt).to(dev)
                        for h in (w.H, h_kv, h_kv, w.H))
-        o, lse = fa2.forward(q, k, v, causal=w.causal, scale=w.scale)
+        o, lse = fa2.forward(q, k, v, causal=w.causal, scale=w.scale,
+                             block_mask=(torch.from_numpy(sparse[w.name]).to(dev) if w.name in sparse else None))
         ws = torch.empty(fa2.backward_workspace_bytes(w.B, w.H, w.N, w.d, q.dtype, h_kv), dtype=torch.uint8, device=dev)
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         f_fwd, f_bwd = flops(w)
+        bm = None
+        if w.name in sparse:
+            bm = torch.from_numpy(sparse[w.name]).to(dev)
+            pc = w.B * w.H * block_sparse_pairs(sparse[w.name], w.causal)
+            f_fwd, f_bwd = 4.0 * w.d * pc, 10.0 * w.d * pc
         b_fwd, b_bwd = alg_bytes(w)
         reps = max(3, min(args.steps, 20))
         tf, tb = [], []
@@ -266,13 +298,13 @@ def run_table(args):
             flush.zero_()
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             e[0].record()
-            fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+            fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, block_mask=bm)
             e[1].record()
             flush.zero_()
             e2 = torch.cuda.Event(enable_timing=True)
             e2.record()
             fa2.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws,
-                         dq=dq, dk=dk, dv=dv)
+                         dq=dq, dk=dk, dv=dv, block_mask=bm)
             e[2].record()
             torch.cuda.synchronize()
             if i >= 3:

@@ -68,15 +68,36 @@ def _stream_handle(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+BLOCK = 128  # rows per block of a block-sparse mask (the kernels' tile size)
+
+
+def _check_block_mask(block_mask: torch.Tensor, q: torch.Tensor, N: int, Nk: int) -> torch.Tensor:
+    """block_mask: CUDA bool / uint8 tensor [ceil(N / 128), ceil(Nk / 128)] on q's
+    device; returned as a contiguous uint8 tensor (nonzero = block computed)."""
+    want = ((N + BLOCK - 1) // BLOCK, (Nk + BLOCK - 1) // BLOCK)
+    if tuple(block_mask.shape) != want:
+        raise ValueError(f"block_mask must have shape {want} (blocks of {BLOCK} rows), got "
+                         f"{tuple(block_mask.shape)}")
+    if not block_mask.is_cuda or block_mask.device != q.device:
+        raise ValueError("block_mask must be a CUDA tensor on the device of q")
+    if block_mask.dtype not in (torch.bool, torch.uint8):
+        raise TypeError("block_mask must be torch.bool or torch.uint8")
+    return block_mask.to(torch.uint8).contiguous()
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
             scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
-            lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+            lse: Optional[torch.Tensor] = None,
+            block_mask: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """O = softmax(scale * Q K^T (+ causal mask)) V and L = logsumexp (fp32).
 
     q: contiguous CUDA tensor [B, H, N, d] (bf16, fp16 or fp32); k, v:
     [B, H_kv, Nk, d] with H a multiple of H_kv (grouped-query attention when
     H_kv < H: query head h uses key/value head h // (H // H_kv)); with
-    causal, key j is visible to query i iff j <= i.
+    causal, key j is visible to query i iff j <= i.  ``block_mask`` (optional,
+    16-bit inputs): block-sparse attention, a CUDA bool / uint8 tensor
+    [ceil(N / 128), ceil(Nk / 128)]; zero blocks of 128 x 128 rows are skipped,
+    rows that see no key get O = 0 and L = -inf.
     Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).
     """
     B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
@@ -86,6 +107,14 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if block_mask is not None:
+        bm = _check_block_mask(block_mask, q, N, Nk)
+        with torch.cuda.device(q.device):
+            _native.check(_native.lib().fa2_forward_block_sparse(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                B, H, H_kv, N, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
+                bm.data_ptr(), _stream_handle(q.device)))
+        return out, lse
     with torch.cuda.device(q.device):
         if H_kv == H and Nk == N:
             _native.check(_native.lib().fa2_forward(
@@ -112,7 +141,8 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              lse: torch.Tensor, do: torch.Tensor, causal: bool = True,
              scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
              dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
-             dv: Optional[torch.Tensor] = None, events=None):
+             dv: Optional[torch.Tensor] = None, events=None,
+             block_mask: Optional[torch.Tensor] = None):
     """dQ, dK, dV of sum(dO * O) via the recomputation backward.
 
     ``o`` and ``lse`` are the forward's outputs; ``workspace`` (optional) is a
@@ -120,6 +150,7 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     ``events`` (optional, for profiling): four recorded-once torch.cuda.Event
     objects the library records at its kernel boundaries (before the D/L
     pre-pass, after it, after the main pass, after the dQ finalisation).
+    ``block_mask``: the forward's block-sparse mask (see forward()).
     """
     B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
@@ -142,6 +173,17 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         if H_kv != H or Nk != N:
             raise ValueError("events are supported for H_kv == H and Nk == N only")
         ev_arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    if block_mask is not None:
+        if events is not None:
+            raise ValueError("events are not supported with a block mask")
+        bm = _check_block_mask(block_mask, q, N, Nk)
+        with torch.cuda.device(q.device):
+            _native.check(_native.lib().fa2_backward_block_sparse(
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, Nk, d,
+                int(bool(causal)), float(scale), _dtype_code(q), bm.data_ptr(), workspace.data_ptr(),
+                workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
+        return dq, dk, dv
     if H_kv != H or Nk != N:
         with torch.cuda.device(q.device):
             _native.check(_native.lib().fa2_backward_ex(

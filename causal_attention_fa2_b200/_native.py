@@ -33,6 +33,11 @@ SIGNATURES = {
     "fa2_backward_ex": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7
                         + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                            ctypes.c_void_p]),
+    "fa2_forward_block_sparse": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 7
+                                 + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
+    "fa2_backward_block_sparse": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7
+                                  + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_size_t, ctypes.c_void_p]),
     "fa2_backward": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                      + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                         ctypes.c_void_p]),

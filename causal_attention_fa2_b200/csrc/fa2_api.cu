@@ -141,7 +141,7 @@ constexpr bool use_two_tile_forward() {
 template <int ES, int D, bool F16 = false>
 fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                           int H, int H_kv, int N, int Nk, int causal, float scale, fa2_dtype dtype,
-                          cudaStream_t stream, uint32_t* status) {
+                          cudaStream_t stream, uint32_t* status, const uint8_t* block_mask = nullptr) {
     using Cfg = FwdCfg<ES, D>;
     const int BH = B * H;
     const int BH_kv = B * H_kv;
@@ -165,10 +165,11 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.causal = causal;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
+    p.block_mask = block_mask;
     if constexpr (use_two_tile_forward<ES, D>()) {
         // Two query tiles per CTA (softmax of one overlaps the MMAs of the other).
         using Cfg2 = Fwd2Cfg<ES, D, F16>;
-        auto kern = fa2_fwd2_kernel<ES, D, F16>;
+        auto kern = block_mask ? fa2_fwd2_kernel<ES, D, F16, true> : fa2_fwd2_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
         const unsigned pairs = static_cast<unsigned>((p.n_tiles + 1) / 2);
         kern<<<pairs * static_cast<unsigned>(BH), Cfg2::kThreads, Cfg2::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
@@ -184,13 +185,14 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
 template <int ES, bool F16 = false>
 fa2_status dispatch_forward(int d, const void* q, const void* k, const void* v, void* o,
                             float* lse, int B, int H, int H_kv, int N, int Nk, int causal, float scale,
-                            fa2_dtype dtype, cudaStream_t stream, uint32_t* status) {
+                            fa2_dtype dtype, cudaStream_t stream, uint32_t* status,
+                            const uint8_t* block_mask = nullptr) {
     switch (d) {
-        case 16: return launch_forward<ES, 16, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
-        case 32: return launch_forward<ES, 32, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
-        case 64: return launch_forward<ES, 64, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
-        case 80: return launch_forward<ES, 80, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
-        case 128: return launch_forward<ES, 128, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status);
+        case 16: return launch_forward<ES, 16, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status, block_mask);
+        case 32: return launch_forward<ES, 32, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status, block_mask);
+        case 64: return launch_forward<ES, 64, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status, block_mask);
+        case 80: return launch_forward<ES, 80, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status, block_mask);
+        case 128: return launch_forward<ES, 128, F16>(q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, stream, status, block_mask);
         default: return FA2_ERR_UNSUPPORTED_HEAD_DIM;
     }
 }
@@ -201,7 +203,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
                              int B, int H, int H_kv, int N, int Nk, int causal, float scale, fa2_dtype dtype,
                              uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                              uint32_t* status, unsigned long long timeout_ns,
-                             void* const* events) {
+                             void* const* events, const uint8_t* block_mask = nullptr) {
     using T = typename std::conditional<ES == 2, uint16_t, float>::type;
     using Cfg = BwdCfg<ES, D, F16>;
     auto mark = [&](int i) -> bool {
@@ -246,19 +248,20 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
+    p.block_mask = block_mask;
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
     // 2. dK, dV: key/value-tile-outer pass.
     {
-        auto kern = fa2_bwd_dkdv_kernel<ES, D, F16>;
+        auto kern = block_mask ? fa2_bwd_dkdv_kernel<ES, D, F16, true> : fa2_bwd_dkdv_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         kern<<<grid_kv, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     }
     // 3. dQ: query-tile-outer pass.
     {
-        auto kern = fa2_bwd_dq_kernel<ES, D, F16>;
+        auto kern = block_mask ? fa2_bwd_dq_kernel<ES, D, F16, true> : fa2_bwd_dq_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
         kern<<<grid, Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
@@ -331,6 +334,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
+    p.block_mask = nullptr;                              // block-sparse: 16-bit inputs only
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
@@ -366,7 +370,8 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
                            const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                            int H, int H_kv, int N, int Nk, int d, int causal, float scale, fa2_dtype dtype,
                            uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
-                           uint32_t* status, unsigned long long timeout_ns, void* const* events) {
+                           uint32_t* status, unsigned long long timeout_ns, void* const* events,
+                           const uint8_t* block_mask = nullptr) {
 #define FA2_BWD_CASE(DD)                                                                      \
     case DD:                                                                                  \
         if (dtype == FA2_FP32)                                                                \
@@ -375,9 +380,10 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
         if (dtype == FA2_FP16)                                                                \
             return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, \
                                                   causal, scale, dtype, ws_base, ws, stream,    \
-                                                  status, timeout_ns, events);                  \
+                                                  status, timeout_ns, events, block_mask);      \
         return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, causal, \
-                                        scale, dtype, ws_base, ws, stream, status, timeout_ns, events);
+                                        scale, dtype, ws_base, ws, stream, status, timeout_ns, events, \
+                                        block_mask);
     switch (d) {
         FA2_BWD_CASE(16)
         FA2_BWD_CASE(32)
@@ -409,13 +415,23 @@ fa2_status check_keys(int B, int H_kv, int Nk) {
     return FA2_OK;
 }
 
+// Block mask (optional): 16-bit inputs only, at most kMaxMaskTiles tiles per side.
+fa2_status check_block_mask(const uint8_t* block_mask, int N, int Nk, fa2_dtype dtype) {
+    if (!block_mask) return FA2_OK;
+    if (dtype == FA2_FP32) return FA2_ERR_UNSUPPORTED_DTYPE;
+    if ((N + kTileRows - 1) / kTileRows > kMaxMaskTiles || (Nk + kTileRows - 1) / kTileRows > kMaxMaskTiles)
+        return FA2_ERR_BAD_SHAPE;
+    return FA2_OK;
+}
+
 fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int H, int H_kv, int N, int Nk, int d, int causal, float scale,
-                        fa2_dtype dtype, fa2_stream_t stream) {
+                        fa2_dtype dtype, fa2_stream_t stream, const uint8_t* block_mask = nullptr) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
+    if ((st = check_block_mask(block_mask, N, Nk, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
@@ -425,9 +441,11 @@ fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, fl
     if ((st = init_device(&dev, &status)) != FA2_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == FA2_BF16)
-        return dispatch_forward<2>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
+        return dispatch_forward<2>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status,
+                                   block_mask);
     if (dtype == FA2_FP16)
-        return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
+        return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s,
+                                         status, block_mask);
     return dispatch_forward<4>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
 }
 
@@ -435,11 +453,12 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
                          const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                          int H, int H_kv, int N, int Nk, int d, int causal, float scale,
                          fa2_dtype dtype, void* workspace, size_t workspace_bytes,
-                         fa2_stream_t stream, void* const* events) {
+                         fa2_stream_t stream, void* const* events, const uint8_t* block_mask = nullptr) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
+    if ((st = check_block_mask(block_mask, N, Nk, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -454,7 +473,7 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                            dtype, static_cast<uint8_t*>(workspace), ws, s, status,
-                           kDefaultTimeoutNs, events);
+                           kDefaultTimeoutNs, events, block_mask);
 }
 
 }  // namespace
@@ -511,6 +530,25 @@ fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const vo
                            fa2_stream_t stream) {
     return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                          dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+fa2_status fa2_forward_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                    int B, int H, int H_kv, int N, int Nk, int d, int causal,
+                                    float scale, fa2_dtype dtype, const uint8_t* block_mask,
+                                    fa2_stream_t stream) {
+    if (!block_mask) return FA2_ERR_NULL_PTR;
+    return forward_impl(q, k, v, o, lse, B, H, H_kv, N, Nk, d, causal, scale, dtype, stream,
+                        block_mask);
+}
+
+fa2_status fa2_backward_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                                     int B, int H, int H_kv, int N, int Nk, int d, int causal,
+                                     float scale, fa2_dtype dtype, const uint8_t* block_mask,
+                                     void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+    if (!block_mask) return FA2_ERR_NULL_PTR;
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
+                         dtype, workspace, workspace_bytes, stream, nullptr, block_mask);
 }
 
 fa2_status fa2_last_device_status(void) {

@@ -138,6 +138,7 @@ struct BwdParams {
     float scale_log2;      // scale * log2(e)
     float scale;
     unsigned long long timeout_ns;
+    const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
 };
 
 template <int ES, int D, bool F16 = false>
@@ -150,16 +151,16 @@ struct BwdCfg {
     static constexpr int kThreadsDq = 352;
     static constexpr int kTile = G::kTileBytesK;
     // 227 KB minus the alignment pad and the static shared memory.
-    static constexpr int kBudget = 227 * 1024 - 1024 - 9 * 1024;
+    static constexpr int kBudget = 227 * 1024 - 1024 - 10 * 1024;
     // Two resident tiles (K,V or Q,dO) plus two rings of streamed tiles.
     static constexpr int kRing0 = (kBudget - 2 * kTile) / (2 * kTile);
     static constexpr int kRing = kRing0 > 3 ? 3 : kRing0;
     static_assert(kRing >= 2, "shared memory too small for the streaming rings");
     static constexpr int kSmemBytes = 1024 + 2 * kTile + 2 * kRing * kTile;
-    // dQ pass (static shared memory under 1 KB): Q, dO resident, K and V
+    // dQ pass (static shared memory under 2 KB): Q, dO resident, K and V
     // streamed.  K_j stays until dQ += dS K_j has read it, two MMA groups
     // after S(j), so K takes the deeper ring.
-    static constexpr int kDqStream = (227 * 1024 - 1024 - 1024) / kTile - 2;
+    static constexpr int kDqStream = (227 * 1024 - 1024 - 2048) / kTile - 2;
     static constexpr int kRingK = kDqStream - 2 > 3 ? 3 : kDqStream - 2;
     static constexpr int kRingV = kDqStream - kRingK > 3 ? 3 : kDqStream - kRingK;
     static_assert(kRingK >= 2 && kRingV >= 2, "shared memory too small for the dQ rings");
@@ -183,7 +184,7 @@ __host__ __device__ constexpr uint32_t a_col(int kk) {
 //   dV += P^T(i) dO(i)      (A = P^T from TMEM)     ; S^T(i+1) = K Q(i+1)^T
 //   dK += dS^T(i) Q(i)      (A = dS^T from TMEM)    ; dP^T(i+1) = V dO(i+1)^T
 // while the groups compute P^T(i+1) and dS^T(i+1).
-template <int ES, int D, bool F16 = false>
+template <int ES, int D, bool F16 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(320, 1)
 fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -205,6 +206,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // the warp's 64 query columns (double-buffered; each warp syncs itself).
     __shared__ __align__(16) float sL2[8][2][64];
     __shared__ __align__(16) float sDv[8][2][64];
+    // Block-sparse: the query tiles whose block with this key tile is set.
+    __shared__ uint16_t s_q[SPARSE ? kMaxMaskTiles : 1];
+    __shared__ int s_nq;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -224,14 +228,14 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int kv_tile = item / p.BH_kv;
     const int bh = item - kv_tile * p.BH_kv;            // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
-    // Query tiles per query head; none when no query reaches this key tile
-    // (causal, keys longer than queries): then dK = dV = 0 is written.
-    const int n_q = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;
-    const int n_it = n_q * p.group;                     // (query head, query tile) steps
     const int kv_row0 = kv_tile * kTileRows;
-    // Step it: query tile i_begin + it % n_q of the it / n_q-th query head of the group.
-    auto q_tile_of = [&](int it) { return i_begin + it % n_q; };
-    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
+    constexpr bool sparse = SPARSE;
+    if (sparse && warp == 0) {
+        const int n = warp_compact(s_q, p.n_tiles > i_begin ? p.n_tiles - i_begin : 0,
+            [&](int t) { return p.block_mask[static_cast<size_t>(i_begin + t) * p.n_tiles_k + kv_tile] != 0; },
+            [&](int t) { return i_begin + t; });
+        if (lane == 0) s_nq = n;
+    }
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -259,6 +263,14 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Query tiles per query head; none when no query reaches this key tile
+    // (causal with keys longer than queries, or an empty block column): then
+    // dK = dV = 0 is written.
+    const int n_q = sparse ? s_nq : (p.n_tiles > i_begin ? p.n_tiles - i_begin : 0);
+    const int n_it = n_q * p.group;                     // (query head, query tile) steps
+    // Step it: the (it % n_q)-th query tile of the it / n_q-th query head of the group.
+    auto q_tile_of = [&](int it) { return sparse ? static_cast<int>(s_q[it % n_q]) : i_begin + it % n_q; };
+    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -546,7 +558,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 // tensor core.  A thread that waits on an mbarrier after committing MMAs
 // stalls until those MMAs are done; with two issuers the other one's MMAs
 // keep the tensor core busy meanwhile.
-template <int ES, int D, bool F16 = false>
+template <int ES, int D, bool F16 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(352, 1)
 fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -564,6 +576,9 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __shared__ uint64_t bar_dq_done, bar_drain[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    // Block-sparse: the key tiles whose block with this query tile is set.
+    __shared__ uint16_t s_kv[SPARSE ? kMaxMaskTiles : 1];
+    __shared__ int s_nkv;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -581,7 +596,14 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int bh = item - rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
     // Key tiles this query tile sees (causal: key index <= query index).
-    const int n_kv = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
+    const int n_kv_lim = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
+    constexpr bool sparse = SPARSE;
+    if (sparse && warp == 0) {
+        const uint8_t* row = p.block_mask + static_cast<size_t>(q_tile) * p.n_tiles_k;
+        const int n = warp_compact(s_kv, n_kv_lim, [&](int j) { return row[j] != 0; },
+                                   [&](int j) { return j; });
+        if (lane == 0) s_nkv = n;
+    }
     const int q_row0 = q_tile * kTileRows;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
 
@@ -614,10 +636,14 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Key-tile steps; none for an empty block row, whose dQ is written as 0
+    // (nothing is loaded, so the Q slot can stage the zeros).
+    const int n_kv = sparse ? s_nkv : n_kv_lim;
+    auto kv_of = [&](int j) { return sparse ? static_cast<int>(s_kv[j]) : j; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && (!SPARSE || n_kv > 0)) {
             ptx::prefetch_tmap(&tm_k);
             ptx::prefetch_tmap(&tm_v);
             const uint64_t keep = ptx::policy_evict_last();
@@ -632,13 +658,13 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (j >= RK && !ptx::mbar_wait(&bar_k_empty[sk], ((j / RK) & 1) ^ 1, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_k_full[sk], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sKr + sk * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[sk], b * G::kBoxK, j * kTileRows, bh_kv, keep);
+                    ptx::tma_load_3d_hint(sKr + sk * TB + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[sk], b * G::kBoxK, kv_of(j) * kTileRows, bh_kv, keep);
                 k_issued = j + 1;
                 const int sv = j % RV;
                 if (j >= RV && !ptx::mbar_wait(&bar_v_empty[sv], ((j / RV) & 1) ^ 1, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[sv], TB);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d_hint(sVr + sv * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[sv], b * G::kBoxK, j * kTileRows, bh_kv, keep);
+                    ptx::tma_load_3d_hint(sVr + sv * TB + b * kTileRows * G::kRowBK, &tm_v, &bar_v_full[sv], b * G::kBoxK, kv_of(j) * kTileRows, bh_kv, keep);
                 v_issued = j + 1;
             }
             if (abort_flag) {
@@ -659,7 +685,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // tensor core busy while the other waits.  K_j's slot is released by
         // both S(j) and dQ(j); V_j's by dP(j).
         const int role = warp == 1 ? 0 : 1;
-        if (lane == 0) {
+        if (lane == 0 && (!SPARSE || n_kv > 0)) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_dq = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr = ptx::smem_addr(sQ);
@@ -725,8 +751,9 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const float dr = p.dvec[vrow];                   // D_i (0 past N)
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const bool diag = p.causal && (j == q_tile);
-            const int kv_valid = p.Nk - j * kTileRows - kc0;  // this group's key columns < Nk
+            const int kv = kv_of(j);
+            const bool diag = p.causal && (kv == q_tile);
+            const int kv_valid = p.Nk - kv * kTileRows - kc0;  // this group's key columns < Nk
             // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14)
             if (!ptx::mbar_wait(&bar_s_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -784,14 +811,19 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         // ---------------- epilogue (group 0): dQ * scale -> shared memory -> TMA store.
         if (g == 0) {
-            if (ok) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
+            if (ok && (!SPARSE || n_kv > 0)) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
             if (ok) {
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
                     uint32_t u[16];
-                    ptx::tmem_ld16(lane_base + Cfg::kColDQ + c0, u);
-                    ptx::tmem_wait_ld();
+                    if (SPARSE && n_kv == 0) {
+#pragma unroll
+                        for (int c = 0; c < 16; ++c) u[c] = 0u;
+                    } else {
+                        ptx::tmem_ld16(lane_base + Cfg::kColDQ + c0, u);
+                        ptx::tmem_wait_ld();
+                    }
 #pragma unroll
                     for (int h8 = 0; h8 < 2; ++h8) {
                         const int cc = c0 + 8 * h8;

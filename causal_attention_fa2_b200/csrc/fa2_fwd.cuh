@@ -59,6 +59,7 @@ struct FwdParams {
     int causal;
     float scale_log2;      // scale * log2(e)
     unsigned long long timeout_ns;
+    const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
 };
 
 template <int ES, int D>

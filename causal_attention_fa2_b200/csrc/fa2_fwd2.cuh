@@ -56,11 +56,11 @@ struct Fwd2Cfg {
 
 // One softmax warpgroup: processes query tile `t` (0 = A, 1 = B) for key
 // tiles 0 .. n_kv-1, then writes its O tile and L rows.
-template <int ES, int D, bool F16>
+template <int ES, int D, bool F16, bool SPARSE>
 __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_tile, int n_kv,
                                              int bh, uint32_t tmem, uint8_t* sQt,
                                              uint64_t* bar_s_full, uint64_t* bar_p_full,
-                                             uint64_t* bar_o_done,
+                                             uint64_t* bar_o_done, const uint16_t* kv_list,
                                              volatile uint32_t* abort_flag,
                                              const CUtensorMap* tm_o) {
     using Cfg = Fwd2Cfg<ES, D, F16>;
@@ -79,6 +79,10 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
+        // Key tile of step j, and (block-sparse) whether its block is set for this
+        // query tile: a step the other tile needs but this one does not is masked.
+        const int kv = SPARSE ? (kv_list[j] & 0x3FFF) : j;
+        const bool blk_on = !SPARSE || ((kv_list[j] >> (14 + t)) & 1);
         if (!ptx::mbar_wait(bar_s_full, j & 1, abort_flag, tmo)) { ok = false; break; }
         ptx::tc_fence_after();
         float s[128];
@@ -91,8 +95,12 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
 #pragma unroll
             for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(u[c]);
         }
-        const int kv_valid = p.Nk - j * kTileRows;
-        if (p.causal && j == q_tile) {
+        const int kv_valid = p.Nk - kv * kTileRows;
+        if (SPARSE && !blk_on) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = -INFINITY;
+        }
+        if (p.causal && kv == q_tile) {
 #pragma unroll
             for (int c = 0; c < 128; ++c)
                 if (c > r) s[c] = -INFINITY;
@@ -131,7 +139,9 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
             }
         }
         l *= alpha;
-        const float neg = -m_raw * sl2;
+        // Until the row has seen a key (block-sparse: leading masked steps) the
+        // reference max is -inf; exponentiate against 0 so masked scores give 0.
+        const float neg = (SPARSE && m_raw == -INFINITY) ? 0.f : -m_raw * sl2;
         const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg, neg);
         float2 rs = make_float2(0.f, 0.f);      // even / odd column sums
         // Exponentiate 32 columns at a time and store them as P right away.
@@ -163,15 +173,22 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
         if (lane == 0) ptx::mbar_arrive(bar_p_full);
     }
     // ---------------- epilogue: O / l -> shared memory (this tile's Q slot) -> TMA.
-    if (ok) ok = ptx::mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag, tmo);
+    // A row that saw no key (l = 0: an empty or fully masked block row) gets O = 0
+    // and L = -inf; a tile with no key step writes that without touching TMEM.
+    if (ok && (!SPARSE || n_kv > 0)) ok = ptx::mbar_wait(bar_o_done, (n_kv - 1) & 1, abort_flag, tmo);
     if (ok) {
         ptx::tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = (!SPARSE || l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
         for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
             uint32_t u[16];
-            ptx::tmem_ld16(o_tmem + c0, u);
-            ptx::tmem_wait_ld();
+            if (SPARSE && n_kv == 0) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) u[c] = 0u;
+            } else {
+                ptx::tmem_ld16(o_tmem + c0, u);
+                ptx::tmem_wait_ld();
+            }
             if constexpr (G::kF32) {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
@@ -219,7 +236,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
     }
 }
 
-template <int ES, int D, bool F16 = false>
+template <int ES, int D, bool F16 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(320, 1)
 fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -235,6 +252,10 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2], bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    // Block-sparse: the pair's key tiles, in order, with bit 14 / 15 set when
+    // the block of query tile A / B is set; s_cnt = steps of tile A, of the pair.
+    __shared__ uint16_t s_kv[SPARSE ? kMaxMaskTiles : 1];
+    __shared__ int s_cnt[2];
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -254,11 +275,29 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int pair = p.causal ? (n_pairs - 1 - rank) : rank;
     const int tile[2] = {2 * pair, 2 * pair + 1};
     const bool has_b = tile[1] < p.n_tiles;
-    // Key tiles each query tile sees (causal: key index <= query index).
-    const int n_kv_t[2] = {p.causal ? min(tile[0] + 1, p.n_tiles_k) : p.n_tiles_k,
-                           has_b ? (p.causal ? min(tile[1] + 1, p.n_tiles_k) : p.n_tiles_k) : 0};
-    const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
+    constexpr bool sparse = SPARSE;
+    if (sparse && warp == 0) {
+        // Key tiles of the pair: those whose block is set for tile A or tile B
+        // (and, causal, at or below that tile).  Tile A visits the prefix up to
+        // its own diagonal; steps whose block is set only for B are masked for A.
+        const uint8_t* row_a = p.block_mask + static_cast<size_t>(tile[0]) * p.n_tiles_k;
+        const uint8_t* row_b = p.block_mask + static_cast<size_t>(has_b ? tile[1] : tile[0]) * p.n_tiles_k;
+        auto on_a = [&](int j) { return (!p.causal || j <= tile[0]) && row_a[j] != 0; };
+        auto on_b = [&](int j) { return has_b && (!p.causal || j <= tile[1]) && row_b[j] != 0; };
+        auto any = [&](int j) { return on_a(j) || on_b(j); };
+        const int n_pair = warp_compact(s_kv, p.n_tiles_k, any,
+            [&](int j) { return j | (on_a(j) ? 0x4000 : 0) | (on_b(j) ? 0x8000 : 0); });
+        int n_a = n_pair;
+        if (p.causal) {
+            n_a = 0;
+            for (int base = 0; base <= tile[0] && base < p.n_tiles_k; base += 32) {
+                const int j = base + lane;
+                n_a += __popc(__ballot_sync(0xffffffffu, j <= tile[0] && j < p.n_tiles_k && any(j)));
+            }
+        }
+        if (lane == 0) { s_cnt[0] = n_a; s_cnt[1] = n_pair; }
+    }
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -286,19 +325,36 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Key-tile steps each query tile takes (causal: key index <= query index);
+    // tile A's steps are a prefix of tile B's.
+    int n_kv_t[2];
+    if (sparse) {
+        n_kv_t[0] = s_cnt[0];
+        n_kv_t[1] = has_b ? s_cnt[1] : 0;
+    } else {
+        n_kv_t[0] = p.causal ? min(tile[0] + 1, p.n_tiles_k) : p.n_tiles_k;
+        n_kv_t[1] = has_b ? (p.causal ? min(tile[1] + 1, p.n_tiles_k) : p.n_tiles_k) : 0;
+    }
+    const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
+    const bool load_q[2] = {n_kv_t[0] > 0, n_kv_t[1] > 0};
+    auto kv_of = [&](int j) { return sparse ? (s_kv[j] & 0x3FFF) : j; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // (no Q load for a query tile without key steps: its epilogue stages
+        // zeros in that Q slot)
+        if (lane == 0 && (!SPARSE || n_kv > 0)) {
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_k);
             ptx::prefetch_tmap(&tm_v);
             const uint64_t keep = ptx::policy_evict_last();
-            ptx::mbar_arrive_expect_tx(&bar_q_full, (has_b ? 2 : 1) * G::kTileBytesK);
-            for (int t = 0; t < (has_b ? 2 : 1); ++t)
+            ptx::mbar_arrive_expect_tx(&bar_q_full, ((load_q[0] ? 1 : 0) + (load_q[1] ? 1 : 0)) * G::kTileBytesK);
+            for (int t = 0; t < 2; ++t) {
+                if (!load_q[t]) continue;
                 for (int b = 0; b < G::kNBoxK; ++b)
                     ptx::tma_load_3d(sQ[t] + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full,
                                      b * G::kBoxK, tile[t] * kTileRows, bh);
+            }
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j % ST;
@@ -307,13 +363,13 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mbar_arrive_expect_tx(&bar_k_full[s], G::kTileBytesK);
                 for (int b = 0; b < G::kNBoxK; ++b)
                     ptx::tma_load_3d_hint(sK + s * G::kTileBytesK + b * kTileRows * G::kRowBK, &tm_k,
-                                          &bar_k_full[s], b * G::kBoxK, j * kTileRows, bh_kv, keep);
+                                          &bar_k_full[s], b * G::kBoxK, kv_of(j) * kTileRows, bh_kv, keep);
                 k_issued = j + 1;
                 if (j >= ST && !ptx::mbar_wait(&bar_v_empty[s], ph, &abort_flag, tmo)) break;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[s], G::kTileBytesMN);
                 for (int b = 0; b < G::kNBoxMN; ++b)
                     ptx::tma_load_3d_hint(sV + s * G::kTileBytesMN + b * kTileRows * G::kRowBMN, &tm_v,
-                                          &bar_v_full[s], b * G::kBoxMN, j * kTileRows, bh_kv, keep);
+                                          &bar_v_full[s], b * G::kBoxMN, kv_of(j) * kTileRows, bh_kv, keep);
                 v_issued = j + 1;
             }
             if (abort_flag) {
@@ -327,7 +383,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && (!SPARSE || n_kv > 0)) {
             constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr[2] = {ptx::smem_addr(sQ[0]), ptx::smem_addr(sQ[1])};
@@ -365,7 +421,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (ok) ok = ptx::mbar_wait(&bar_k_full[0], 0, &abort_flag, tmo);
             if (ok) {
                 ptx::tc_fence_after();
-                issue_s(0, 0);
+                if (!SPARSE || n_kv_t[0] > 0) issue_s(0, 0);
                 if (n_kv_t[1] > 0) issue_s(1, 0);
                 ptx::mma_commit(&bar_k_empty[0]);
             }
@@ -408,9 +464,11 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     } else {
         // ------------------------------------------------ softmax warpgroups
         const int t = (warp - 2) >> 2;       // 0: warps 2-5 (tile A), 1: warps 6-9 (tile B)
-        if (n_kv_t[t] > 0) {
-            fwd2_softmax<ES, D, F16>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
-                                &bar_p_full[t], &bar_o_done[t], &abort_flag, &tm_o);
+        // Every existing query tile writes O and L, also one without key steps.
+        if (SPARSE ? tile[t] < p.n_tiles : n_kv_t[t] > 0) {
+            fwd2_softmax<ES, D, F16, SPARSE>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
+                                &bar_p_full[t], &bar_o_done[t], s_kv,
+                                &abort_flag, &tm_o);
         }
     }
 

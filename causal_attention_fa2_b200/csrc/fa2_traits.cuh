@@ -35,6 +35,31 @@ __host__ __device__ inline int kv_head_of(int bh, int H, int H_kv, int group) {
     return (bh / H) * H_kv + (bh % H) / group;
 }
 
+// Block-sparse attention ("Notes on flashattention", section "Block-sparse
+// Flashattention"): a byte per (query tile, key tile) pair of kTileRows x
+// kTileRows blocks, row-major with one row per query tile; zero blocks are
+// skipped.  A CTA compacts the tiles it visits into a shared-memory list of at
+// most kMaxMaskTiles entries, so masks cover at most that many tiles per side.
+constexpr int kMaxMaskTiles = 512;
+
+// Warp-cooperative compaction (whole warp): writes, in increasing order, the
+// value val(t) of every t in [0, n) with keep(t) into list[], and returns the
+// count (the same in every lane).
+template <class Keep, class Val>
+__device__ __forceinline__ int warp_compact(uint16_t* list, int n, Keep keep, Val val) {
+    const int lane = threadIdx.x & 31;
+    int count = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int t = base + lane;
+        const bool k = t < n && keep(t);
+        const unsigned bal = __ballot_sync(0xffffffffu, k);
+        if (k && count + __popc(bal & ((1u << lane) - 1u)) < kMaxMaskTiles)
+            list[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(val(t));
+        count += __popc(bal);
+    }
+    return count < kMaxMaskTiles ? count : kMaxMaskTiles;
+}
+
 // Device status codes the kernels record (same values as fa2_status).
 constexpr uint32_t kDevStatusTimeout = 8;
 

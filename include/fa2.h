@@ -43,6 +43,7 @@
 #define FA2_H_
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -160,6 +161,37 @@ fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const vo
                            int B, int H, int H_kv, int N, int Nk, int d, int causal, float scale,
                            fa2_dtype dtype, void* workspace, size_t workspace_bytes,
                            fa2_stream_t stream);
+
+/*
+ * Block-sparse attention ("Notes on flashattention" post, section
+ * "Block-sparse Flashattention", Proposition 4): blocks of 128 query rows by
+ * 128 key rows whose mask byte is 0 are skipped; their scores take no part in
+ * the softmax.
+ *   block_mask  in : DEVICE pointer to ceil(N / 128) * ceil(Nk / 128) bytes,
+ *                    row-major (one row per 128-row query tile); entry (a, b)
+ *                    nonzero lets query rows [128a, 128a + 128) attend to key
+ *                    rows [128b, 128b + 128).  One mask for every batch and
+ *                    head; owned by the caller, read by the kernels only.
+ * With causal = 1 key j is visible to query i iff j <= i and its block is set.
+ * A query row that sees no key (its block row is empty) gets O = 0 and
+ * L = -inf; its dQ is 0 and it adds nothing to dK or dV.  Other arguments,
+ * results and the workspace are those of fa2_forward_ex / fa2_backward_ex.
+ * Errors: block_mask NULL -> FA2_ERR_NULL_PTR; FA2_FP32 inputs ->
+ * FA2_ERR_UNSUPPORTED_DTYPE (16-bit inputs only); more than 512 query or key
+ * tiles (N or Nk above 65536) -> FA2_ERR_BAD_SHAPE.  A mask of all ones gives
+ * the results of fa2_forward_ex / fa2_backward_ex.
+ */
+fa2_status fa2_forward_block_sparse(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int H, int H_kv, int N, int Nk, int d,
+                                    int causal, float scale, fa2_dtype dtype,
+                                    const uint8_t* block_mask, fa2_stream_t stream);
+
+fa2_status fa2_backward_block_sparse(const void* q, const void* k, const void* v, const void* o,
+                                     const float* lse, const void* dout, void* dq, void* dk,
+                                     void* dv, int B, int H, int H_kv, int N, int Nk, int d,
+                                     int causal, float scale, fa2_dtype dtype,
+                                     const uint8_t* block_mask, void* workspace,
+                                     size_t workspace_bytes, fa2_stream_t stream);
 
 /*
  * fa2_backward plus timing hooks, for profiling: identical arguments and

@@ -146,3 +146,32 @@ def test_ex_shape_validation(fa2lib):
     for Nk in (0, -5, (1 << 24) + 1):
         assert fwd_ex(4, 2, Nk) == 2, Nk
         assert bwd_ex(4, 2, Nk) == 2, Nk
+
+
+def test_block_sparse_validation(fa2lib):
+    """fa2_forward_block_sparse / fa2_backward_block_sparse: the mask pointer is
+    required, fp32 inputs are rejected, and at most 512 query / key tiles of 128
+    rows are accepted; all before touching the device."""
+    L = fa2lib
+
+    def fwd(mask, N=256, Nk=256, dtype=0):
+        return L.fa2_forward_block_sparse(P, P, P, P, P, 1, 4, 2, N, Nk, 64, 1, 0.125, dtype,
+                                          mask, None)
+
+    def bwd(mask, N=256, Nk=256, dtype=0):
+        return L.fa2_backward_block_sparse(P, P, P, P, P, P, P, P, P, 1, 4, 2, N, Nk, 64, 1, 0.125,
+                                           dtype, mask, P, 1 << 30, None)
+
+    assert fwd(None) == 1 and bwd(None) == 1                # FA2_ERR_NULL_PTR
+    assert fwd(P, dtype=1) == 4 and bwd(P, dtype=1) == 4    # fp32: FA2_ERR_UNSUPPORTED_DTYPE
+    for N, Nk in ((512 * 128 + 1, 256), (256, 512 * 128 + 1)):
+        assert fwd(P, N, Nk) == 2 and bwd(P, N, Nk) == 2    # > 512 tiles: FA2_ERR_BAD_SHAPE
+
+
+def test_binding_block_mask_checks():
+    import causal_attention_fa2_b200 as fa2
+    q = torch.zeros(1, 1, 300, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa2._check_block_mask(torch.ones(2, 3, dtype=torch.bool), q, 300, 300)   # wrong shape
+    with pytest.raises(ValueError):
+        fa2._check_block_mask(torch.ones(3, 3, dtype=torch.bool), q, 300, 300)   # not on CUDA

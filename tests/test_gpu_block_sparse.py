@@ -1,0 +1,146 @@
+"""Block-sparse attention (fa2_forward_block_sparse / fa2_backward_block_sparse):
+blocks of 128 query rows x 128 key rows whose mask byte is zero are skipped;
+with causal, key j is visible to query i iff j <= i and its block is set.  Rows
+that see no key: O = 0, L = -inf, dQ = 0, no contribution to dK, dV.
+
+Reference: the oracle's block-sparse functions run per query head with that
+head's key/value head; dK, dV of a key/value head sum over the query heads
+sharing it.  Masks are seeded inputs (random density 1/2 with some empty block
+rows, diagonal, band, a pattern where the two query tiles of one forward CTA
+differ, and the empty mask)."""
+import numpy as np
+import pytest
+import torch
+
+import fa2_inputs
+from parity_util import TOL, default_scale, to64
+
+pytestmark = pytest.mark.gpu
+
+BLOCK = 128
+
+
+def _mask(kind, nq_t, nk_t, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "random":
+        m = (rng.random((nq_t, nk_t)) < 0.5).astype(np.uint8)
+        m[rng.integers(0, nq_t)] = 0                       # one empty block row
+        return m
+    if kind == "diag":
+        return np.eye(nq_t, nk_t, dtype=np.uint8)
+    if kind == "band":                                     # each query tile sees itself and the tile before
+        return (np.eye(nq_t, nk_t, dtype=np.uint8) + np.eye(nq_t, nk_t, k=-1, dtype=np.uint8)).clip(0, 1)
+    if kind == "pair_split":                               # tiles 2t and 2t+1 differ
+        m = np.zeros((nq_t, nk_t), dtype=np.uint8)
+        for i in range(nq_t):
+            if i % 2 == 0:
+                m[i, 0] = 1
+            else:
+                m[i, min(i, nk_t - 1)] = 1
+                m[i, max(0, i - 2)] = 1
+        return m
+    if kind == "empty":
+        return np.zeros((nq_t, nk_t), dtype=np.uint8)
+    if kind == "ones":
+        return np.ones((nq_t, nk_t), dtype=np.uint8)
+    raise ValueError(kind)
+
+
+def _inputs(B, H, H_kv, N, Nk, d, dtype, seed):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    dt = fa2_inputs.DTYPES[dtype]
+    q = torch.randn((B, H, N, d), generator=g).to(dt)
+    k = torch.randn((B, H_kv, Nk, d), generator=g).to(dt)
+    v = torch.randn((B, H_kv, Nk, d), generator=g).to(dt)
+    do = torch.randn((B, H, N, d), generator=g).to(dt)
+    return q, k, v, do
+
+
+CASES = [
+    # (B, H, H_kv, N, Nk, d, dtype, causal, mask kind)
+    (1, 2, 2, 640, 640, 64, "bf16", True, "random"),
+    (1, 2, 2, 640, 640, 128, "bf16", False, "random"),
+    (1, 4, 2, 600, 700, 80, "fp16", True, "random"),
+    (1, 2, 2, 700, 450, 32, "bf16", False, "random"),
+    (2, 2, 1, 512, 512, 128, "bf16", True, "diag"),
+    (1, 2, 2, 1024, 1024, 128, "bf16", True, "band"),
+    (1, 2, 2, 768, 768, 64, "bf16", True, "pair_split"),
+    (1, 2, 2, 768, 640, 16, "fp16", False, "pair_split"),
+    (1, 2, 2, 384, 384, 32, "bf16", True, "empty"),
+]
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,Nk,d,dtype,causal,kind", CASES)
+def test_block_sparse_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal, kind):
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    nq_t, nk_t = -(-N // BLOCK), -(-Nk // BLOCK)
+    mask = _mask(kind, nq_t, nk_t, seed=N + Nk + d)
+    q, k, v, do = _inputs(B, H, H_kv, N, Nk, d, dtype, seed=500 + N + Nk + d)
+    scale = default_scale(d)
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    md = torch.from_numpy(mask).to(dev)
+    o, lse = fa2.forward(qd, kd, vd, causal=causal, scale=scale, block_mask=md)
+    dq, dk, dv = fa2.backward(qd, kd, vd, o, lse, dod, causal=causal, scale=scale, block_mask=md)
+    torch.cuda.synchronize()
+    assert fa2.last_device_status() == 0
+
+    grp = H // H_kv
+    ref = {"o": np.zeros((B, H, N, d)), "lse": np.zeros((B, H, N)), "dq": np.zeros((B, H, N, d)),
+           "dk": np.zeros((B, H_kv, Nk, d)), "dv": np.zeros((B, H_kv, Nk, d))}
+    for b in range(B):
+        for h in range(H):
+            hk = h // grp
+            qh, kh, vh, doh = (to64(t.float()) for t in (q[b, h], k[b, hk], v[b, hk], do[b, h]))
+            ro, rl = oracle_mod.forward_block_sparse(qh, kh, vh, causal, scale, mask, BLOCK, BLOCK)
+            rdq, rdk, rdv = oracle_mod.backward_block_sparse(qh, kh, vh, doh, causal, scale, mask,
+                                                             BLOCK, BLOCK)
+            ref["o"][b, h], ref["lse"][b, h], ref["dq"][b, h] = ro, rl, rdq
+            ref["dk"][b, hk] += rdk
+            ref["dv"][b, hk] += rdv
+
+    atol, rtol = TOL[dtype]
+    empty = np.isneginf(ref["lse"])                       # rows that see no key
+    got = {n: to64(t) for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    assert np.array_equal(np.isneginf(got["lse"]), empty), "rows with L = -inf differ"
+    assert np.all(got["o"][empty] == 0) and np.all(got["dq"][empty] == 0)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        g, r = got[name], ref[name]
+        if name in ("o", "lse", "dq"):
+            keep = ~empty
+            g, r = g[keep], r[keep]
+        assert np.isfinite(g).all(), f"{name}: non-finite values"
+        scale_t = grp if name in ("dk", "dv") else 1
+        err = np.abs(g - r)
+        bound = scale_t * atol + rtol * np.abs(r)
+        assert (err <= bound).all(), (name, float(err.max()), int((err > bound).sum()))
+
+
+def test_all_ones_mask_is_bitwise_dense():
+    """A mask of ones gives the bits of the dense entry points."""
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    B, H, N, d = 1, 4, 700, 64
+    q, k, v, do = (t.to(dev) for t in _inputs(B, H, H, N, N, d, "bf16", seed=9))
+    ones = torch.ones(-(-N // BLOCK), -(-N // BLOCK), dtype=torch.bool, device=dev)
+    for causal in (True, False):
+        o, lse = fa2.forward(q, k, v, causal=causal)
+        o2, lse2 = fa2.forward(q, k, v, causal=causal, block_mask=ones)
+        g = fa2.backward(q, k, v, o, lse, do, causal=causal)
+        g2 = fa2.backward(q, k, v, o, lse, do, causal=causal, block_mask=ones)
+        torch.cuda.synchronize()
+        assert torch.equal(o, o2) and torch.equal(lse, lse2)
+        assert all(torch.equal(a, b) for a, b in zip(g, g2))
+
+
+def test_block_sparse_deterministic():
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    q, k, v, do = (t.to(dev) for t in _inputs(1, 4, 2, 1024, 1024, 128, "bf16", seed=3))
+    m = torch.from_numpy(_mask("random", 8, 8, seed=4)).to(dev)
+    o, lse = fa2.forward(q, k, v, block_mask=m)
+    g1 = fa2.backward(q, k, v, o, lse, do, block_mask=m)
+    g2 = fa2.backward(q, k, v, o, lse, do, block_mask=m)
+    torch.cuda.synchronize()
+    assert all(torch.equal(a, b) for a, b in zip(g1, g2))
