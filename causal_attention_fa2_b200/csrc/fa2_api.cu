@@ -249,15 +249,27 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.scale = scale;
     p.timeout_ns = timeout_ns;
     p.block_mask = block_mask;
-    // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
-    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
+    p.kv_splits = ws.kv_splits;
+    p.part = ws.kv_splits > 1 ? reinterpret_cast<float*>(ws_base + ws.part_off) : nullptr;
+    // dK/dV pass: kv_splits CTAs per (key tile, key/value head); dQ pass: one per
+    // (query tile, query head).
+    const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv) *
+                             static_cast<unsigned>(p.kv_splits);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-    // 2. dK, dV: key/value-tile-outer pass.
+    // 2. dK, dV: key/value-tile-outer pass (+ the sum of a split group's partials).
     {
         auto kern = block_mask ? fa2_bwd_dkdv_kernel<ES, D, F16, true> : fa2_bwd_dkdv_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         kern<<<grid_kv, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
-        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
+        if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+        if (p.kv_splits > 1) {
+            const size_t groups4 = 2 * static_cast<size_t>(p.BH_kv) * Nk * D / 4;
+            fa2_bwd_kv_reduce_kernel<F16><<<static_cast<unsigned>((groups4 + 255) / 256), 256, 0, stream>>>(
+                p.part, static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), p.kv_splits, p.BH_kv, Nk,
+                p.n_tiles_k * kTileRows, D, scale);
+            if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+        }
+        if (!mark(2)) return FA2_ERR_CUDA;
     }
     // 3. dQ: query-tile-outer pass.
     {
@@ -335,6 +347,8 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     p.scale = scale;
     p.timeout_ns = timeout_ns;
     p.block_mask = nullptr;                              // block-sparse: 16-bit inputs only
+    p.kv_splits = 1;                                     // fp32: one CTA per group
+    p.part = nullptr;
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);

@@ -44,11 +44,28 @@ namespace fa2 {
 // dout ([BH][N][d]) and of k and v ([BH_kv][Nk][d]) rounded to TF32 (offsets 0
 // when absent).
 struct BwdWorkspace {
-    size_t l2_off, d_off, q_off, k_off, v_off, do_off, total;
+    size_t l2_off, d_off, q_off, k_off, v_off, do_off, part_off, total;
     int n_pad;
+    int kv_splits;   // dK/dV pass: CTAs per (key tile, key/value head)
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// With few key/value heads (grouped-query / multi-query attention) the dK/dV
+// pass has few CTAs: n_tiles_k * BH_kv of them, each looping over its whole
+// query-head group.  Below kSplitMinCtas CTAs the (query head, query tile)
+// steps of a group are split over up to `group` CTAs, each writing fp32 partial
+// dK, dV that a reduction pass sums in split order (so results stay
+// deterministic).  A function of the shapes only, so the workspace size does
+// not depend on the device.
+constexpr int kSplitMinCtas = 148;
+constexpr int kSplitTargetCtas = 296;
+__host__ __device__ inline int dkdv_splits(int n_tiles_k, int BH_kv, int group) {
+    const long long ctas = static_cast<long long>(n_tiles_k) * BH_kv;
+    if (group <= 1 || ctas >= kSplitMinCtas) return 1;
+    const long long want = (kSplitTargetCtas + ctas - 1) / ctas;
+    return static_cast<int>(want < group ? want : group);
+}
 
 inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d, int elem_bytes) {
     BwdWorkspace w;
@@ -57,7 +74,14 @@ inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d
     w.l2_off = 0;
     w.d_off = vec;
     w.total = 2 * vec;
-    w.q_off = w.k_off = w.v_off = w.do_off = 0;
+    w.q_off = w.k_off = w.v_off = w.do_off = w.part_off = 0;
+    const int n_tiles_k = (Nk + kTileRows - 1) / kTileRows;
+    w.kv_splits = elem_bytes == 2 ? dkdv_splits(n_tiles_k, BH_kv, BH / BH_kv) : 1;
+    if (w.kv_splits > 1) {
+        // fp32 partial dK and dV: [2][splits][BH_kv][n_tiles_k * 128][d]
+        w.part_off = w.total;
+        w.total += align256(2ull * w.kv_splits * BH_kv * n_tiles_k * kTileRows * d * sizeof(float));
+    }
     if (elem_bytes == 4) {
         const size_t tq = align256(static_cast<size_t>(BH) * N * d * sizeof(float));
         const size_t tk = align256(static_cast<size_t>(BH_kv) * Nk * d * sizeof(float));
@@ -139,6 +163,8 @@ struct BwdParams {
     float scale;
     unsigned long long timeout_ns;
     const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
+    int kv_splits;         // dK/dV pass CTAs per (key tile, key/value head)
+    float* part;           // fp32 partial dK, dV when kv_splits > 1
 };
 
 template <int ES, int D, bool F16 = false>
@@ -225,8 +251,10 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // key/value head, whose dK and dV sum over all of them; small j carries
     // the most work and is issued first.
     const int item = blockIdx.x;
-    const int kv_tile = item / p.BH_kv;
-    const int bh = item - kv_tile * p.BH_kv;            // key/value head
+    const int kv_tile = item / (p.BH_kv * p.kv_splits);
+    const int item_r = item - kv_tile * p.BH_kv * p.kv_splits;
+    const int split = item_r / p.BH_kv;                 // which share of the group's steps
+    const int bh = item_r - split * p.BH_kv;            // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
     const int kv_row0 = kv_tile * kTileRows;
     constexpr bool sparse = SPARSE;
@@ -267,10 +295,18 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // (causal with keys longer than queries, or an empty block column): then
     // dK = dV = 0 is written.
     const int n_q = sparse ? s_nq : (p.n_tiles > i_begin ? p.n_tiles - i_begin : 0);
-    const int n_it = n_q * p.group;                     // (query head, query tile) steps
-    // Step it: the (it % n_q)-th query tile of the it / n_q-th query head of the group.
-    auto q_tile_of = [&](int it) { return sparse ? static_cast<int>(s_q[it % n_q]) : i_begin + it % n_q; };
-    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
+    // (query head, query tile) steps of the group, this CTA taking the split-th
+    // of kv_splits consecutive shares.
+    const int n_all = n_q * p.group;
+    const int share = (n_all + p.kv_splits - 1) / p.kv_splits;
+    const int it0 = min(split * share, n_all);
+    const int n_it = min(n_all - it0, share);
+    // Step it: global step it0 + it = (query head) * n_q + (query tile index).
+    auto q_tile_of = [&](int it) {
+        const int g = (it0 + it) % n_q;
+        return sparse ? static_cast<int>(s_q[g]) : i_begin + g;
+    };
+    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + (it0 + it) / n_q; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -499,6 +535,33 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ---------------- epilogue: dV (group 0) / dK (group 1) -> shared memory -> TMA store
         // (zeros when no query reaches this key tile).
         if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
+        if (p.kv_splits > 1) {
+            // Split group: this CTA's fp32 partial sums, one key row per thread, to
+            // part[dK = 0 / dV = 1][split][head][row][d]; the reduction pass scales
+            // dK, sums the splits in order and rounds.
+            if (ok) {
+                ptx::tc_fence_after();
+                const uint32_t col = g == 0 ? Cfg::kColDV : Cfg::kColDK;
+                const size_t nk_pad = static_cast<size_t>(p.n_tiles_k) * kTileRows;
+                float* rowp = p.part + ((((g == 0 ? 1 : 0) * static_cast<size_t>(p.kv_splits) + split) *
+                                         p.BH_kv + bh) * nk_pad + kv_row0 + r) * D;
+#pragma unroll
+                for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
+                    uint32_t u[16] = {};
+                    if (n_it > 0) {
+                        ptx::tmem_ld16(lane_base + col + c0, u);
+                        ptx::tmem_wait_ld();
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        if (c0 + 4 * q4 < D)
+                            *reinterpret_cast<float4*>(rowp + c0 + 4 * q4) =
+                                make_float4(__uint_as_float(u[4 * q4]), __uint_as_float(u[4 * q4 + 1]),
+                                            __uint_as_float(u[4 * q4 + 2]), __uint_as_float(u[4 * q4 + 3]));
+                    }
+                }
+            }
+        } else {
         uint8_t* out_stage = g == 0 ? sV : sK;
         if (ok) {
             ptx::tc_fence_after();
@@ -538,6 +601,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
         }
+        }
     }
 
     ptx::tc_fence_before();
@@ -547,6 +611,41 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::tmem_dealloc(tmem, Cfg::kTmemCols);
     }
     if (threadIdx.x == 0 && abort_flag) atomicCAS(p.status, 0u, kDevStatusTimeout);
+}
+
+// dK, dV of a split group: element e of head hd, key row row (of Nk), column
+// col = sum over the kv_splits partials in split order; dK times scale; rounded
+// once to the 16-bit output type.  One thread per 4 consecutive columns.
+template <bool F16>
+__global__ void __launch_bounds__(256)
+fa2_bwd_kv_reduce_kernel(const float* __restrict__ part, uint16_t* __restrict__ dk,
+                         uint16_t* __restrict__ dv, int splits, int BH_kv, int Nk, int nk_pad, int d,
+                         float scale) {
+    const size_t per = static_cast<size_t>(BH_kv) * Nk * d / 4;   // 4-column groups per tensor
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= 2 * per) return;
+    const int which = i >= per ? 1 : 0;                              // 0: dK, 1: dV
+    const size_t e = (i - which * per) * 4;
+    const size_t hd = e / (static_cast<size_t>(Nk) * d);
+    const size_t rem = e - hd * Nk * d;
+    const size_t row = rem / d, col = rem - row * d;
+    const size_t stride = static_cast<size_t>(BH_kv) * nk_pad * d;  // one split's tensor
+    const float* src = part + (static_cast<size_t>(which) * splits * BH_kv + hd) * nk_pad * d + row * d + col;
+    float4 acc = *reinterpret_cast<const float4*>(src);
+    for (int s = 1; s < splits; ++s) {
+        const float4 x = *reinterpret_cast<const float4*>(src + s * stride);
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    const float m = which == 0 ? scale : 1.f;
+    uint2 w;
+    if constexpr (F16) {
+        w.x = ptx::pack_f16x2(acc.x * m, acc.y * m);
+        w.y = ptx::pack_f16x2(acc.z * m, acc.w * m);
+    } else {
+        w.x = ptx::pack_bf16x2(acc.x * m, acc.y * m);
+        w.y = ptx::pack_bf16x2(acc.z * m, acc.w * m);
+    }
+    *reinterpret_cast<uint2*>((which == 0 ? dk : dv) + e) = w;
 }
 
 // ------------------------------------------------------------------ dQ pass

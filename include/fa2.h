@@ -123,8 +123,13 @@ size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype)
 
 /*
  * Workspace of fa2_backward_ex: as fa2_backward_workspace_bytes, except that
- * the FA2_FP32 copies of k and v have B * H_kv * Nk * d elements.  Returns 0
- * for arguments fa2_backward_ex would reject.
+ * the FA2_FP32 copies of k and v have B * H_kv * Nk * d elements, and that for
+ * 16-bit inputs with few key/value tiles (ceil(Nk / 128) * B * H_kv < 148 and
+ * H_kv < H) the dK/dV pass splits each query-head group over S =
+ * min(H / H_kv, ceil(296 / (ceil(Nk / 128) * B * H_kv))) thread blocks whose
+ * fp32 partial dK and dV, 2 * S * B * H_kv * ceil(Nk / 128) * 128 * d * 4
+ * bytes, are summed in a fixed order afterwards.  Returns 0 for arguments
+ * fa2_backward_ex would reject.
  */
 size_t fa2_backward_workspace_bytes_ex(int B, int H, int H_kv, int N, int Nk, int d,
                                        fa2_dtype dtype);

@@ -175,3 +175,22 @@ def test_binding_block_mask_checks():
         fa2._check_block_mask(torch.ones(2, 3, dtype=torch.bool), q, 300, 300)   # wrong shape
     with pytest.raises(ValueError):
         fa2._check_block_mask(torch.ones(3, 3, dtype=torch.bool), q, 300, 300)   # not on CUDA
+
+
+def test_workspace_size_split_groups(fa2lib):
+    """16-bit grouped-query shapes with fewer than 148 (key tile, key/value
+    head) blocks: the workspace adds fp32 partial dK, dV for S splits."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    for B, H, hkv, N, nk, d in ((1, 8, 1, 512, 512, 64), (2, 36, 4, 4096, 4096, 128), (1, 4, 2, 300, 300, 80)):
+        n_pad = -(-N // 128) * 128
+        tk = -(-nk // 128)
+        base = 2 * up(B * H * n_pad * 4)
+        ctas = tk * B * hkv
+        S = 1 if ctas >= 148 else min(H // hkv, -(-296 // ctas))
+        part = up(2 * S * B * hkv * tk * 128 * d * 4) if S > 1 else 0
+        for dt in (0, 2):
+            assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, hkv, N, nk, d, dt) == base + part, (B, H, hkv, S)
+    # multi-head: never split
+    assert fa2lib.fa2_backward_workspace_bytes_ex(1, 4, 4, 256, 256, 64, 0) == \
+        fa2lib.fa2_backward_workspace_bytes(1, 4, 256, 64, 0)
