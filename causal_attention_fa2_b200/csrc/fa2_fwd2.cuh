@@ -39,7 +39,9 @@ namespace fa2 {
 template <int ES, int D, bool F16 = false>
 struct Fwd2Cfg {
     using G = TileGeom<ES, D, F16>;
-    static constexpr int kThreads = 320;
+    // Warp 0 TMA producer, 1 MMA issuer, 2-5 / 6-9 softmax of query tile A / B,
+    // 10 load watcher.
+    static constexpr int kThreads = 352;
     static constexpr int kBudget = 227 * 1024 - 2048;
     static constexpr int kQBytes = 2 * G::kTileBytesK;
     static constexpr int kFree = kBudget - kQBytes;
@@ -237,7 +239,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
 }
 
 template <int ES, int D, bool F16 = false, bool SPARSE = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
 fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const FwdParams p) {
@@ -310,7 +312,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(&bar_s_full[t], 1);
-            ptx::mbar_init(&bar_p_full[t], 4);
+            ptx::mbar_init(&bar_p_full[t], 5);   // 4 softmax warps + the load watcher
             ptx::mbar_init(&bar_o_done[t], 1);
         }
         ptx::mbar_init(&bar_drain, 1);
@@ -425,40 +427,46 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (n_kv_t[1] > 0) issue_s(1, 0);
                 ptx::mma_commit(&bar_k_empty[0]);
             }
+            // P_t(j) ready also means V_j and K_{j+1} have landed: the load watcher
+            // (warp 10) checks them before its arrival on that barrier, so this
+            // thread waits only on P (each wait here stalls it behind its own
+            // pending MMAs).  Every key tile j < n_kv is used by the query tile
+            // with the most steps, so both slots are released only after a
+            // checked load.
             for (int j = 0; ok && j < n_kv; ++j) {
-                const int s = j % ST;
-                const bool next_k = (j + 1) < n_kv;
-                if (!ptx::mbar_wait(&bar_v_full[s], (j / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                ptx::tc_fence_after();
-                bool k_waited = false;
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j < n_kv_t[t]) {
                         if (!issue_pv(t, j)) { ok = false; break; }
                     }
-                    if (j + 1 < n_kv_t[t]) {
-                        if (!k_waited) {
-                            const int s1 = (j + 1) % ST;
-                            if (!ptx::mbar_wait(&bar_k_full[s1], ((j + 1) / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                            ptx::tc_fence_after();
-                            k_waited = true;
-                        }
-                        issue_s(t, j + 1);
-                    }
+                    if (j + 1 < n_kv_t[t]) issue_s(t, j + 1);
                 }
                 if (!ok) break;
-                ptx::mma_commit(&bar_v_empty[s]);
-                if (next_k) {
-                    if (!k_waited) {
-                        // No tile uses K_{j+1}; keep the ring's bookkeeping.
-                        const int s1 = (j + 1) % ST;
-                        if (!ptx::mbar_wait(&bar_k_full[s1], ((j + 1) / ST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                    }
-                    ptx::mma_commit(&bar_k_empty[(j + 1) % ST]);
-                }
+                ptx::mma_commit(&bar_v_empty[j % ST]);
+                if (j + 1 < n_kv) ptx::mma_commit(&bar_k_empty[(j + 1) % ST]);
             }
             if (!ok) {
                 ptx::mma_commit(&bar_drain);
                 ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
+            }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------ load watcher
+        // For step j of query tile t: once V_j and (if tile t goes on) K_{j+1}
+        // have landed and the barrier's previous phase is complete, add the
+        // fifth arrival to P_t(j)'s barrier, so that the issuer's wait on P
+        // covers the loads too.  Off every critical path: it runs ahead of the
+        // softmax groups by up to one phase.
+        if (lane == 0 && (!SPARSE || n_kv > 0)) {
+            bool ok = true;
+            for (int j = 0; ok && j < n_kv; ++j) {
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (j >= n_kv_t[t]) continue;
+                    ok = ptx::mbar_wait(&bar_v_full[j % ST], (j / ST) & 1, &abort_flag, tmo);
+                    if (ok && j + 1 < n_kv_t[t])
+                        ok = ptx::mbar_wait(&bar_k_full[(j + 1) % ST], ((j + 1) / ST) & 1, &abort_flag, tmo);
+                    if (ok && j > 0) ok = ptx::mbar_wait(&bar_p_full[t], (j - 1) & 1, &abort_flag, tmo);
+                    if (ok) ptx::mbar_arrive(&bar_p_full[t]);
+                }
             }
         }
     } else {
