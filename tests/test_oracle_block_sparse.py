@@ -62,16 +62,18 @@ def test_block_diagonal_is_blockwise_dense(oracle_mod):
 
 
 @pytest.mark.parametrize("causal", [True, False])
-@pytest.mark.parametrize("seed", [0, 1, 2])
-def test_against_torch_sdpa_with_element_mask(oracle_mod, causal, seed):
+@pytest.mark.parametrize("seed,bq,bk", [(0, 8, 8), (1, 8, 8), (2, 8, 8), (3, 8, 4), (4, 4, 8)])
+def test_against_torch_sdpa_with_element_mask(oracle_mod, causal, seed, bq, bk):
     """Independent library routine: torch SDPA in float64 with autograd, the
-    boolean element mask expanded from the blocks.  Every query block keeps
-    its diagonal block so that every row sees at least one key (SDPA returns
-    NaN for rows with none)."""
-    nq, nk, d, bq, bk = 40, 40, 8, 8, 8
+    boolean element mask expanded from the blocks (also with different query
+    and key block sizes).  Every query block keeps a block on the diagonal
+    rows so that every row sees at least one key (SDPA returns NaN for rows
+    with none)."""
+    nq, nk, d = 40, 40, 8
     rng = np.random.default_rng(300 + seed)
     mask = (rng.random((nq // bq, nk // bk)) < 0.5).astype(np.uint8)
-    np.fill_diagonal(mask, 1)
+    for a in range(nq // bq):
+        mask[a, (a * bq) // bk] = 1              # the block holding key a*bq: row a*bq sees it
     g = torch.Generator().manual_seed(seed)
     q, k, v, do = (torch.randn(1, 1, 40, d, generator=g, dtype=torch.float64) for _ in range(4))
     allowed = torch.from_numpy(element_mask(mask, nq, nk, bq, bk, causal))

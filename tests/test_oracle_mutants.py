@@ -8,6 +8,7 @@ import subprocess
 
 import pytest
 
+import test_oracle_block_sparse as bsp
 import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
@@ -57,6 +58,51 @@ def test_pins_reject_planted_mistake(oracle_mod, tmp_path, name, old, new):
     oracle_mod._swap_library(str(so))
     try:
         for pin in _pin_suite(oracle_mod):
+            try:
+                pin()
+            except (AssertionError, RuntimeError, FloatingPointError):
+                caught.append(True)
+    finally:
+        oracle_mod._swap_library(None)
+    assert caught, f"no pin caught the planted mistake {name}"
+
+
+# Planted mistakes in the block-sparse functions, checked by the block-sparse pins.
+BS_MUTANTS = [
+    ("bs-causal-flip", "if (causal && j > i) return 0;", "if (causal && j >= i) return 0;"),
+    ("bs-block-sizes-swapped", "return mask[(i / bq) * nbk + (j / bk)] != 0;",
+     "return mask[(i / bk) * nbk + (j / bq)] != 0;"),
+    ("bs-empty-row-lse", "lse[h * nq + i] = -INFINITY;", "lse[h * nq + i] = 0.0;"),
+    ("bs-jacobian-dropped", "double ds = s[r] * dp[r] - s[r] * ci;", "double ds = s[r] * dp[r];"),
+    ("bs-key-visibility-dropped",
+     "if (!visible_bs(i, j, causal, mask, nbk, bq, bk)) continue;\n                    const double* qi",
+     "const double* qi"),
+    ("bs-dv-transposed-operand", "dvj[t] += p * doi[t];", "dvj[t] += p * qi[t];"),
+]
+
+
+def _bs_pin_suite(o):
+    yield lambda: bsp.test_all_ones_mask_is_dense(o, True)
+    yield lambda: bsp.test_block_diagonal_is_blockwise_dense(o)
+    yield lambda: bsp.test_against_torch_sdpa_with_element_mask(o, True, 3, 8, 4)
+    yield lambda: bsp.test_against_torch_sdpa_with_element_mask(o, False, 0, 8, 8)
+    yield lambda: bsp.test_rows_without_keys(o, True)
+    yield lambda: bsp.test_finite_differences(o, True)
+
+
+@pytest.mark.parametrize("name,old,new", BS_MUTANTS, ids=[m[0] for m in BS_MUTANTS])
+def test_block_sparse_pins_reject_planted_mistake(oracle_mod, tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found once"
+    cfile = tmp_path / "mutant.c"
+    cfile.write_text(src.replace(old, new, 1))
+    so = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(cfile),
+                    "-o", str(so), "-lm"], check=True)
+    caught = []
+    oracle_mod._swap_library(str(so))
+    try:
+        for pin in _bs_pin_suite(oracle_mod):
             try:
                 pin()
             except (AssertionError, RuntimeError, FloatingPointError):
