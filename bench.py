@@ -161,19 +161,23 @@ def oracle_step(w, sel):
     return dt, 14.0 * w.d * pairs
 
 
-def cpu_baseline(w, heads: int = 8):
-    """The oracle as it stands, timed on the host cores on `heads` full heads."""
+def cpu_baseline(w, budget_s: float = 20.0):
+    """The oracle as it stands, timed on the host cores over whole heads of the
+    workload, head after head, until every head is done or `budget_s` seconds
+    of oracle time have passed."""
     import oracle
     inp = fa2_inputs.workload_inputs(w)
-    t = 0.0
-    for hh in range(min(heads, w.heads)):
+    t, n = 0.0, 0
+    for hh in range(w.heads):
+        if t >= budget_s:
+            break
         b, h = divmod(hh, w.H)
-        sel = {n: inp[n][b, h].double().numpy() for n in ("q", "k", "v", "do")}
+        sel = {k: inp[k][b, h].double().numpy() for k in ("q", "k", "v", "do")}
         t0 = time.perf_counter()
         oracle.forward(sel["q"], sel["k"], sel["v"], w.causal, w.scale)
         oracle.backward(sel["q"], sel["k"], sel["v"], sel["do"], w.causal, w.scale)
         t += time.perf_counter() - t0
-    n = min(heads, w.heads)
+        n += 1
     f = 14.0 * w.d * (w.N * (w.N + 1) / 2 if w.causal else w.N * w.N) * n
     return {"value": f / t / 1e12, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
             "sample": f"{n} of {w.heads} heads at full N={w.N}, d={w.d}, fwd+bwd, fp64",
