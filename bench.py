@@ -327,6 +327,30 @@ def run_table(args):
     return 0
 
 
+# --------------------------------------------------------------------- ranks
+
+def rank_seed(w, rank: int) -> int:
+    """Seed of a rank's own batch: every rank draws a different batch of the
+    same shape (weak scaling; heads are independent, so ranks never exchange
+    data)."""
+    return w.seed + rank
+
+
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of `values` over all ranks, returned on every rank;
+    the values unchanged when there is one process (`dist` None)."""
+    if dist is None:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, ms: float) -> float:
+    """Work of all ranks over `steps` steps divided by the slowest rank's time."""
+    return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------------- GPU arm
 
 def main():
@@ -367,7 +391,7 @@ def main():
             dist.barrier()
 
     # Inputs: each rank its own seeded batch (weak scaling).
-    inp = fa2_inputs.make_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed + rank)
+    inp = fa2_inputs.make_inputs(w.B, w.H, w.N, w.d, w.dtype, rank_seed(w, rank))
     host = {n: t.pin_memory() for n, t in inp.items()}
     q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "do"))
     o = torch.empty_like(q)
@@ -413,10 +437,7 @@ def main():
     t_step = [a + b for a, b in zip(t_fwd, t_bwd)]
     total_ms = sum(t_step)
     fwd_ms, bwd_ms = sum(t_fwd), sum(t_bwd)
-    if dist is not None:
-        t = torch.tensor([total_ms, fwd_ms, bwd_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, fwd_ms, bwd_ms = t.tolist()
+    total_ms, fwd_ms, bwd_ms = max_over_ranks(dist, (total_ms, fwd_ms, bwd_ms), dev)
     status = fa2.last_device_status()
     if status != 0:
         raise SystemExit(f"device status after timing: {fa2.status_string(status)}")
@@ -448,17 +469,14 @@ def main():
     e_end.record()
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    (e2e_ms,) = max_over_ranks(dist, (e2e_ms,), dev)
     barrier()
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        value = world * (f_fwd + f_bwd) * K / (total_ms * 1e-3) / 1e12
-        fwd_tf = world * f_fwd * K / (fwd_ms * 1e-3) / 1e12
-        bwd_tf = world * f_bwd * K / (bwd_ms * 1e-3) / 1e12
+        value = whole_job_tflops(world, f_fwd + f_bwd, K, total_ms)
+        fwd_tf = whole_job_tflops(world, f_fwd, K, fwd_ms)
+        bwd_tf = whole_job_tflops(world, f_bwd, K, bwd_ms)
         avg_fwd = sum(t_fwd) / K
         avg_dkdv = sum(t_dkdv) / K
         avg_dq = sum(t_dq) / K
@@ -493,7 +511,7 @@ def main():
             "bwd_frac_of_measured_bf16": bwd_tf / world / peaks["bf16_tflops"],
             "ms": {"fwd": avg_fwd, "bwd_pre": sum(t_pre) / K, "bwd_dkdv": avg_dkdv,
                    "bwd_dq": avg_dq},
-            "e2e": {"value": world * (f_fwd + f_bwd) * K_e2e / (e2e_ms * 1e-3) / 1e12,
+            "e2e": {"value": whole_job_tflops(world, f_fwd + f_bwd, K_e2e, e2e_ms),
                     "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": K_e2e},
             "gpu_launches": 4 * K,
