@@ -50,3 +50,27 @@ def gpu_fwd_bwd(inp, causal: bool, scale: float, do_backward: bool = True):
 
 def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
+
+
+def grouped_reference(oracle_mod, q, k, v, do, causal: bool, scale: float):
+    """Oracle results for H query heads sharing H_kv key/value heads (query head
+    h reads key/value head h // (H // H_kv)) with query length N and key length
+    Nk: the oracle runs once per query head on that head's shared K and V, and
+    dK, dV of a key/value head are the sums of the per-query-head gradients over
+    the heads sharing it (the chain rule through the broadcast of K and V).
+    Tensors are [B, H, N, d] and [B, H_kv, Nk, d]; results are float64 numpy."""
+    B, H, N, d = q.shape
+    H_kv, Nk = k.shape[1], k.shape[2]
+    grp = H // H_kv
+    ref = {n: np.zeros(s) for n, s in (("o", (B, H, N, d)), ("lse", (B, H, N)), ("dq", (B, H, N, d)),
+                                         ("dk", (B, H_kv, Nk, d)), ("dv", (B, H_kv, Nk, d)))}
+    for b in range(B):
+        for h in range(H):
+            hk = h // grp
+            qh, kh, vh, doh = (to64(t) for t in (q[b, h], k[b, hk], v[b, hk], do[b, h]))
+            o, lse = oracle_mod.forward(qh, kh, vh, causal, scale)
+            dq, dk, dv = oracle_mod.backward(qh, kh, vh, doh, causal, scale)
+            ref["o"][b, h], ref["lse"][b, h], ref["dq"][b, h] = o, lse, dq
+            ref["dk"][b, hk] += dk
+            ref["dv"][b, hk] += dv
+    return ref

@@ -14,7 +14,7 @@ import pytest
 import torch
 
 import fa2_inputs
-from parity_util import assert_close, default_scale, to64
+from parity_util import assert_close, default_scale, grouped_reference, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -49,24 +49,6 @@ def _inputs(B, H, H_kv, N, Nk, d, dtype, seed):
     return q, k, v, do
 
 
-def _reference(oracle_mod, q, k, v, do, causal, scale):
-    B, H, N, d = q.shape
-    H_kv, Nk = k.shape[1], k.shape[2]
-    grp = H // H_kv
-    ref = {n: np.zeros(s) for n, s in (("o", (B, H, N, d)), ("lse", (B, H, N)), ("dq", (B, H, N, d)),
-                                         ("dk", (B, H_kv, Nk, d)), ("dv", (B, H_kv, Nk, d)))}
-    for b in range(B):
-        for h in range(H):
-            hk = h // grp
-            qh, kh, vh, doh = (to64(t.float()) for t in (q[b, h], k[b, hk], v[b, hk], do[b, h]))
-            o, lse = oracle_mod.forward(qh, kh, vh, causal, scale)
-            dq, dk, dv = oracle_mod.backward(qh, kh, vh, doh, causal, scale)
-            ref["o"][b, h], ref["lse"][b, h], ref["dq"][b, h] = o, lse, dq
-            ref["dk"][b, hk] += dk
-            ref["dv"][b, hk] += dv
-    return ref
-
-
 @pytest.mark.parametrize("B,H,H_kv,N,Nk,d,dtype,causal", CASES)
 def test_ex_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal):
     import causal_attention_fa2_b200 as fa2
@@ -82,7 +64,7 @@ def test_ex_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal):
     dq, dk, dv = fa2.backward(qd, kd, vd, o, lse, dod, causal=causal, scale=scale)
     torch.cuda.synchronize()
     assert dk.shape == k.shape and dv.shape == v.shape
-    ref = _reference(oracle_mod, q, k, v, do, causal, scale)
+    ref = grouped_reference(oracle_mod, q, k, v, do, causal, scale)
     if causal and Nk > N:
         # No query reaches keys N .. Nk-1: their gradients are exactly zero.
         assert not dk[:, :, N:].any() and not dv[:, :, N:].any()
