@@ -3,17 +3,22 @@ section "Block-sparse Flashattention": zero blocks of the block mask are
 skipped, i.e. their scores take no part in the softmax; combined with the
 causal rule key j is visible to query i iff j <= i and its block is set).
 
-Checked against facts that do not come from these functions: the dense oracle
+Checked against facts that do not come from these functions: a hand-derived
+worked example with every value in closed form (tests/golden/), the dense oracle
 (already pinned) for an all-ones mask and, block by block, for a block-diagonal
 mask; torch's float64 scaled_dot_product_attention with the element mask the
 blocks expand to; central finite differences; and the rule that a query row
 seeing no key has O = 0, L = -inf, dQ = 0 and no influence on dK, dV.
 """
+import json
 import math
+import os
 
 import numpy as np
 import pytest
 import torch
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
 def rand(shape, seed):
@@ -25,6 +30,19 @@ def element_mask(block_mask, nq, nk, bq, bk, causal):
     if causal:
         m &= np.tril(np.ones((nq, nk), dtype=bool))
     return m
+
+
+def test_worked_example_block_sparse_n4_d2(oracle_mod):
+    with open(os.path.join(GOLDEN, "worked_example_block_sparse_n4_d2.json")) as f:
+        g = json.load(f)
+    inp, exp = g["inputs"], g["expected"]
+    q, k, v, do = (np.array(inp[n])[None] for n in ("q", "k", "v", "do"))
+    args = (inp["causal"], inp["scale"], np.array(inp["block_mask"]), inp["block_q"], inp["block_k"])
+    o, lse = oracle_mod.forward_block_sparse(q, k, v, *args)
+    dq, dk, dv = oracle_mod.backward_block_sparse(q, k, v, do, *args)
+    tol = g["tolerance"]
+    for name, got in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        np.testing.assert_allclose(got[0], exp[name], atol=tol, rtol=0, err_msg=name)
 
 
 @pytest.mark.parametrize("causal", [True, False])

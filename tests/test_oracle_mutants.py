@@ -82,6 +82,7 @@ BS_MUTANTS = [
 
 
 def _bs_pin_suite(o):
+    yield lambda: bsp.test_worked_example_block_sparse_n4_d2(o)
     yield lambda: bsp.test_all_ones_mask_is_dense(o, True)
     yield lambda: bsp.test_block_diagonal_is_blockwise_dense(o)
     yield lambda: bsp.test_against_torch_sdpa_with_element_mask(o, True, 3, 8, 4)
