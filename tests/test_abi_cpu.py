@@ -194,3 +194,16 @@ def test_workspace_size_split_groups(fa2lib):
     # multi-head: never split
     assert fa2lib.fa2_backward_workspace_bytes_ex(1, 4, 4, 256, 256, 64, 0) == \
         fa2lib.fa2_backward_workspace_bytes(1, 4, 256, 64, 0)
+
+
+def test_plain_c_caller(fa2lib, tmp_path):
+    """include/fa2.h compiles as strict C11 and a C program linked against
+    libfa2.so gets the documented validation codes (tests/c_abi_check.c)."""
+    import subprocess
+    pkg = os.path.join(ROOT, "causal_attention_fa2_b200")
+    exe = tmp_path / "c_abi_check"
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_check.c"),
+                    "-L", pkg, "-lfa2", f"-Wl,-rpath,{pkg}", "-lm", "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
