@@ -39,9 +39,21 @@ namespace fa2 {
 template <int ES, int D, bool F16 = false>
 struct Fwd2Cfg {
     using G = TileGeom<ES, D, F16>;
-    // Warp 0 TMA producer, 1 MMA issuer, 2-5 / 6-9 softmax of query tile A / B,
-    // 10 load watcher.
-    static constexpr int kThreads = 352;
+    // Warpgroup 0: warp 0 TMA producer, 1 MMA issuer, 2 load watcher, 3 idle;
+    // warpgroups 1 / 2 (warps 4-7 / 8-11): softmax of query tile A / B.
+    static constexpr int kThreads = 384;
+    // Twelve warps put three on each SM sub-partition, so a thread starts with
+    // (16384 / 96) rounded down to a multiple of 8 = 168 registers.  Warpgroup
+    // 0 gives registers back (setmaxnreg.dec) and the softmax warpgroups, which
+    // hold a whole 128-column fp32 score row, take them (setmaxnreg.inc); the
+    // split must fit in what the block was launched with.
+    static constexpr int kLaunchRegs = 168;
+    static constexpr int kRegsLow = 72;
+    static constexpr int kRegsHigh = 216;
+    static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs,
+                  "register split exceeds the registers the block is launched with");
+    static_assert(kRegsLow % 8 == 0 && kRegsHigh % 8 == 0 && kRegsLow >= 24 && kRegsHigh <= 256,
+                  "setmaxnreg counts are multiples of 8 in [24, 256]");
     static constexpr int kBudget = 227 * 1024 - 2048;
     static constexpr int kQBytes = 2 * G::kTileBytesK;
     static constexpr int kFree = kBudget - kQBytes;
@@ -239,7 +251,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
 }
 
 template <int ES, int D, bool F16 = false, bool SPARSE = false>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(384, 1)
 fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const FwdParams p) {
@@ -341,6 +353,10 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const bool load_q[2] = {n_kv_t[0] > 0, n_kv_t[1] > 0};
     auto kv_of = [&](int j) { return sparse ? (s_kv[j] & 0x3FFF) : j; };
 
+    // Each warpgroup changes its register count inside its own branch, so the
+    // compiler allocates each role's code for the count that role runs with.
+    if (warp < 4) {
+    ptx::setmaxnreg_dec<Cfg::kRegsLow>();
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         // (no Q load for a query tile without key steps: its epilogue stages
@@ -428,7 +444,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mma_commit(&bar_k_empty[0]);
             }
             // P_t(j) ready also means V_j and K_{j+1} have landed: the load watcher
-            // (warp 10) checks them before its arrival on that barrier, so this
+            // (warp 2) checks them before its arrival on that barrier, so this
             // thread waits only on P (each wait here stalls it behind its own
             // pending MMAs).  Every key tile j < n_kv is used by the query tile
             // with the most steps, so both slots are released only after a
@@ -449,7 +465,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
             }
         }
-    } else if (warp == 10) {
+    } else if (warp == 2) {
         // ------------------------------------------------ load watcher
         // For step j of query tile t: once V_j and (if tile t goes on) K_{j+1}
         // have landed and the barrier's previous phase is complete, add the
@@ -469,9 +485,11 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
+    }
     } else {
+        ptx::setmaxnreg_inc<Cfg::kRegsHigh>();
         // ------------------------------------------------ softmax warpgroups
-        const int t = (warp - 2) >> 2;       // 0: warps 2-5 (tile A), 1: warps 6-9 (tile B)
+        const int t = (warp - 4) >> 2;       // 0: warps 4-7 (tile A), 1: warps 8-11 (tile B)
         // Every existing query tile writes O and L, also one without key steps.
         if (SPARSE ? tile[t] < p.n_tiles : n_kv_t[t] > 0) {
             fwd2_softmax<ES, D, F16, SPARSE>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],

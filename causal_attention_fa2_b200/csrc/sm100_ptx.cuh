@@ -14,6 +14,15 @@
 namespace fa2 {
 namespace ptx {
 
+// Per-warpgroup register reallocation (all four warps of an aligned
+// warpgroup execute the same instruction); N a multiple of 8 in [24, 256].
+template <int N> __device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(N));
+}
+template <int N> __device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(N));
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
