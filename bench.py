@@ -443,32 +443,67 @@ def main():
         raise SystemExit(f"device status after timing: {fa2.status_string(status)}")
 
     # ---------------- end to end through the public API with host buffers
+    # Every step copies its inputs from pinned host memory, runs forward and
+    # backward, and copies its results back.  Three streams and two device
+    # buffer sets let step i's input copies and step i-1's output copies run
+    # while step i-1's / step i's kernels do: a set's inputs are overwritten
+    # only after the kernels of the step two back have read them, and its
+    # outputs only after their copy to the host has finished.
+    out_names = ("o", "lse", "dq", "dk", "dv")
     out_host = {n: torch.empty_like(t if n != "lse" else lse, device="cpu").pin_memory()
                 for n, t in (("o", q), ("lse", lse), ("dq", q), ("dk", q), ("dv", q))}
     h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "do"))
     d2h = sum(t.numel() * t.element_size() for t in out_host.values())
     K_e2e = max(3, min(K, 50))
+    sets = [dict(q=q, k=k, v=v, do=do, o=o, lse=lse, dq=dq, dk=dk, dv=dv)]
+    sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
 
-    def e2e_step():
-        for n, dst in (("q", q), ("k", k), ("v", v), ("do", do)):
-            dst.copy_(host[n], non_blocking=True)
-        fa2.forward(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
-        fa2.backward(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws,
-                     dq=dq, dk=dk, dv=dv)
-        for n, src in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
-            out_host[n].copy_(src, non_blocking=True)
+    def e2e_run(n_steps, start=None, end=None):
+        ev_in = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_cmp = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_out = [torch.cuda.Event() for _ in range(n_steps)]
+        if start is not None:
+            start.record(s_in)
+        for i in range(n_steps):
+            b = sets[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[i - 2])
+                for n in ("q", "k", "v", "do"):
+                    b[n].copy_(host[n], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[i - 2])
+                fa2.forward(b["q"], b["k"], b["v"], causal=w.causal, scale=w.scale,
+                            out=b["o"], lse=b["lse"])
+                fa2.backward(b["q"], b["k"], b["v"], b["o"], b["lse"], b["do"], causal=w.causal,
+                             scale=w.scale, workspace=ws, dq=b["dq"], dk=b["dk"], dv=b["dv"])
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                for n in out_names:
+                    out_host[n].copy_(b[n], non_blocking=True)
+                ev_out[i].record(s_out)
+        if end is not None:
+            end.record(s_out)
 
-    for _ in range(2):
-        e2e_step()
+    torch.cuda.synchronize()
+    ref_host = {n: sets[0][n].cpu() for n in out_names}     # the device-timed loop's results
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier()
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record()
-    for _ in range(K_e2e):
-        e2e_step()
-    e_end.record()
+    e2e_run(K_e2e, e_start, e_end)
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end)
+    # The last step's results, read back on the host, must be the bits the
+    # device-timed loop produced from the same inputs.
+    for n in out_names:
+        if not torch.equal(out_host[n], ref_host[n]):
+            raise SystemExit(f"end-to-end leg: host copy of {n} differs from the device result")
     (e2e_ms,) = max_over_ranks(dist, (e2e_ms,), dev)
     barrier()
 
