@@ -27,7 +27,7 @@ from ._native import (FA2_BF16, FA2_FP16, FA2_FP32, FA2Error, clear_device_statu
 __all__ = [
     "forward", "backward", "backward_workspace_bytes", "flash_attention",
     "FlashAttention2Function", "last_device_status", "clear_device_status",
-    "status_string", "FA2Error", "library_path",
+    "status_string", "FA2Error", "library_path", "watchdog_selftest",
 ]
 
 SUPPORTED_HEAD_DIMS = (16, 32, 64, 80, 128)
@@ -68,6 +68,21 @@ def _stream_handle(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _check_buffer(name: str, t: torch.Tensor, shape, dtype: torch.dtype, device: torch.device) -> None:
+    """A caller-supplied output or scratch tensor must be exactly what the
+    library will write through its raw pointer."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)} on "
+                         f"{device}; got {t.dtype} {tuple(t.shape)} on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
+
+
+def _check_workspace(t: torch.Tensor, device: torch.device) -> None:
+    if t.dtype != torch.uint8 or t.dim() != 1 or t.device != device or not t.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous 1-D torch.uint8 tensor on {device}; got "
+                         f"{t.dtype} {tuple(t.shape)} on {t.device}")
+
+
 BLOCK = 128  # rows per block of a block-sparse mask (the kernels' tile size)
 
 
@@ -105,8 +120,12 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
         scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty_like(q)
+    else:
+        _check_buffer("out", out, q.shape, q.dtype, q.device)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    else:
+        _check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     if block_mask is not None:
         bm = _check_block_mask(block_mask, q, N, Nk)
         with torch.cuda.device(q.device):
@@ -154,15 +173,18 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     """
     B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
-        if t.shape != q.shape or t.dtype != q.dtype or not t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous CUDA tensor like q")
-    if lse.shape != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 tensor [B, H, N]")
+        _check_buffer(name, t, q.shape, q.dtype, q.device)
+    _check_buffer("lse", lse, (B, H, N), torch.float32, q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     need = backward_workspace_bytes(B, H, N, d, q.dtype, H_kv, Nk)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    else:
+        _check_workspace(workspace, q.device)
+    for name, t, like in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t is not None:
+            _check_buffer(name, t, like.shape, like.dtype, like.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
@@ -199,6 +221,16 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
             int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), _stream_handle(q.device), ev_arr))
     return dq, dk, dv
+
+
+def watchdog_selftest(limit_ns: int = 1_000_000, device: Optional[torch.device] = None) -> None:
+    """Enqueue the library's watchdog self-test on the current stream of
+    ``device`` (default: the current CUDA device): one wait that nothing
+    satisfies ends after ``limit_ns`` ns and records FA2_ERR_DEVICE_TIMEOUT in
+    the status word, which last_device_status() returns after a synchronize."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _native.check(_native.lib().fa2_watchdog_selftest(int(limit_ns), _stream_handle(dev)))
 
 
 class FlashAttention2Function(torch.autograd.Function):

@@ -49,6 +49,7 @@ SIGNATURES = {
     "fa2_last_device_status": (ctypes.c_int, []),
     "fa2_clear_device_status": (ctypes.c_int, []),
     "fa2_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fa2_watchdog_selftest": (ctypes.c_int, [ctypes.c_ulonglong, ctypes.c_void_p]),
 }
 
 

@@ -599,7 +599,7 @@ const char* fa2_status_string(fa2_status status) {
         case FA2_ERR_CUDA: return "FA2_ERR_CUDA: a CUDA call or kernel launch failed";
         case FA2_ERR_DEVICE_TIMEOUT: return "FA2_ERR_DEVICE_TIMEOUT: a kernel pipeline wait expired";
         case FA2_ERR_UNSUPPORTED_DEVICE: return "FA2_ERR_UNSUPPORTED_DEVICE: needs an sm_100 (B200) device";
-        case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1 and scale finite and > 0";
+        case FA2_ERR_BAD_ARGUMENT: return "FA2_ERR_BAD_ARGUMENT: causal must be 0/1, scale finite and > 0, a watchdog limit in [1e3, 1e10] ns";
         case FA2_ERR_SCRATCH_TOO_SMALL: return "FA2_ERR_SCRATCH_TOO_SMALL: the problem needs more than the 64 MiB built-in scratch of fa2_backward_noalloc; use fa2_backward with a workspace";
     }
     return "unknown fa2_status";
@@ -660,4 +660,47 @@ extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const v
     return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, N, d, causal, scale, dtype,
                            scratch, ws, reinterpret_cast<cudaStream_t>(stream), status,
                            kDefaultTimeoutNs, nullptr);
+}
+
+// ---------------------------------------------------------------------------
+// fa2_watchdog_selftest: proves on the running device that a pipeline wait
+// which is never satisfied ends after its limit and is reported through the
+// status word (see fa2.h), without faulting or hanging the GPU.
+
+namespace fa2 {
+
+constexpr unsigned long long kSelftestMinNs = 1000ull;            // 1 us
+constexpr unsigned long long kSelftestMaxNs = 10000000000ull;     // 10 s
+
+// One warp.  Thread 0 sets up an mbarrier that expects one arrival, which no
+// thread ever makes, and waits for its first phase with the same bounded wait
+// the attention kernels use; on expiry it records the timeout exactly as they
+// do.  Nothing else is touched.
+__global__ void __launch_bounds__(32, 1)
+fa2_watchdog_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ volatile uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0u;
+        ptx::mbar_init(&bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        const bool done = ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns);
+        if (!done && abort_flag) atomicCAS(status, 0u, kDevStatusTimeout);
+    }
+}
+
+}  // namespace fa2
+
+extern "C" fa2_status fa2_watchdog_selftest(unsigned long long limit_ns, fa2_stream_t stream) {
+    if (limit_ns < kSelftestMinNs || limit_ns > kSelftestMaxNs) return FA2_ERR_BAD_ARGUMENT;
+    int dev;
+    uint32_t* status;
+    fa2_status st = init_device(&dev, &status);
+    if (st != FA2_OK) return st;
+    fa2_watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status,
+                                                                                      limit_ns);
+    return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }

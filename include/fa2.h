@@ -70,7 +70,8 @@ typedef enum {
     FA2_ERR_CUDA = 7,                 /* a CUDA runtime/driver call or launch failed */
     FA2_ERR_DEVICE_TIMEOUT = 8,       /* a kernel's pipeline watchdog expired      */
     FA2_ERR_UNSUPPORTED_DEVICE = 9,   /* the current device is not sm_100          */
-    FA2_ERR_BAD_ARGUMENT = 10,        /* scale not finite and > 0, causal not 0/1  */
+    FA2_ERR_BAD_ARGUMENT = 10,        /* scale not finite and > 0, causal not 0/1,
+                                         watchdog self-test limit out of range     */
     FA2_ERR_SCRATCH_TOO_SMALL = 11    /* problem too big for fa2_backward_noalloc  */
 } fa2_status;
 
@@ -262,6 +263,24 @@ fa2_status fa2_clear_device_status(void);
 
 /* Static, human-readable name of a status code. */
 const char* fa2_status_string(fa2_status status);
+
+/*
+ * fa2_watchdog_selftest -- checks, on the current device, the pipeline
+ * watchdog every kernel wait relies on.  (Not part of the method; it tests
+ * this library's failure detection.)
+ *
+ * Enqueues on `stream` one warp whose first thread waits, with the kernels'
+ * bounded wait, on an mbarrier that no thread ever arrives on.  The wait ends
+ * after `limit_ns` nanoseconds (1e3 <= limit_ns <= 1e10, else
+ * FA2_ERR_BAD_ARGUMENT) and records FA2_ERR_DEVICE_TIMEOUT in the device's
+ * status word, exactly as an expired wait in an attention kernel does.  No
+ * memory is read or written besides the status word; the GPU context stays
+ * usable.  After synchronising `stream`, fa2_last_device_status() returns
+ * FA2_ERR_DEVICE_TIMEOUT (unless an earlier error is already recorded);
+ * fa2_clear_device_status() resets it.  Returns FA2_OK once enqueued, or a
+ * validation / launch error.
+ */
+fa2_status fa2_watchdog_selftest(unsigned long long limit_ns, fa2_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -67,6 +67,10 @@ int main(void) {
     CHECK(fa2_forward_block_sparse(P, P, P, P, (float*)P, 1, 2, 2, 128, 128, 64, 1, 0.125f,
                                    FA2_BF16, NULL, NULL) == FA2_ERR_NULL_PTR);
 
+    /* Watchdog self-test: the wait limit must lie in [1e3, 1e10] ns. */
+    CHECK(fa2_watchdog_selftest(0ull, NULL) == FA2_ERR_BAD_ARGUMENT);
+    CHECK(fa2_watchdog_selftest(20000000000ull, NULL) == FA2_ERR_BAD_ARGUMENT);
+
     if (failures) return 1;
     printf("ok\n");
     return 0;

@@ -118,6 +118,12 @@ def test_workspace_size(fa2lib, B, H, N, d):
 def test_valid_call_without_gpu_reports_cuda_error(fa2lib):
     assert fwd(fa2lib) in (7, 9)                   # FA2_ERR_CUDA / UNSUPPORTED_DEVICE
     assert fa2lib.fa2_last_device_status() in (7, 9)
+    assert fa2lib.fa2_watchdog_selftest(1_000_000, None) in (7, 9)
+
+
+def test_watchdog_selftest_limit_validation(fa2lib):
+    for bad in (0, 999, 10**10 + 1, 2**64 - 1):
+        assert fa2lib.fa2_watchdog_selftest(bad, None) == 10      # FA2_ERR_BAD_ARGUMENT
 
 
 def test_binding_rejects_cpu_tensors():
@@ -207,3 +213,27 @@ def test_plain_c_caller(fa2lib, tmp_path):
                     "-L", pkg, "-lfa2", f"-Wl,-rpath,{pkg}", "-lm", "-o", str(exe)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+def test_binding_buffer_checks():
+    """Caller-supplied outputs and workspace must match what the library writes
+    through their raw pointers (checked before any call; CPU tensors suffice)."""
+    from causal_attention_fa2_b200 import _check_buffer, _check_workspace
+    cpu = torch.device("cpu")
+    good = torch.empty(2, 3, 5, 8, dtype=torch.bfloat16)
+    _check_buffer("o", good, (2, 3, 5, 8), torch.bfloat16, cpu)
+    bad = [
+        torch.empty(2, 3, 5, 4, dtype=torch.bfloat16),                 # wrong shape
+        torch.empty(2, 3, 5, 8, dtype=torch.float16),                  # wrong dtype
+        torch.empty(2, 3, 8, 5, dtype=torch.bfloat16).transpose(2, 3),  # not contiguous
+    ]
+    for t in bad:
+        with pytest.raises(ValueError):
+            _check_buffer("o", t, (2, 3, 5, 8), torch.bfloat16, cpu)
+    with pytest.raises(ValueError):
+        _check_buffer("o", good, (2, 3, 5, 8), torch.bfloat16, torch.device("cuda", 0))
+    _check_workspace(torch.empty(1024, dtype=torch.uint8), cpu)
+    for t in (torch.empty(256, dtype=torch.float32), torch.empty(4, 256, dtype=torch.uint8),
+              torch.empty(2048, dtype=torch.uint8)[::2]):
+        with pytest.raises(ValueError):
+            _check_workspace(t, cpu)
