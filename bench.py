@@ -232,8 +232,8 @@ def config_of(w, n):
 
 def alg_bytes(w):
     """Algorithmic HBM bytes: forward reads Q, K, V and writes O and L; the
-    backward reads Q, K, V, O, dO, L and writes dQ, dK, dV (D and L*log2(e)
-    are workspace, counted as one write and one read each)."""
+    backward reads Q, K, V, O, dO and L and writes dQ, dK, dV, with its two
+    workspace vectors (D and L*log2(e)) counted once each."""
     es = 4 if w.dtype == "fp32" else 2
     t = w.B * w.H * w.N * w.d * es
     rows = w.B * w.H * w.N * 4
