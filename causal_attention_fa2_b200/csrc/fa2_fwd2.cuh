@@ -14,8 +14,13 @@
 //                  O_B += P_B(j) V_j ; S_B(j+1) = Q_B K_{j+1}^T
 //              so while softmax warpgroup A works on S_A(j+1) the tensor core
 //              runs PV_B(j) and S_B(j+1), and the other way round.
-//   warps 2-5  softmax warpgroup for tile A; warps 6-9 for tile B.  Thread t
+//   warp 2     load watcher: adds the arrival that tells the issuer V_j and
+//              K_{j+1} have landed to the P-ready barrier, so the issuer waits
+//              on that barrier alone.  Warp 3 idles.
+//   warps 4-7  softmax warpgroup for tile A; warps 8-11 for tile B.  Thread t
 //              owns query row t of its tile (tensor-memory lane t).
+//   Warpgroup 0 (warps 0-3) runs with fewer registers and the softmax
+//   warpgroups with more (setmaxnreg), so the score rows fit without spills.
 //
 // Tensor memory (512 columns): S_A | S_B | O_A | O_B, 128 columns each; P is
 // written over its S buffer (bf16 pairs, or fp32 for the TF32 path) and read
