@@ -17,13 +17,17 @@
 //   fa2_bwd_pre_kernel    per query row: D_i and L_i * log2(e), padded to
 //                         whole 128-row tiles with 0 / +inf so padded rows
 //                         drop out of P and dS.
-//   fa2_bwd_dkdv_kernel   one CTA per (key tile j, head), looping over the
-//                         query tiles i that see key tile j (i >= j causal).
+//   fa2_bwd_dkdv_kernel   one CTA per (key tile j, key/value head), looping over
+//                         the (query head, query tile i) steps that see key
+//                         tile j (i >= j causal); with grouped-query heads and
+//                         few key tiles the steps are split over several CTAs
+//                         whose fp32 partials fa2_bwd_kv_reduce_kernel sums.
 //   fa2_bwd_dq_kernel     one CTA per (query tile i, head), looping over the
 //                         key tiles j that query tile i sees (j <= i causal).
 //
-// Both main kernels use 10 warps: 0 TMA producer, 1 MMA issuer (one thread),
-// 2-5 and 6-9 two elementwise groups.  The thread holding TMEM lane t of either
+// Both main kernels use warp 0 as TMA producer, warp 1 as MMA issuer (one
+// thread) and warps 2-5 and 6-9 as two elementwise groups; the dQ pass adds
+// warp 10 as a second MMA issuer.  The thread holding TMEM lane t of either
 // group owns row t of the 128-row tile the CTA owns; group g handles columns
 // [64g, 64g+64) of the 128 x 128 score tile.  P and dS are written back into
 // tensor memory over the scores they came from (bf16 pairs) and read by the
