@@ -85,6 +85,10 @@ def _check_workspace(t: torch.Tensor, device: torch.device) -> None:
 
 BLOCK = 128  # rows per block of a block-sparse mask (the kernels' tile size)
 
+# backward(mode=...) -> flags of fa2_backward_opts
+_BWD_MODES = {"default": 0, "two-pass": _native.FA2_BWD_DETERMINISTIC,
+              "one-pass": _native.FA2_BWD_ONE_PASS}
+
 
 def _check_block_mask(block_mask: torch.Tensor, q: torch.Tensor, N: int, Nk: int) -> torch.Tensor:
     """block_mask: CUDA bool / uint8 tensor [ceil(N / 128), ceil(Nk / 128)] on q's
@@ -161,16 +165,24 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
              dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
              dv: Optional[torch.Tensor] = None, events=None,
-             block_mask: Optional[torch.Tensor] = None):
+             block_mask: Optional[torch.Tensor] = None, mode: str = "default"):
     """dQ, dK, dV of sum(dO * O) via the recomputation backward.
 
     ``o`` and ``lse`` are the forward's outputs; ``workspace`` (optional) is a
     uint8 CUDA tensor of at least backward_workspace_bytes(...) bytes.
     ``events`` (optional, for profiling): four recorded-once torch.cuda.Event
     objects the library records at its kernel boundaries (before the D/L
-    pre-pass, after it, after the main pass, after the dQ finalisation).
+    pre-pass, after it, after the query-tile pass, after the key-tile pass).
     ``block_mask``: the forward's block-sparse mask (see forward()).
+    ``mode``: "default" (the library's choice, flags = 0), "two-pass"
+    (FA2_BWD_DETERMINISTIC: every output bitwise reproducible) or "one-pass"
+    (FA2_BWD_ONE_PASS where it applies: one pass over key tiles with dQ summed
+    by fp32 reduce-add, so dQ bits can change from run to run; dK and dV are
+    bitwise reproducible either way).
     """
+    flags = _BWD_MODES.get(mode)
+    if flags is None:
+        raise ValueError(f"mode must be one of {sorted(_BWD_MODES)}, got {mode!r}")
     B, H, H_kv, N, Nk, d = _check_qkv(q, k, v)
     for name, t in (("o", o), ("do", do)):
         _check_buffer(name, t, q.shape, q.dtype, q.device)
@@ -195,25 +207,18 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         if H_kv != H or Nk != N:
             raise ValueError("events are supported for H_kv == H and Nk == N only")
         ev_arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
-    if block_mask is not None:
-        if events is not None:
-            raise ValueError("events are not supported with a block mask")
-        bm = _check_block_mask(block_mask, q, N, Nk)
+    if events is None:
+        bm = None if block_mask is None else _check_block_mask(block_mask, q, N, Nk)
         with torch.cuda.device(q.device):
-            _native.check(_native.lib().fa2_backward_block_sparse(
+            _native.check(_native.lib().fa2_backward_opts(
                 q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, Nk, d,
-                int(bool(causal)), float(scale), _dtype_code(q), bm.data_ptr(), workspace.data_ptr(),
+                int(bool(causal)), float(scale), _dtype_code(q),
+                None if bm is None else bm.data_ptr(), flags, workspace.data_ptr(),
                 workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
         return dq, dk, dv
-    if H_kv != H or Nk != N:
-        with torch.cuda.device(q.device):
-            _native.check(_native.lib().fa2_backward_ex(
-                q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, H_kv, N, Nk, d,
-                int(bool(causal)), float(scale), _dtype_code(q), workspace.data_ptr(),
-                workspace.numel() * workspace.element_size(), _stream_handle(q.device)))
-        return dq, dk, dv
+    if block_mask is not None or flags:
+        raise ValueError("events are supported for the default mode without a block mask only")
     with torch.cuda.device(q.device):
         _native.check(_native.lib().fa2_backward_timed(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),

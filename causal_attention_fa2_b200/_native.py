@@ -17,6 +17,9 @@ FA2_FP16 = 2
 FA2_OK = 0
 FA2_ERR_DEVICE_TIMEOUT = 8
 
+FA2_BWD_DETERMINISTIC = 1
+FA2_BWD_ONE_PASS = 2
+
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libfa2.so")
 _lib: Optional[ctypes.CDLL] = None
@@ -44,6 +47,9 @@ SIGNATURES = {
     "fa2_backward_timed": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                            + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
                               ctypes.c_void_p, ctypes.c_void_p]),
+    "fa2_backward_opts": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 7
+                          + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p, ctypes.c_uint,
+                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fa2_backward_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 5
                              + [ctypes.c_float, ctypes.c_int, ctypes.c_void_p]),
     "fa2_last_device_status": (ctypes.c_int, []),

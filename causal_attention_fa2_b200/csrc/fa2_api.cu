@@ -14,6 +14,7 @@
 
 #include "../../include/fa2.h"
 #include "fa2_bwd.cuh"
+#include "fa2_bwd_fused.cuh"
 #include "fa2_bwd32.cuh"
 #include "fa2_fwd.cuh"
 #include "fa2_fwd2.cuh"
@@ -25,6 +26,9 @@ namespace {
 __device__ uint32_t g_device_status;
 
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
+// Whether flags = 0 selects the one-pass backward where it applies (else only
+// FA2_BWD_ONE_PASS does).
+constexpr bool kOnePassDefault = false;
 constexpr int kMaxDevices = 64;
 constexpr int kMaxN = 1 << 24;
 
@@ -105,6 +109,22 @@ fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int
                           : dtype == FA2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                               : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                           3, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+}
+
+// [BH][n_pad][d] fp32 accumulator, reduce-added in boxes of box_cols columns x
+// 128 rows x 1 head whose rows use the swizzle of their width (128 or 64 bytes).
+fa2_status make_map_f32_reduce(CUtensorMap* m, void* ptr, int d, int n_pad, int BH, int box_cols) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n_pad),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                             static_cast<cuuint64_t>(d) * 4 * static_cast<cuuint64_t>(n_pad)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kTileRows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = box_cols * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
@@ -203,9 +223,15 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
                              int B, int H, int H_kv, int N, int Nk, int causal, float scale, fa2_dtype dtype,
                              uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                              uint32_t* status, unsigned long long timeout_ns,
-                             void* const* events, const uint8_t* block_mask = nullptr) {
+                             void* const* events, const uint8_t* block_mask, unsigned flags) {
     using T = typename std::conditional<ES == 2, uint16_t, float>::type;
     using Cfg = BwdCfg<ES, D, F16>;
+    // One pass (key tiles outer, dQ by fp32 reduce-add) where it applies and the
+    // caller did not ask for the bitwise-reproducible two-pass form.
+    const bool want_one = (flags & FA2_BWD_ONE_PASS) || (kOnePassDefault && !(flags & FA2_BWD_DETERMINISTIC));
+    const bool one_pass = want_one && ws.dqacc_off != 0 &&
+                          one_pass_applies((Nk + kTileRows - 1) / kTileRows, ES, ws.kv_splits, block_mask != nullptr);
+    float* dq_acc = one_pass ? reinterpret_cast<float*>(ws_base + ws.dqacc_off) : nullptr;
     auto mark = [&](int i) -> bool {
         if (!events || !events[i]) return true;
         return cudaEventRecord(static_cast<cudaEvent_t>(events[i]), stream) == cudaSuccess;
@@ -219,7 +245,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     if (!mark(0)) return FA2_ERR_CUDA;
     constexpr int kPreRows = BwdPreCfg<D>::kRowsPerBlock;
     fa2_bwd_pre_kernel<D, F16><<<static_cast<unsigned>((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
-        static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows);
+        static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows, dq_acc);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
@@ -251,12 +277,50 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.block_mask = block_mask;
     p.kv_splits = ws.kv_splits;
     p.part = ws.kv_splits > 1 ? reinterpret_cast<float*>(ws_base + ws.part_off) : nullptr;
+    p.item0 = 0;
+    if (one_pass) {
+        // 2. dQ and D of the query tiles whose rows see a single key tile (causal:
+        // query tile 0 of every head, the pass's last BH work items).
+        if (causal) {
+            auto kern = fa2_bwd_dq_kernel<ES, D, F16, false>;
+            if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
+            p.item0 = (p.n_tiles - 1) * BH;
+            kern<<<static_cast<unsigned>(BH), Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+            p.item0 = 0;
+            if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+        }
+        if (!mark(2)) return FA2_ERR_CUDA;
+        // 3. dK, dV and the other query tiles' dQ in one key-tile-outer pass, then
+        // dQ = scale * dQ_acc rounded once.
+        using FC = BwdFusedCfg<ES, D, F16>;
+        CUtensorMap macc;
+        if ((st = make_map_f32_reduce(&macc, dq_acc, D, ws.n_pad, BH, FC::kCW)) != FA2_OK) return st;
+        auto kern = fa2_bwd_fused_kernel<ES, D, F16>;
+        if ((st = set_smem(kern, FC::kSmemBytes)) != FA2_OK) return st;
+        const unsigned grid_f = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
+        kern<<<grid_f, FC::kThreads, FC::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, macc, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
+        const long long groups8 = static_cast<long long>(BH) * N * D / 8;
+        fa2_bwd_dq_finalize_kernel<F16><<<static_cast<unsigned>((groups8 + 255) / 256), 256, 0, stream>>>(
+            dq_acc, static_cast<uint16_t*>(dq), N, ws.n_pad, D, groups8, causal ? kTileRows : 0, scale);
+        if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
+        return FA2_OK;
+    }
     // dK/dV pass: kv_splits CTAs per (key tile, key/value head); dQ pass: one per
     // (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv) *
                              static_cast<unsigned>(p.kv_splits);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-    // 2. dK, dV: key/value-tile-outer pass (+ the sum of a split group's partials).
+    // 2. dQ: query-tile-outer pass.  It runs first because a query tile that sees
+    // a single key tile rewrites its rows' D (formed there from P and dP), which
+    // the dK/dV pass then reads.
+    {
+        auto kern = block_mask ? fa2_bwd_dq_kernel<ES, D, F16, true> : fa2_bwd_dq_kernel<ES, D, F16, false>;
+        if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
+    }
+    // 3. dK, dV: key/value-tile-outer pass (+ the sum of a split group's partials).
     {
         auto kern = block_mask ? fa2_bwd_dkdv_kernel<ES, D, F16, true> : fa2_bwd_dkdv_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
@@ -269,14 +333,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
                 p.n_tiles_k * kTileRows, D, scale);
             if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
         }
-        if (!mark(2)) return FA2_ERR_CUDA;
-    }
-    // 3. dQ: query-tile-outer pass.
-    {
-        auto kern = block_mask ? fa2_bwd_dq_kernel<ES, D, F16, true> : fa2_bwd_dq_kernel<ES, D, F16, false>;
-        if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
-        kern<<<grid, Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
-        if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
+        if (!mark(3)) return FA2_ERR_CUDA;
     }
     return FA2_OK;
 }
@@ -352,6 +409,19 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
+    // dQ pass first, then dK/dV (the order of the 16-bit path).
+    {
+        constexpr int W = Cfg::kWq;
+        CUtensorMap mq, mdo, mkk, mkmn, mvk, mdq;
+        if ((st = kmap(&mq, q, kTileRows, BH, N)) != FA2_OK || (st = kmap(&mdo, dout, kTileRows, BH, N)) != FA2_OK ||
+            (st = kmap(&mkk, k, W, BH_kv, Nk)) != FA2_OK || (st = mnmap(&mkmn, k, W, BH_kv, Nk)) != FA2_OK ||
+            (st = kmap(&mvk, v, W, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows, BH, N)) != FA2_OK)
+            return st;
+        auto kern = fa2_bwd32_dq_kernel<D>;
+        if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
+        kern<<<grid, Cfg::kThreads, Cfg::kSmemQ, stream>>>(mq, mdo, mkk, mkmn, mvk, mdq, p);
+        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
+    }
     {
         constexpr int W = Cfg::kWkv;
         CUtensorMap mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv;
@@ -363,18 +433,6 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
         auto kern = fa2_bwd32_dkdv_kernel<D>;
         if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
         kern<<<grid_kv, Cfg::kThreads, Cfg::kSmemKV, stream>>>(mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
-        if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
-    }
-    {
-        constexpr int W = Cfg::kWq;
-        CUtensorMap mq, mdo, mkk, mkmn, mvk, mdq;
-        if ((st = kmap(&mq, q, kTileRows, BH, N)) != FA2_OK || (st = kmap(&mdo, dout, kTileRows, BH, N)) != FA2_OK ||
-            (st = kmap(&mkk, k, W, BH_kv, Nk)) != FA2_OK || (st = mnmap(&mkmn, k, W, BH_kv, Nk)) != FA2_OK ||
-            (st = kmap(&mvk, v, W, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows, BH, N)) != FA2_OK)
-            return st;
-        auto kern = fa2_bwd32_dq_kernel<D>;
-        if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemQ, stream>>>(mq, mdo, mkk, mkmn, mvk, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
     }
     return FA2_OK;
@@ -385,7 +443,7 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
                            int H, int H_kv, int N, int Nk, int d, int causal, float scale, fa2_dtype dtype,
                            uint8_t* ws_base, const BwdWorkspace& ws, cudaStream_t stream,
                            uint32_t* status, unsigned long long timeout_ns, void* const* events,
-                           const uint8_t* block_mask = nullptr) {
+                           const uint8_t* block_mask, unsigned flags) {
 #define FA2_BWD_CASE(DD)                                                                      \
     case DD:                                                                                  \
         if (dtype == FA2_FP32)                                                                \
@@ -394,10 +452,11 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
         if (dtype == FA2_FP16)                                                                \
             return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, \
                                                   causal, scale, dtype, ws_base, ws, stream,    \
-                                                  status, timeout_ns, events, block_mask);      \
+                                                  status, timeout_ns, events, block_mask,       \
+                                                  flags);                                       \
         return launch_backward_t<2, DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, causal, \
                                         scale, dtype, ws_base, ws, stream, status, timeout_ns, events, \
-                                        block_mask);
+                                        block_mask, flags);
     switch (d) {
         FA2_BWD_CASE(16)
         FA2_BWD_CASE(32)
@@ -467,7 +526,8 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
                          const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                          int H, int H_kv, int N, int Nk, int d, int causal, float scale,
                          fa2_dtype dtype, void* workspace, size_t workspace_bytes,
-                         fa2_stream_t stream, void* const* events, const uint8_t* block_mask = nullptr) {
+                         fa2_stream_t stream, void* const* events, const uint8_t* block_mask = nullptr,
+                         unsigned flags = 0) {
     fa2_status st = check_common(B, H, N, d, causal, scale, dtype);
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
@@ -479,7 +539,11 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4) || !aligned(workspace, 256))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H_kv, Nk, d, dtype == FA2_FP32 ? 4 : 2);
+    // The two-pass form needs no dQ accumulator, so it accepts the smaller workspace.
+    const bool two_pass_only = (flags & FA2_BWD_DETERMINISTIC) ||
+                               (!kOnePassDefault && !(flags & FA2_BWD_ONE_PASS)) || block_mask;
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H_kv, Nk, d, dtype == FA2_FP32 ? 4 : 2,
+                                                 !two_pass_only);
     if (workspace_bytes < ws.total) return FA2_ERR_WORKSPACE_TOO_SMALL;
     int dev;
     uint32_t* status;
@@ -487,7 +551,7 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                            dtype, static_cast<uint8_t*>(workspace), ws, s, status,
-                           kDefaultTimeoutNs, events, block_mask);
+                           kDefaultTimeoutNs, events, block_mask, flags);
 }
 
 }  // namespace
@@ -563,6 +627,18 @@ fa2_status fa2_backward_block_sparse(const void* q, const void* k, const void* v
     if (!block_mask) return FA2_ERR_NULL_PTR;
     return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
                          dtype, workspace, workspace_bytes, stream, nullptr, block_mask);
+}
+
+fa2_status fa2_backward_opts(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                             fa2_dtype dtype, const uint8_t* block_mask, unsigned flags,
+                             void* workspace, size_t workspace_bytes, fa2_stream_t stream) {
+    if ((flags & ~(FA2_BWD_DETERMINISTIC | FA2_BWD_ONE_PASS)) ||
+        ((flags & FA2_BWD_DETERMINISTIC) && (flags & FA2_BWD_ONE_PASS)))
+        return FA2_ERR_BAD_ARGUMENT;
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, d, causal, scale,
+                         dtype, workspace, workspace_bytes, stream, nullptr, block_mask, flags);
 }
 
 fa2_status fa2_last_device_status(void) {
@@ -650,7 +726,8 @@ extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const v
         !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
         !aligned(lse, 4))
         return FA2_ERR_MISALIGNED;
-    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H, N, d, dtype == FA2_FP32 ? 4 : 2);
+    // The two-pass (deterministic) form: its scratch holds no dQ accumulator.
+    const BwdWorkspace ws = bwd_workspace_layout(B * H, N, B * H, N, d, dtype == FA2_FP32 ? 4 : 2, false);
     if (ws.total > kNoAllocScratchBytes) return FA2_ERR_SCRATCH_TOO_SMALL;
     int dev;
     uint32_t* status;
@@ -659,7 +736,7 @@ extern "C" fa2_status fa2_backward_noalloc(const void* q, const void* k, const v
     if ((st = noalloc_scratch(dev, &scratch)) != FA2_OK) return st;
     return launch_backward(q, k, v, o, lse, dout, dq, dk, dv, B, H, H, N, N, d, causal, scale, dtype,
                            scratch, ws, reinterpret_cast<cudaStream_t>(stream), status,
-                           kDefaultTimeoutNs, nullptr);
+                           kDefaultTimeoutNs, nullptr, nullptr, FA2_BWD_DETERMINISTIC);
 }
 
 // ---------------------------------------------------------------------------

@@ -48,7 +48,7 @@ namespace fa2 {
 // dout ([BH][N][d]) and of k and v ([BH_kv][Nk][d]) rounded to TF32 (offsets 0
 // when absent).
 struct BwdWorkspace {
-    size_t l2_off, d_off, q_off, k_off, v_off, do_off, part_off, total;
+    size_t l2_off, d_off, q_off, k_off, v_off, do_off, part_off, dqacc_off, total;
     int n_pad;
     int kv_splits;   // dK/dV pass: CTAs per (key tile, key/value head)
 };
@@ -71,20 +71,33 @@ __host__ __device__ inline int dkdv_splits(int n_tiles_k, int BH_kv, int group) 
     return static_cast<int>(want < group ? want : group);
 }
 
-inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d, int elem_bytes) {
+// The one-pass backward (fa2_bwd_fused.cuh) runs where it applies: 16-bit
+// inputs, no block mask, no split dK/dV groups, more than one key tile.
+inline bool one_pass_applies(int n_tiles_k, int elem_bytes, int kv_splits, bool block_sparse) {
+    return elem_bytes == 2 && !block_sparse && kv_splits == 1 && n_tiles_k > 1;
+}
+
+// with_dq_acc: also reserve the one-pass backward's fp32 dQ accumulator
+// [BH][n_pad][d] when the one-pass backward applies to these sizes.
+inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d, int elem_bytes,
+                                         bool with_dq_acc = true) {
     BwdWorkspace w;
     w.n_pad = (N + kTileRows - 1) / kTileRows * kTileRows;
     const size_t vec = align256(static_cast<size_t>(BH) * w.n_pad * sizeof(float));
     w.l2_off = 0;
     w.d_off = vec;
     w.total = 2 * vec;
-    w.q_off = w.k_off = w.v_off = w.do_off = w.part_off = 0;
+    w.q_off = w.k_off = w.v_off = w.do_off = w.part_off = w.dqacc_off = 0;
     const int n_tiles_k = (Nk + kTileRows - 1) / kTileRows;
     w.kv_splits = elem_bytes == 2 ? dkdv_splits(n_tiles_k, BH_kv, BH / BH_kv) : 1;
     if (w.kv_splits > 1) {
         // fp32 partial dK and dV: [2][splits][BH_kv][n_tiles_k * 128][d]
         w.part_off = w.total;
         w.total += align256(2ull * w.kv_splits * BH_kv * n_tiles_k * kTileRows * d * sizeof(float));
+    }
+    if (with_dq_acc && one_pass_applies(n_tiles_k, elem_bytes, w.kv_splits, false)) {
+        w.dqacc_off = w.total;
+        w.total += align256(static_cast<size_t>(BH) * w.n_pad * d * sizeof(float));
     }
     if (elem_bytes == 4) {
         const size_t tq = align256(static_cast<size_t>(BH) * N * d * sizeof(float));
@@ -114,11 +127,14 @@ struct BwdPreCfg {
 // D_i = rowsum(O_i o dO_i) and L_i * log2(e) per query row; rows past N (up
 // to the padded length) get D = 0 and L = +inf so they drop out of P and dS.
 // O and dO are 16-bit (bf16, or fp16 when F16), read as raw 16-bit pairs.
+// With dq_acc (the one-pass backward's fp32 dQ accumulator, [BH][n_pad][D])
+// the row is also zeroed there.
 template <int D, bool F16 = false>
 __global__ void __launch_bounds__(256)
 fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                    const float* __restrict__ lse, float* __restrict__ l2,
-                   float* __restrict__ dvec, int N, int n_pad, long long rows_total) {
+                   float* __restrict__ dvec, int N, int n_pad, long long rows_total,
+                   float* __restrict__ dq_acc = nullptr) {
     using C = BwdPreCfg<D>;
     const int sub = threadIdx.x % C::kTPR;
     const long long row = static_cast<long long>(blockIdx.x) * C::kRowsPerBlock + threadIdx.x / C::kTPR;
@@ -126,6 +142,11 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ 
     const long long bh = row / n_pad;
     const int n = static_cast<int>(row - bh * n_pad);
     float acc = 0.f;
+    if (dq_acc && live && sub < C::kUsed) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + row * D + sub * C::kVec);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (live && n < N && sub < C::kUsed) {
         const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * C::kVec;
         const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + base));
@@ -158,7 +179,8 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ 
 
 struct BwdParams {
     const float* l2;       // [BH][n_pad]  L * log2(e), +inf past N
-    const float* dvec;     // [BH][n_pad]  D, 0 past N
+    float* dvec;           // [BH][n_pad]  D, 0 past N (the dQ pass rewrites the
+                           // rows of a query tile that sees a single key tile)
     uint32_t* status;
     int N, BH, n_tiles, n_pad, causal;   // query length, B * H, query tiles, padded rows
     int Nk, n_tiles_k;                   // key/value length and tiles
@@ -169,6 +191,7 @@ struct BwdParams {
     const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
     int kv_splits;         // dK/dV pass CTAs per (key tile, key/value head)
     float* part;           // fp32 partial dK, dV when kv_splits > 1
+    int item0;             // dQ pass: work item of the first CTA (a launch may cover a suffix)
 };
 
 template <int ES, int D, bool F16 = false>
@@ -239,6 +262,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // Block-sparse: the query tiles whose block with this key tile is set.
     __shared__ uint16_t s_q[SPARSE ? kMaxMaskTiles : 1];
     __shared__ int s_nq;
+    // Block-sparse, causal: the query tile kv_tile (the diagonal step) has no set
+    // block before this key tile, so its rows see this key tile only.
+    __shared__ int s_diag_single;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -266,7 +292,13 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int n = warp_compact(s_q, p.n_tiles > i_begin ? p.n_tiles - i_begin : 0,
             [&](int t) { return p.block_mask[static_cast<size_t>(i_begin + t) * p.n_tiles_k + kv_tile] != 0; },
             [&](int t) { return i_begin + t; });
-        if (lane == 0) s_nq = n;
+        bool before = false;
+        if (p.causal && kv_tile < p.n_tiles) {
+            const uint8_t* row = p.block_mask + static_cast<size_t>(kv_tile) * p.n_tiles_k;
+            for (int base = 0; base < kv_tile; base += 32)
+                before |= __any_sync(0xffffffffu, base + lane < kv_tile && row[base + lane] != 0);
+        }
+        if (lane == 0) { s_nq = n; s_diag_single = before ? 0 : 1; }
     }
 
     if (threadIdx.x == 0) {
@@ -311,6 +343,15 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         return sparse ? static_cast<int>(s_q[g]) : i_begin + g;
     };
     auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + (it0 + it) / n_q; };
+    // Steps whose query tile sees this key tile only (causal: query tile 0, or
+    // with a block mask the diagonal step of a block row with nothing before
+    // it; or a single key tile), where rows see few keys and |dS| is of the
+    // order of |dP|: dS^T goes to the dK MMA as two 16-bit parts hi + lo, so it
+    // is not rounded before the contraction.  With a mask of all ones this is
+    // the rule without a mask.
+    auto hilo_of = [&](int i) {
+        return p.n_tiles_k == 1 || (p.causal && (sparse ? (i == kv_tile && s_diag_single != 0) : i == 0));
+    };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -402,6 +443,12 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
                     ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                if (hilo_of(q_tile_of(it))) {
+                    // dK_j += dS^T_lo Q_i: the low parts sit 32 columns after the high parts.
+#pragma unroll
+                    for (int kk = 0; kk < G::kStepsRows; ++kk)
+                        ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col(kk) + 32, desc_mnmajor<G>(qa, kk), idesc_kv, 1u);
+                }
                 ptx::mma_commit(&bar_q_empty[it % RS]);
                 if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
             }
@@ -503,6 +550,46 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- dS^T = P^T o (dP^T - D)   (Eq. 17)
             if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
+            if (hilo_of(i)) {
+                // dS^T = hi + lo, both rounded to the 16-bit type: hi into the group's
+                // first 32 dP^T columns, lo into the next 32 (the issuer's second dK
+                // group reads them).  Columns are overwritten only after they are read.
+                uint32_t lo_a[16];
+                {
+                    uint32_t ud[32], hi[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0, ud);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[c >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])),
+                                                                  make_float2(-sDv[wi][b][c], -sDv[wi][b][c + 1])));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo_a[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0, hi);          // hi, values 0..31
+                }
+                {
+                    uint32_t ud[32], hi[16], lo[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32, ud);
+                    ptx::tmem_wait_ld();
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 32, lo_a);     // lo, values 0..31
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[(32 + c) >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])),
+                                                                  make_float2(-sDv[wi][b][32 + c], -sDv[wi][b][33 + c])));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 16, hi);     // hi, values 32..63
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 48, lo);     // lo, values 32..63
+                }
+            } else {
             uint32_t dk[32];                               // this group's dS^T row, bf16 pairs
             {
                 uint32_t ud[64];
@@ -525,6 +612,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // dS^T -> this group's own dP^T columns [128 + 64g, ... + 32), A operand
             // of dK += dS^T Q.
             ptx::tmem_st32(lane_base + Cfg::kColDP + qc0, dk);
+            }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -693,8 +781,10 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: causal query tile i sees key tiles 0..i; longest first.
-    const int item = blockIdx.x;
+    // Work item: causal query tile i sees key tiles 0..i; longest first.  A
+    // launch may cover only the last items (item0 > 0: the single-tile query
+    // tiles ahead of the one-pass backward).
+    const int item = blockIdx.x + p.item0;
     const int rank = item / p.BH;
     const int bh = item - rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
@@ -743,6 +833,11 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // (nothing is loaded, so the Q slot can stage the zeros).
     const int n_kv = sparse ? s_nkv : n_kv_lim;
     auto kv_of = [&](int j) { return sparse ? static_cast<int>(s_kv[j]) : j; };
+    // A query tile that sees one key tile only (causal: the first query tile;
+    // or a single key tile; or a block row with one block): every key its rows
+    // see is in that tile, so those rows take D from the tile's own P and dP and
+    // their dS goes to the dQ MMA as two 16-bit parts (see the groups below).
+    const bool single = n_kv == 1;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -831,6 +926,12 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                     for (int kk = 0; kk < G::kStepsRows; ++kk)
                         ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                    if (single) {
+                        // dQ += dS_lo K_j: the low parts sit 32 columns after the high parts.
+#pragma unroll
+                        for (int kk = 0; kk < G::kStepsRows; ++kk)
+                            ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + a_col(kk) + 32, desc_mnmajor<G>(ka, kk), idesc_dq, 1u);
+                    }
                     ptx::mma_commit(&bar_k_empty[j % RK]);
                     if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
                 }
@@ -853,7 +954,101 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const float l2r = p.l2[vrow];                    // L_i * log2(e) (+inf past N)
         const float dr = p.dvec[vrow];                   // D_i (0 past N)
         bool ok = true;
-        for (int j = 0; j < n_kv; ++j) {
+        if (single) {
+            // The rows of this tile see no other key tile (kv_of(0) is the only one), so
+            //   D_i = sum_j P_ij dP_ij
+            // (the softmax-Jacobian form of rowsum(O o dO), equal to it in exact
+            // arithmetic) is formed here from the recomputed P and dP.  Rows that see
+            // only a few keys have |dS| of the order of |dP|, and there D taken from
+            // the rounded O is not accurate enough; this D keeps sum_j dS_ij = 0.  It
+            // is written back for the dK/dV pass.  D uses the fp32 P; dS = P_16 (dP -
+            // D), with P_16 the 16-bit P the other passes use, goes to the dQ MMA as
+            // two 16-bit parts: hi into the group's first 32 dP columns, lo into the
+            // next 32.  With one key tile there is nothing to overlap, so both S and dP
+            // are awaited first.  Every elementwise thread reaches the named barrier
+            // below exactly once, also when a wait gave up.
+            const int kv = kv_of(0);
+            const bool diag = p.causal && (kv == q_tile);
+            const int kv_valid = p.Nk - kv * kTileRows - kc0;
+            uint32_t pk[32];
+            bool got = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_s_full, 0, &abort_flag, tmo) &&
+                                                   ptx::mbar_wait(&bar_dp_full, 0, &abort_flag, tmo));
+            float part = 0.f;
+            if (got) {
+                ptx::tc_fence_after();
+                const float2 sl2v = make_float2(sl2, sl2), nl2v = make_float2(-l2r, -l2r);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t us[32], ud[32];
+                    ptx::tmem_ld32(lane_base + Cfg::kColS + kc0 + 32 * h, us);
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0 + 32 * h, ud);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        const int cc = 32 * h + c;
+                        const float2 a = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, nl2v);
+                        const float p0 = ((diag && kc0 + cc > r) || cc >= kv_valid) ? 0.f : ptx::ex2_approx(a.x);
+                        const float p1 = ((diag && kc0 + cc + 1 > r) || cc + 1 >= kv_valid) ? 0.f : ptx::ex2_approx(a.y);
+                        pk[cc >> 1] = G::pack2(p0, p1);
+                        part = fmaf(p0, __uint_as_float(ud[c]), part);
+                        part = fmaf(p1, __uint_as_float(ud[c + 1]), part);
+                    }
+                }
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_s_read);
+            }
+            // Both groups' partial sums meet in the V ring's second slot (unused: this
+            // CTA loads one key tile).
+            float* s_dpart = reinterpret_cast<float*>(sVr + TB);
+            s_dpart[g * kTileRows + r] = part;
+            asm volatile("bar.sync 3, 256;" ::: "memory");
+            if (!got) {
+                ok = false;
+            } else {
+                const float dfull = s_dpart[r] + s_dpart[kTileRows + r];
+                if (g == 0 && q_row0 + r < p.N) p.dvec[vrow] = dfull;
+                const float2 ndv = make_float2(-dfull, -dfull);
+                uint32_t lo_a[16];
+                {
+                    uint32_t ud[32], hi[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0, ud);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[c >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])), ndv));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo_a[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + kc0, hi);          // dS_hi, values 0..31
+                }
+                {
+                    uint32_t ud[32], hi[16], lo[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0 + 32, ud);
+                    ptx::tmem_wait_ld();
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + kc0 + 32, lo_a);     // dS_lo, values 0..31
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[(32 + c) >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])), ndv));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + kc0 + 16, hi);     // dS_hi, values 32..63
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + kc0 + 48, lo);     // dS_lo, values 32..63
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+            }
+        }
+        for (int j = 0; !single && j < n_kv; ++j) {
             const int kv = kv_of(j);
             const bool diag = p.causal && (kv == q_tile);
             const int kv_valid = p.Nk - kv * kTileRows - kc0;  // this group's key columns < Nk

@@ -190,6 +190,11 @@ __device__ __forceinline__ void tma_store_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
+// Wait until at most one committed bulk group still has to read its source.
+__device__ __forceinline__ void tma_store_wait_read_1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy
 // (TMA stores, MMA operand reads).
 __device__ __forceinline__ void fence_async_smem() {

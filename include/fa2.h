@@ -37,7 +37,11 @@
  *     fa2_last_device_status() reads once the caller has synchronised.
  *   - Thread safety: entry points may be called concurrently from several
  *     host threads; the only shared host state is a mutex-guarded cache of
- *     per-device kernel attributes.
+ *     per-device kernel attributes and of the device addresses of the
+ *     library's own device variables (the status word, the scratch array of
+ *     fa2_backward_noalloc), looked up once per device.  A device reset
+ *     (cudaDeviceReset) invalidates those addresses: the library is not
+ *     usable on that device afterwards in the same process.
  */
 #ifndef FA2_H_
 #define FA2_H_
@@ -115,10 +119,12 @@ fa2_status fa2_forward_ex(const void* q, const void* k, const void* v, void* o, 
 
 /*
  * Bytes of device workspace fa2_backward needs for these sizes: the fp32 D
- * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes, and
- * for FA2_FP32 also copies of q, k, v and dout rounded to TF32 (round to
- * nearest), 4 * 4 * B * H * N * d bytes (every region rounded up to 256
- * bytes).  Returns 0 for arguments fa2_backward would reject.
+ * and log2-scaled L vectors, 2 * 4 * B * H * ceil(N / 128) * 128 bytes; for
+ * 16-bit inputs with N > 128 (where the one-pass form of fa2_backward_opts
+ * can run) also the fp32 dQ accumulator, 4 * B * H * ceil(N / 128) * 128 * d bytes; for FA2_FP32 instead
+ * copies of q, k, v and dout rounded to TF32 (round to nearest),
+ * 4 * 4 * B * H * N * d bytes (every region rounded up to 256 bytes).
+ * Returns 0 for arguments fa2_backward would reject.
  */
 size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype);
 
@@ -129,7 +135,8 @@ size_t fa2_backward_workspace_bytes(int B, int H, int N, int d, fa2_dtype dtype)
  * H_kv < H) the dK/dV pass splits each query-head group over S =
  * min(H / H_kv, ceil(296 / (ceil(Nk / 128) * B * H_kv))) thread blocks whose
  * fp32 partial dK and dV, 2 * S * B * H_kv * ceil(Nk / 128) * 128 * d * 4
- * bytes, are summed in a fixed order afterwards.  Returns 0 for arguments
+ * bytes, are summed in a fixed order afterwards (such problems take the
+ * two-pass form and need no dQ accumulator).  Returns 0 for arguments
  * fa2_backward_ex would reject.
  */
 size_t fa2_backward_workspace_bytes_ex(int B, int H, int H_kv, int N, int Nk, int d,
@@ -138,16 +145,22 @@ size_t fa2_backward_workspace_bytes_ex(int B, int H, int H_kv, int N, int Nk, in
 /*
  * Backward pass with recomputation (handout section 4.2.2, Eqs. 13-19;
  * D = rowsum(O o dO)), organised as the handout's Algorithm 2 (section
- * 4.2.3): one pass over key/value tiles accumulates dK and dV, a second pass
- * over query tiles recomputes P and accumulates dQ, so nothing is added
- * across thread blocks.
+ * 4.2.3): one pass over query tiles recomputes P and accumulates dQ, a second
+ * pass over key/value tiles accumulates dK and dV, so nothing is added across
+ * thread blocks.  Rows of a query tile that sees a single key tile (causal:
+ * the first 128 rows) take D in its equivalent form sum_j P_ij dP_ij from the
+ * recomputed P and dP, and their dS enters the dQ and dK contractions as two
+ * 16-bit parts (hi + lo); these rows see few keys, so |dS| is of the order of
+ * |dP| and D from the rounded O would not be accurate enough.
  *   q, k, v, o, dout  in : [B, H, N, d] `dtype` (o as produced by fa2_forward)
  *   lse               in : [B, H, N] float32 from fa2_forward
  *   dq, dk, dv        out: [B, H, N, d] `dtype`
  *   workspace         scratch of at least fa2_backward_workspace_bytes bytes,
  *                     256-byte aligned, owned by the caller; its contents on
  *                     entry do not matter and on return are unspecified
- * Every output is deterministic (bitwise equal from run to run).
+ * This is fa2_backward_opts with flags = 0 (the two-pass form: every output
+ * is bitwise reproducible); fa2_backward_opts with FA2_BWD_ONE_PASS selects
+ * the one-pass form.
  */
 fa2_status fa2_backward(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, void* dq, void* dk, void* dv,
@@ -199,13 +212,54 @@ fa2_status fa2_backward_block_sparse(const void* q, const void* k, const void* v
                                      const uint8_t* block_mask, void* workspace,
                                      size_t workspace_bytes, fa2_stream_t stream);
 
+/* Flags of fa2_backward_opts. */
+#define FA2_BWD_DETERMINISTIC 1u
+#define FA2_BWD_ONE_PASS 2u
+
+/*
+ * The backward pass with a choice of organisation; fa2_backward,
+ * fa2_backward_ex and fa2_backward_block_sparse are this entry point with
+ * flags = 0.
+ *
+ * FA2_BWD_DETERMINISTIC: the two-pass form described at fa2_backward (the
+ *   handout's Algorithm 2, section 4.2.3): every output bitwise reproducible.
+ * FA2_BWD_ONE_PASS: where it applies -- 16-bit inputs, no block mask, more
+ *   than one key tile (Nk > 128), and dK/dV work not split across thread
+ *   blocks (see fa2_backward_workspace_bytes_ex) -- ONE pass over key/value
+ *   tiles (the FlashAttention-2 backward with the key/value tile outermost,
+ *   handout section 4.2.2): P, dP and dS are computed once per (key tile,
+ *   query tile) pair, and each key tile's contribution scale * dS K to dQ is
+ *   added into an fp32 accumulator in the workspace with TMA reduce-add; a
+ *   last kernel rounds dQ once.  dK and dV are bitwise reproducible (and
+ *   equal to the two-pass form's); the BITS OF dQ DEPEND ON THE ORDER in which
+ *   key tiles' contributions arrive and can change from run to run (the
+ *   result stays within the same tolerance).  Query tiles whose rows see a
+ *   single key tile (causal: the first 128 rows) take their dQ and D from the
+ *   two-pass form's query-tile pass.  Where the one-pass form does not apply,
+ *   the two-pass form runs.
+ * 0: currently the two-pass form.
+ * Both bits together, or any other bit, give FA2_ERR_BAD_ARGUMENT.
+ * block_mask: NULL, or the block mask of fa2_backward_block_sparse.
+ * workspace: fa2_backward_workspace_bytes_ex(...) bytes, which covers both
+ *   forms; the two-pass form also accepts the same size without the dQ
+ *   accumulator (4 * B * H * ceil(N / 128) * 128 * d bytes, rounded up to 256).
+ */
+fa2_status fa2_backward_opts(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int H, int H_kv, int N, int Nk, int d, int causal, float scale,
+                             fa2_dtype dtype, const uint8_t* block_mask, unsigned flags,
+                             void* workspace, size_t workspace_bytes, fa2_stream_t stream);
+
 /*
  * fa2_backward plus timing hooks, for profiling: identical arguments and
  * behaviour, and additionally records the caller's CUDA events (cudaEvent_t
  * handles created on the current device; any entry may be NULL) on `stream`
- * at the boundaries of the three kernels the backward enqueues:
+ * at the boundaries of the kernels the backward enqueues:
  *   events[0] before the D / L pre-pass,   events[1] after it,
- *   events[2] after the dK / dV pass,      events[3] after the dQ pass.
+ *   events[2] after the pass over query tiles (two-pass form: the dQ pass;
+ *             one-pass form: that pass on the single-tile query tiles),
+ *   events[3] after the pass over key tiles (the one-pass form then enqueues
+ *             one more kernel, which rounds dQ).
  * `events` itself may be NULL (then this is fa2_backward).  The library only
  * records the events; the caller owns and destroys them.
  */
@@ -239,7 +293,9 @@ fa2_status fa2_backward_timed(const void* q, const void* k, const void* v, const
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call on a device shares the one array:
+ * before any stream capture.  The address is kept for the life of the
+ * process: after cudaDeviceReset on a device (which frees the array with the
+ * context) this entry point must not be called on that device again.  Every call on a device shares the one array:
  * the kernels re-initialise all of it that must start from zero, but two
  * calls whose work overlaps on the GPU (different streams, no ordering
  * between them) race on it and give wrong results.  Order such calls on one

@@ -35,10 +35,13 @@ int main(void) {
     }
     CHECK(strcmp(fa2_status_string(FA2_OK), "FA2_OK") == 0);
 
-    /* Workspace: two fp32 [B*H][ceil(N/128)*128] regions, each rounded up to
-     * 256 bytes, for 16-bit inputs; the _ex form agrees with MHA shapes. */
+    /* Workspace: two fp32 [B*H][ceil(N/128)*128] regions and, with more than
+     * one key tile, the fp32 dQ accumulator [B*H][ceil(N/128)*128][d], each
+     * rounded up to 256 bytes, for 16-bit inputs; the _ex form agrees with
+     * MHA shapes. */
     size_t ws = fa2_backward_workspace_bytes(2, 3, 200, 80, FA2_BF16);
-    CHECK(ws == 2 * (size_t)(2 * 3 * 256 * 4));
+    CHECK(ws == 2 * (size_t)(2 * 3 * 256 * 4) + (size_t)(2 * 3 * 256 * 80 * 4));
+    CHECK(fa2_backward_workspace_bytes(2, 3, 128, 80, FA2_BF16) == 2 * (size_t)(2 * 3 * 128 * 4));
     CHECK(fa2_backward_workspace_bytes_ex(2, 3, 3, 200, 200, 80, FA2_BF16) == ws);
     CHECK(fa2_backward_workspace_bytes(2, 3, 200, 80, FA2_FP16) == ws);
     CHECK(fa2_backward_workspace_bytes(2, 3, 200, 24, FA2_BF16) == 0);
@@ -58,6 +61,16 @@ int main(void) {
                        FA2_BF16, P, need - 1, NULL) == FA2_ERR_WORKSPACE_TOO_SMALL);
     CHECK(fa2_backward(P, P, P, P, (const float*)P, P, P, P, P, 1, 2, 128, 64, 1, 0.125f,
                        FA2_BF16, (char*)P + 16, need, NULL) == FA2_ERR_MISALIGNED);
+
+    /* Backward options: unknown flag bits are rejected before anything else. */
+    CHECK(fa2_backward_opts(P, P, P, P, (const float*)P, P, P, P, P, 1, 2, 2, 128, 128, 64, 1,
+                            0.125f, FA2_BF16, NULL, 4u, P, need, NULL) == FA2_ERR_BAD_ARGUMENT);
+    CHECK(fa2_backward_opts(P, P, P, P, (const float*)P, P, P, P, P, 1, 2, 2, 128, 128, 64, 1,
+                            0.125f, FA2_BF16, NULL, FA2_BWD_DETERMINISTIC | FA2_BWD_ONE_PASS, P,
+                            need, NULL) == FA2_ERR_BAD_ARGUMENT);
+    CHECK(fa2_backward_opts(P, P, P, P, (const float*)P, P, P, P, P, 1, 2, 2, 128, 128, 64, 1,
+                            0.125f, FA2_BF16, NULL, FA2_BWD_DETERMINISTIC, P, need - 1, NULL) ==
+          FA2_ERR_WORKSPACE_TOO_SMALL);
 
     /* Grouped-query shapes: H must be a multiple of H_kv. */
     CHECK(fa2_forward_ex(P, P, P, P, (float*)P, 1, 6, 4, 128, 128, 64, 1, 0.125f, FA2_BF16,

@@ -34,7 +34,10 @@ def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, name: str) -> flo
     return float(err.max()) if err.size else 0.0
 
 
-def gpu_fwd_bwd(inp, causal: bool, scale: float, do_backward: bool = True):
+def gpu_fwd_bwd(inp, causal: bool, scale: float, do_backward: bool = True,
+                mode: str = "default"):
+    """Forward and backward on cuda:0 through the binding; ``mode`` is the
+    backward's form ("default", "two-pass" or "one-pass")."""
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
@@ -42,7 +45,8 @@ def gpu_fwd_bwd(inp, causal: bool, scale: float, do_backward: bool = True):
     out = {"o": o, "lse": lse}
     if do_backward:
         do = inp["do"].to(dev)
-        dq, dk, dv = fa2.backward(q, k, v, o, lse, do, causal=causal, scale=scale)
+        dq, dk, dv = fa2.backward(q, k, v, o, lse, do, causal=causal, scale=scale,
+                                  mode=mode)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     return out

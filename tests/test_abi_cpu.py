@@ -95,13 +95,16 @@ def test_backward_validation(fa2lib):
 @pytest.mark.parametrize("B,H,N,d", [(1, 1, 1, 16), (2, 3, 200, 80), (1, 36, 4096, 128)])
 def test_workspace_size(fa2lib, B, H, N, d):
     """D and log2-scaled L (fp32, padded to whole 128-row tiles), each region
-    rounded up to 256 bytes; for fp32 inputs also four operand copies."""
+    rounded up to 256 bytes; for 16-bit inputs with more than one key tile
+    also the one-pass backward's fp32 dQ accumulator; for fp32 inputs four
+    operand copies instead."""
     def up(x):
         return (x + 255) // 256 * 256
     n_pad = (N + 127) // 128 * 128
     expect = 2 * up(B * H * n_pad * 4)
-    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect
-    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 2) == expect      # fp16
+    acc = up(B * H * n_pad * d * 4) if N > 128 else 0
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 0) == expect + acc
+    assert fa2lib.fa2_backward_workspace_bytes(B, H, N, d, 2) == expect + acc  # fp16
     for dt in (0, 1, 2):
         assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, H, N, N, d, dt) == \
             fa2lib.fa2_backward_workspace_bytes(B, H, N, d, dt)
@@ -195,8 +198,10 @@ def test_workspace_size_split_groups(fa2lib):
         ctas = tk * B * hkv
         S = 1 if ctas >= 148 else min(H // hkv, -(-296 // ctas))
         part = up(2 * S * B * hkv * tk * 128 * d * 4) if S > 1 else 0
+        # no split and more than one key tile: the one-pass form's dQ accumulator
+        acc = up(B * H * n_pad * d * 4) if (S == 1 and tk > 1) else 0
         for dt in (0, 2):
-            assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, hkv, N, nk, d, dt) == base + part, (B, H, hkv, S)
+            assert fa2lib.fa2_backward_workspace_bytes_ex(B, H, hkv, N, nk, d, dt) == base + part + acc, (B, H, hkv, S)
     # multi-head: never split
     assert fa2lib.fa2_backward_workspace_bytes_ex(1, 4, 4, 256, 256, 64, 0) == \
         fa2lib.fa2_backward_workspace_bytes(1, 4, 256, 64, 0)

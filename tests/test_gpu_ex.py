@@ -51,13 +51,27 @@ def _inputs(B, H, H_kv, N, Nk, d, dtype, seed):
 
 @pytest.mark.parametrize("B,H,H_kv,N,Nk,d,dtype,causal", CASES)
 def test_ex_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal):
+    q, k, v, do = _inputs(B, H, H_kv, N, Nk, d, dtype, seed=131 + N + d + H_kv + Nk)
+    _check_against_oracle(oracle_mod, q, k, v, do, causal, dtype, f"ex B={B} H={H} H_kv={H_kv} N={N} Nk={Nk} d={d} {dtype}")
+
+
+def test_mqa_early_row_regression(oracle_mod):
+    """The input on which dQ of causal query row 1 once exceeded the bound
+    (0.0169 against 0.0107): multi-query bf16, B=2, H=6, H_kv=1, N=256, d=128,
+    inputs drawn with seed 31 + N + d + H_kv = 416.  Row 1 sees two keys, so
+    dS_1j is of the order of |dP|; the kernels now take D of the first query
+    tile from P and dP and pass its dS in two 16-bit parts.  Same bound as every
+    other case."""
+    B, H, H_kv, N, d = 2, 6, 1, 256, 128
+    q, k, v, do = _inputs(B, H, H_kv, N, N, d, "bf16", seed=31 + N + d + H_kv)
+    _check_against_oracle(oracle_mod, q, k, v, do, True, "bf16", "mqa-regression seed 416")
+
+
+def _check_against_oracle(oracle_mod, q, k, v, do, causal, dtype, label):
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
-    # (With seed 31 + N + d + H_kv the multi-query bf16 case had one dQ element
-    # of query row 1 at 1.6x the bound: with two visible keys each dS_1j is
-    # large and its bf16 rounding before the dQ MMA shows; recorded in the
-    # design notes as a property of the 16-bit dS, not of the head mapping.)
-    q, k, v, do = _inputs(B, H, H_kv, N, Nk, d, dtype, seed=131 + N + d + H_kv + Nk)
+    B, H, N, d = q.shape
+    H_kv, Nk = k.shape[1], k.shape[2]
     scale = default_scale(d)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o, lse = fa2.forward(qd, kd, vd, causal=causal, scale=scale)
@@ -71,10 +85,11 @@ def test_ex_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal):
     # dK and dV add up `group` per-head gradients; the tolerance is the
     # per-element one of a single gradient, scaled by the group size.
     for name, got in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        err = np.abs(to64(got) - ref[name])
+        tol = TOLS[dtype]
+        print(f"RATIO {label} {name} {float((err / (tol + tol * np.abs(ref[name]))).max()):.3f}")
         if name in ("dk", "dv"):
             grp = H // H_kv
-            err = np.abs(to64(got) - ref[name])
-            tol = TOLS[dtype]
             assert (err <= grp * (tol + tol * np.abs(ref[name]) / grp)).all(), (name, err.max())
         else:
             assert_close(to64(got), ref[name], dtype, name)
@@ -108,7 +123,9 @@ def test_ex_with_mha_shapes_is_bitwise_mha():
                                B, H, H, N, N, d, 1, scale, 0, ws.data_ptr(), ws.numel(), s) == 0
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
-    assert all(torch.equal(a, b) for a, b in zip(ref, g))
+    # dK, dV bitwise; dQ of the one-pass form is summed by reduce-add (order-dependent bits).
+    assert torch.equal(ref[1], g[1]) and torch.equal(ref[2], g[2])
+    torch.testing.assert_close(ref[0].float(), g[0].float(), atol=1e-3, rtol=1e-2)
 
 
 def test_gqa_backward_deterministic():
@@ -116,7 +133,7 @@ def test_gqa_backward_deterministic():
     dev = torch.device("cuda", 0)
     q, k, v, do = (t.to(dev) for t in _inputs(2, 8, 2, 512, 700, 128, "bf16", seed=5))
     o, lse = fa2.forward(q, k, v)
-    g1 = fa2.backward(q, k, v, o, lse, do)
-    g2 = fa2.backward(q, k, v, o, lse, do)
+    g1 = fa2.backward(q, k, v, o, lse, do, mode="two-pass")
+    g2 = fa2.backward(q, k, v, o, lse, do, mode="two-pass")
     torch.cuda.synchronize()
     assert all(torch.equal(a, b) for a, b in zip(g1, g2))

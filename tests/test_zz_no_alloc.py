@@ -21,31 +21,42 @@ pytestmark = pytest.mark.gpu
 SCRATCH_BYTES = 64 << 20
 
 
-def _call_noalloc(lib, q, k, v, o, lse, do, dq, dk, dv, causal, scale):
+DTYPE_CODE = {"bf16": 0, "fp32": 1, "fp16": 2}
+
+
+def _call_noalloc(lib, q, k, v, o, lse, do, dq, dk, dv, causal, scale, dtype):
     B, H, N, d = q.shape
     return lib.fa2_backward_noalloc(
         q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(causal), float(scale), 0,
-        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, N, d, int(causal), float(scale),
+        DTYPE_CODE[dtype], ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("B,H,N,d,causal", [(2, 4, 1000, 64, True), (1, 8, 2048, 128, False)])
-def test_noalloc_matches_workspace_backward_twice(B, H, N, d, causal):
+# fp32 inputs keep TF32-rounded copies of q, k, v and dO in the scratch as well
+# (most of its use); fp16 runs the 16-bit kernels with fp16 operands.
+CASES = [(2, 4, 1000, 64, True, "bf16"), (1, 8, 2048, 128, False, "bf16"),
+         (1, 4, 700, 128, True, "fp32"), (2, 2, 333, 80, False, "fp32"),
+         (1, 4, 1000, 64, True, "fp16")]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,dtype", CASES)
+def test_noalloc_matches_workspace_backward_twice(B, H, N, d, causal, dtype):
     import causal_attention_fa2_b200 as fa2
     from causal_attention_fa2_b200 import _native
     lib = _native.lib()
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     scale = 1.0 / math.sqrt(d)
-    inp = fa2_inputs.make_inputs(B, H, N, d, "bf16", seed=123 + N)
+    inp = fa2_inputs.make_inputs(B, H, N, d, dtype, seed=123 + N)
     q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
-    assert fa2.backward_workspace_bytes(B, H, N, d, torch.bfloat16) <= SCRATCH_BYTES
+    assert fa2.backward_workspace_bytes(B, H, N, d, q.dtype) <= SCRATCH_BYTES
     o, lse = fa2.forward(q, k, v, causal=causal, scale=scale)
-    ref = fa2.backward(q, k, v, o, lse, do, causal=causal, scale=scale)
-    atol, rtol = TOL["bf16"]
+    # fa2_backward_noalloc runs the two-pass form; compare with the same form.
+    ref = fa2.backward(q, k, v, o, lse, do, causal=causal, scale=scale, mode="two-pass")
+    atol, rtol = TOL[dtype]
     for _ in range(2):
         dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
-        st = _call_noalloc(lib, q, k, v, o, lse, do, dq, dk, dv, causal, scale)
+        st = _call_noalloc(lib, q, k, v, o, lse, do, dq, dk, dv, causal, scale, dtype)
         assert st == 0, _native.status_string(st)
         torch.cuda.synchronize()
         for got, want in zip((dq, dk, dv), ref):
