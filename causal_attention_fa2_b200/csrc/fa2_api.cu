@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -278,6 +279,9 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.kv_splits = ws.kv_splits;
     p.part = ws.kv_splits > 1 ? reinterpret_cast<float*>(ws_base + ws.part_off) : nullptr;
     p.item0 = 0;
+    // One-pass backward: heads in groups whose (key tile, head) items make about
+    // two waves of the SMs, so the CTAs resident together share L2.
+    p.head_group = std::max(1, std::min(p.BH_kv, (2 * 148 + p.n_tiles_k - 1) / p.n_tiles_k));
     if (one_pass) {
         // 2. dQ and D of the query tiles whose rows see a single key tile (causal:
         // query tile 0 of every head, the pass's last BH work items).
@@ -293,11 +297,11 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
         // 3. dK, dV and the other query tiles' dQ in one key-tile-outer pass, then
         // dQ = scale * dQ_acc rounded once.
         using FC = BwdFusedCfg<ES, D, F16>;
-        CUtensorMap macc;
-        if ((st = make_map_f32_reduce(&macc, dq_acc, D, ws.n_pad, BH, FC::kCW)) != FA2_OK) return st;
         auto kern = fa2_bwd_fused_kernel<ES, D, F16>;
         if ((st = set_smem(kern, FC::kSmemBytes)) != FA2_OK) return st;
         const unsigned grid_f = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
+        CUtensorMap macc;
+        if ((st = make_map_f32_reduce(&macc, dq_acc, D, ws.n_pad, BH, FC::kCW)) != FA2_OK) return st;
         kern<<<grid_f, FC::kThreads, FC::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, macc, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
         const long long groups8 = static_cast<long long>(BH) * N * D / 8;
@@ -406,6 +410,8 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     p.block_mask = nullptr;                              // block-sparse: 16-bit inputs only
     p.kv_splits = 1;                                     // fp32: one CTA per group
     p.part = nullptr;
+    p.item0 = 0;
+    p.head_group = 1;
     // dK/dV pass: one CTA per (key tile, key/value head); dQ pass: per (query tile, query head).
     const unsigned grid_kv = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
     const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);

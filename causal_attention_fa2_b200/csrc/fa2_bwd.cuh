@@ -192,6 +192,7 @@ struct BwdParams {
     int kv_splits;         // dK/dV pass CTAs per (key tile, key/value head)
     float* part;           // fp32 partial dK, dV when kv_splits > 1
     int item0;             // dQ pass: work item of the first CTA (a launch may cover a suffix)
+    int head_group;        // one-pass backward: key/value heads per group of work items
 };
 
 template <int ES, int D, bool F16 = false>

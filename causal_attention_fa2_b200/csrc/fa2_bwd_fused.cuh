@@ -62,7 +62,7 @@ struct BwdFusedCfg {
     static constexpr int kRing0 = (kBudget - 2 * kTile - kDsBytes) / (2 * kTile);
     static constexpr int kRing = kRing0 > 3 ? 3 : kRing0;
     static_assert(kRing >= 2, "shared memory too small for the streaming rings");
-    static constexpr int kSmemBytes = 1024 + 2 * kTile + 2 * kRing * kTile + kDsBytes;
+    static constexpr int kSmemBase = 1024 + 2 * kTile + 2 * kRing * kTile + kDsBytes;
     // Tensor memory.
     static constexpr uint32_t kTmemCols = 512;
     // d > 64 (d = 80, 128): S^T | dP^T (and dQ_i) | dV | dK at columns 0, 128,
@@ -73,25 +73,32 @@ struct BwdFusedCfg {
     static constexpr uint32_t kColDK = kDqInDp ? 384 : 256 + G::kNOut;
     static constexpr uint32_t kColDQ = kDqInDp ? kColDP : 256 + 2 * G::kNOut;
     static_assert(kColDK + G::kNOut <= 512 && kColDQ + G::kNOut <= 512, "tensor memory overflow");
-    // dQ drain: chunks of kCW fp32 columns, staged in halves of the dS tile.
+    // dQ drain: chunks of kCW fp32 columns, staged in halves of the dS tile (free
+    // once dK and dQ have read it).
     static constexpr int kCW = G::kNOut >= 32 ? 32 : G::kNOut;
     static constexpr int kNCh = (G::kNOut + kCW - 1) / kCW;
     static constexpr int kChunkBytes = kTileRows * kCW * 4;
-    static_assert(2 * kChunkBytes <= kDsBytes, "two staging chunks must fit in the dS tile");
+    static_assert(2 * kChunkBytes <= kDsBytes, "two drain chunks must fit in the dS tile");
+    // Where shared memory allows (d <= 64), dQ_i is staged in a buffer of its own
+    // that outlives the step, so the dS tile is free as soon as dK and dQ have
+    // read it; at d = 80 and 128 the staging shares the dS tile.
+    static constexpr bool kOwnStage = kSmemBase + kNCh * kChunkBytes <= kBudget + 1024;
+    static constexpr int kSmemBytes = kSmemBase + (kOwnStage ? kNCh * kChunkBytes : 0);
     // Register split (512 threads launch with 128 registers each): warpgroup 0
     // (producer, issuer) and the drain warpgroup give registers to the two
     // elementwise warpgroups.
     static constexpr int kLaunchRegs = 128;
-    static constexpr int kRegsLow = 112;
-    static constexpr int kRegsEw = 160;
-    static constexpr int kRegsDrain = 56;
+    static constexpr int kRegsLow = 88;
+    static constexpr int kRegsEw = 152;
+    static constexpr int kRegsDrain = 120;
     static_assert(128 * kRegsLow + 256 * kRegsEw + 128 * kRegsDrain <= kThreads * kLaunchRegs,
                   "register split exceeds the registers the block is launched with");
 };
 
 // Staging offset of 16-byte unit u (4 fp32 values) of row r in a chunk of kCW
 // fp32 columns, in the layout the TMA's 128-byte (kCW = 32) or 64-byte
-// (kCW = 16) swizzle expects.
+// (kCW = 16) swizzle expects (which also spreads a warp's row writes over all
+// banks).
 template <int kCW>
 __device__ __forceinline__ uint32_t stage_offset(int r, int u) {
     if constexpr (kCW == 32) return r * 128 + ((u ^ (r & 7)) << 4);
@@ -133,15 +140,21 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t* sQr = sV + TB;
     uint8_t* sDOr = sQr + RS * TB;
     uint8_t* sDS = sDOr + RS * TB;
+    uint8_t* sStage = Cfg::kOwnStage ? sDS + Cfg::kDsBytes : sDS;    // dQ staging
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: (key tile j, key/value head), key tile 0 (the most query tiles
-    // under the causal rule) first.
-    const int item = blockIdx.x;
-    const int kv_tile = item / p.BH_kv;
-    const int bh = item - kv_tile * p.BH_kv;            // key/value head
+    // Work item: (key tile j, key/value head).  Heads are taken in groups of
+    // p.head_group so that the CTAs resident together touch few heads' dQ
+    // accumulator, Q and dO (they stay in L2); inside a group key tile 0 (the
+    // most query tiles under the causal rule) comes first.
+    const int per_group = p.head_group * p.n_tiles_k;
+    const int hgroup = blockIdx.x / per_group;
+    const int in_group = blockIdx.x - hgroup * per_group;
+    const int heads_here = min(p.head_group, p.BH_kv - hgroup * p.head_group);
+    const int kv_tile = in_group / heads_here;
+    const int bh = hgroup * p.head_group + (in_group - kv_tile * heads_here);   // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
     const int kv_row0 = kv_tile * kTileRows;
     const int n_q = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;
@@ -292,6 +305,8 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     for (int kk = 0; kk < G::kStepsRows; ++kk)
                         ptx::mma_f16_ss(tmem + Cfg::kColDQ, desc_mnmajor<GS>(ds_addr, kk), desc_mnmajor<G>(k_addr, kk), idesc_dq, kk > 0 ? 1u : 0u);
                     ptx::mma_commit(&bar_dq_full);
+                    // With its own staging the drain leaves the dS tile alone.
+                    if (Cfg::kOwnStage) ptx::mma_commit(&bar_ds_free);
                     ++n_dq;
                     // dQ shares the dP^T columns: the next dP^T waits for the drain.
                     if (Cfg::kDqInDp && it + 1 < n_it &&
@@ -327,6 +342,13 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const size_t vb = static_cast<size_t>(q_head_of(it)) * p.n_pad + static_cast<size_t>(i) * kTileRows + qc0;
             const float4* l2v = reinterpret_cast<const float4*>(p.l2 + vb);
             const float4* dv4 = reinterpret_cast<const float4*>(p.dvec + vb);
+            if (it + 1 < n_it && lane < 8) {
+                // Bring the next step's L*log2(e) and D (512 bytes each) into L1 early.
+                const size_t nb = static_cast<size_t>(q_head_of(it + 1)) * p.n_pad +
+                                  static_cast<size_t>(q_tile_of(it + 1)) * kTileRows + 32 * (lane & 3);
+                const float* src = (lane < 4 ? p.l2 : p.dvec) + nb;
+                asm volatile("prefetch.global.L1 [%0];" ::"l"(src));
+            }
             // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14)
             if (!ptx::mbar_wait(&bar_s_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -377,15 +399,14 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // ---- dS^T = P^T o (dP^T - D)   (Eq. 17)
             if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            // The previous step's products and dQ drain must have released the dS tile.
-            if (it > 0 && !ptx::mbar_wait(&bar_ds_free, (it - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
-            // Two halves of 32 query columns: dS^T (16-bit) -> the shared-memory dS tile
-            // (row r, columns [64g + 32h, +32)); on single-tile steps the rounding
-            // remainders (lo parts) -> this group's dP^T columns (already read), the A
-            // operand of the issuer's second dK product.
+            // dS^T (16-bit) for this group's 64 query columns, in two halves of 32; on
+            // single-tile steps also the rounding remainders (lo parts), which go to
+            // this group's dP^T columns (already read), the A operand of the issuer's
+            // second dK product.
+            uint32_t dk[32];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                uint32_t ud[32], dk[16], dl[16];
+                uint32_t ud[32], dl[16];
                 ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32 * h, ud);
                 ptx::tmem_wait_ld();
 #pragma unroll
@@ -397,20 +418,24 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         float2 pp;
                         G::unpack2(pk[(32 * h + c + e) >> 1], pp.x, pp.y);
                         const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c + e]), __uint_as_float(ud[c + e + 1])), nd[e >> 1]));
-                        dk[(c + e) >> 1] = G::pack2(ds.x, ds.y);
+                        const int wd = (32 * h + c + e) >> 1;
+                        dk[wd] = G::pack2(ds.x, ds.y);
                         if (single) {
                             float2 hv;
-                            G::unpack2(dk[(c + e) >> 1], hv.x, hv.y);
+                            G::unpack2(dk[wd], hv.x, hv.y);
                             dl[(c + e) >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
                         }
                     }
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    *reinterpret_cast<uint4*>(sDS + kmajor_chunk_offset<GS>(r, qc0 + 32 * h + 8 * u)) =
-                        make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
                 if (single) ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 16 * h, dl);
             }
+            // -> the shared-memory dS tile (row r, query columns [64g, 64g + 64)), once
+            // the previous step's products and dQ drain have released it.
+            if (it > 0 && !ptx::mbar_wait(&bar_ds_free, (it - 1) & 1, &abort_flag, tmo)) { ok = false; break; }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(sDS + kmajor_chunk_offset<GS>(r, qc0 + 8 * u)) =
+                    make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
             ptx::fence_async_smem();
             if (single) ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -469,14 +494,37 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::setmaxnreg_dec<Cfg::kRegsDrain>();
         // ------------------------------------------------ dQ drain (warps 12-15)
         // Thread t owns query row t of the tile (TMEM lane t).  Per step with a
-        // dQ product: read each kCW-column chunk from TMEM, stage it in one half
-        // of the dS tile in the TMA swizzle, and reduce-add it into dQ_acc.  One
-        // thread issues (and waits on) the bulk copies; the others follow it
-        // through a named barrier, so every decision is the same in all four warps.
+        // dQ product, dQ_i leaves TMEM in kCW-column chunks of one row per thread:
+        // the first two chunks into the two halves of the dS tile (free once dK
+        // and dQ have read it), in the layout of the TMA's swizzle, the others
+        // into registers, so that TMEM is released after the loads alone.  One
+        // thread then adds the staged chunks to dQ_acc with TMA reduce-add
+        // (cp.reduce.async.bulk.tensor), waits until the copies have read them,
+        // and the register chunks follow through the same halves.  The copy
+        // engine performs the additions in L2, away from the SM's load/store
+        // queues, which the other roles keep using.  The dS tile is released
+        // once the last copy has read it.  That thread takes every wait; the
+        // others follow it through a named barrier.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const bool leader = threadIdx.x == 384;
+        constexpr int kU = Cfg::kCW / 4;                   // 16-byte units per chunk row
+        constexpr int kInSmem = Cfg::kOwnStage ? Cfg::kNCh : (Cfg::kNCh < 2 ? Cfg::kNCh : 2);
+        constexpr int kInRegs = Cfg::kNCh - kInSmem;       // 0, 1 (d = 80) or 2 (d = 128)
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
+        auto load_chunk = [&](int c, uint32_t (&u)[Cfg::kCW]) {
+            if constexpr (Cfg::kCW == 32)
+                ptx::tmem_ld32(lane_base + Cfg::kColDQ + c * Cfg::kCW, *reinterpret_cast<uint32_t(*)[32]>(u));
+            else
+                ptx::tmem_ld16(lane_base + Cfg::kColDQ + c * Cfg::kCW, *reinterpret_cast<uint32_t(*)[16]>(u));
+            ptx::tmem_wait_ld();
+        };
+        auto put_row = [&](uint8_t* st, const uint32_t (&u)[Cfg::kCW]) {   // this thread's row
+#pragma unroll
+            for (int q4 = 0; q4 < kU; ++q4)
+                *reinterpret_cast<uint4*>(st + stage_offset<Cfg::kCW>(r, q4)) =
+                    make_uint4(u[4 * q4], u[4 * q4 + 1], u[4 * q4 + 2], u[4 * q4 + 3]);
+        };
         int n_dq = 0;
         for (int it = 0; it < n_it; ++it) {
             if (single_of(it)) continue;
@@ -486,37 +534,48 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             ptx::tc_fence_after();
             const int q_row0 = q_tile_of(it) * kTileRows;
             const int qh = q_head_of(it);
-#pragma unroll
-            for (int c = 0; c < Cfg::kNCh; ++c) {
-                uint32_t u[Cfg::kCW];
-                if constexpr (Cfg::kCW == 32)
-                    ptx::tmem_ld32(lane_base + Cfg::kColDQ + c * Cfg::kCW, *reinterpret_cast<uint32_t(*)[32]>(u));
-                else
-                    ptx::tmem_ld16(lane_base + Cfg::kColDQ + c * Cfg::kCW, *reinterpret_cast<uint32_t(*)[16]>(u));
-                ptx::tmem_wait_ld();
-                if (c == Cfg::kNCh - 1) {
-                    // Every column of dQ_i has left TMEM: the issuer may reuse them.
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&bar_dq_drained);
-                }
-                // Half c % 2 of the staging area was last read by chunk c - 2's copy.
-                if (leader && c >= 2) ptx::tma_store_wait_read_1();
+            uint32_t keep[kInRegs > 0 ? kInRegs : 1][Cfg::kCW];
+            if (Cfg::kOwnStage) {
+                // The previous step's copies must have read the staging buffer.
+                if (leader) ptx::tma_store_wait_read_all();
                 asm volatile("bar.sync 4, 128;" ::: "memory");
-                uint8_t* st = sDS + (c & 1) * Cfg::kChunkBytes;
+            }
 #pragma unroll
-                for (int q4 = 0; q4 < Cfg::kCW / 4; ++q4)
-                    *reinterpret_cast<uint4*>(st + stage_offset<Cfg::kCW>(r, q4)) =
-                        make_uint4(u[4 * q4], u[4 * q4 + 1], u[4 * q4 + 2], u[4 * q4 + 3]);
+            for (int c = 0; c < kInSmem; ++c) {
+                uint32_t u[Cfg::kCW];
+                load_chunk(c, u);
+                put_row(sStage + c * Cfg::kChunkBytes, u);
+            }
+#pragma unroll
+            for (int c = 0; c < kInRegs; ++c) load_chunk(kInSmem + c, keep[c]);
+            // Every column of dQ_i has left TMEM: the issuer may reuse them.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bar_dq_drained);
+            ptx::fence_async_smem();
+            asm volatile("bar.sync 4, 128;" ::: "memory");
+            if (leader) {
+#pragma unroll
+                for (int c = 0; c < kInSmem; ++c)
+                    ptx::tma_reduce_add_3d(&tm_dqacc, sStage + c * Cfg::kChunkBytes, c * Cfg::kCW, q_row0, qh);
+                ptx::tma_store_commit();
+                if (kInRegs > 0) ptx::tma_store_wait_read_all();
+            }
+            if (kInRegs > 0) {
+                asm volatile("bar.sync 4, 128;" ::: "memory");    // the halves have been read
+#pragma unroll
+                for (int c = 0; c < kInRegs; ++c) put_row(sDS + c * Cfg::kChunkBytes, keep[c]);
                 ptx::fence_async_smem();
                 asm volatile("bar.sync 4, 128;" ::: "memory");
                 if (leader) {
-                    ptx::tma_reduce_add_3d(&tm_dqacc, st, c * Cfg::kCW, q_row0, qh);
+#pragma unroll
+                    for (int c = 0; c < kInRegs; ++c)
+                        ptx::tma_reduce_add_3d(&tm_dqacc, sDS + c * Cfg::kChunkBytes, (kInSmem + c) * Cfg::kCW, q_row0, qh);
                     ptx::tma_store_commit();
                 }
             }
-            if (leader) {
-                // The staging copies have read the dS tile: the groups may refill it.
+            if (leader && !Cfg::kOwnStage) {
+                // The copies have read the dS tile: the groups may refill it.
                 ptx::tma_store_wait_read_all();
                 ptx::mbar_arrive(&bar_ds_free);
             }

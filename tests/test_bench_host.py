@@ -53,3 +53,15 @@ def test_alg_bytes_10b_head_shape():
     fwd, bwd = bench.alg_bytes(w)
     assert fwd == 4 * t + rows == 151_584_768
     assert bwd == 8 * t + 3 * rows
+
+
+@pytest.mark.parametrize("N", [1, 100, 128, 129, 4096])
+@pytest.mark.parametrize("causal", [True, False])
+def test_single_tile_pairs(N, causal):
+    """Causal pairs of the rows whose query tile sees a single key tile (the
+    first 128 rows under the causal rule): counted by brute force."""
+    w = fa2_inputs.Workload("t", 2, 3, N, 64, "bf16", 0, causal)
+    q = np.arange(N)[:, None]
+    k = np.arange(N)[None, :]
+    brute = int(((k <= q) & (q < 128)).sum()) if causal else 0
+    assert bench.single_tile_pairs(w) == 2 * 3 * brute

@@ -82,17 +82,21 @@ def _check_against_oracle(oracle_mod, q, k, v, do, causal, dtype, label):
     if causal and Nk > N:
         # No query reaches keys N .. Nk-1: their gradients are exactly zero.
         assert not dk[:, :, N:].any() and not dv[:, :, N:].any()
-    # dK and dV add up `group` per-head gradients; the tolerance is the
-    # per-element one of a single gradient, scaled by the group size.
+    # dK and dV of a key/value head sum the gradients of the `group` query heads
+    # that share it.  Each head's part carries its own, independent rounding (P
+    # and dS are rounded to the input type per head), so the absolute error of
+    # the sum grows like sqrt(group): the bound is sqrt(group) * atol + rtol |ref|
+    # (the per-element bound itself for multi-head attention).
+    grp = H // H_kv
     for name, got in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
         err = np.abs(to64(got) - ref[name])
         tol = TOLS[dtype]
-        print(f"RATIO {label} {name} {float((err / (tol + tol * np.abs(ref[name]))).max()):.3f}")
-        if name in ("dk", "dv"):
-            grp = H // H_kv
-            assert (err <= grp * (tol + tol * np.abs(ref[name]) / grp)).all(), (name, err.max())
-        else:
-            assert_close(to64(got), ref[name], dtype, name)
+        widen = np.sqrt(grp) if name in ("dk", "dv") else 1.0
+        bound = widen * tol + tol * np.abs(ref[name])
+        print(f"RATIO {label} {name} {float((err / (tol + tol * np.abs(ref[name]))).max()):.3f} "
+              f"(of the widened bound {float((err / bound).max()):.3f})")
+        assert np.isfinite(to64(got)).all(), name
+        assert (err <= bound).all(), (name, float(err.max()), float((err / bound).max()))
     assert fa2.last_device_status() == 0
 
 
