@@ -11,6 +11,8 @@
 #include <cuda_bf16.h>
 
 #include <mutex>
+#include <utility>
+#include <vector>
 #include <type_traits>
 
 #include "../../include/fa2.h"
@@ -74,6 +76,27 @@ fa2_status init_device(int* dev_out, uint32_t** status_out) {
     return FA2_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel of the stream is still finishing (every kernel of
+// this library starts with griddepcontrol.launch_dependents and then waits,
+// with griddepcontrol.wait, for the previous kernel before touching global
+// memory), which hides the launch latency between the kernels of a pass.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 bool head_dim_supported(int d) { return d == 16 || d == 32 || d == 64 || d == 80 || d == 128; }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -90,6 +113,49 @@ fa2_status check_common(int B, int H, int N, int d, int causal, float scale, fa2
     return FA2_OK;
 }
 
+// Tensor maps are encoded on the host for every call; the last few are kept,
+// keyed by everything that enters the encoding, so a caller that passes the
+// same buffers again (a training loop) skips the driver call.
+struct MapKey {
+    const void* ptr;
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    int dtype, swizzle;
+    bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+constexpr int kMapCache = 64;
+std::mutex g_map_mutex;
+MapKey g_map_keys[kMapCache];
+CUtensorMap g_map_vals[kMapCache];
+int g_map_used = 0, g_map_next = 0;
+
+fa2_status encode_cached(CUtensorMap* m, CUtensorMapDataType type, const void* ptr, const cuuint64_t* dims,
+                         const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+    MapKey key;
+    std::memset(&key, 0, sizeof(key));
+    key.ptr = ptr;
+    for (int i = 0; i < 3; ++i) { key.dims[i] = dims[i]; key.box[i] = box[i]; }
+    for (int i = 0; i < 2; ++i) key.strides[i] = strides[i];
+    key.dtype = static_cast<int>(type);
+    key.swizzle = static_cast<int>(sw);
+    {
+        std::lock_guard<std::mutex> lock(g_map_mutex);
+        for (int i = 0; i < g_map_used; ++i)
+            if (g_map_keys[i] == key) { *m = g_map_vals[i]; return FA2_OK; }
+    }
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, type, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return FA2_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_map_mutex);
+    g_map_keys[g_map_next] = key;
+    g_map_vals[g_map_next] = *m;
+    g_map_next = (g_map_next + 1) % kMapCache;
+    if (g_map_used < kMapCache) ++g_map_used;
+    return FA2_OK;
+}
+
 // 3-D view [BH][N][d] of a contiguous [B,H,N,d] tensor, loaded/stored in boxes
 // of box_cols x 128 rows x 1 head.
 fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int N, int BH,
@@ -100,19 +166,15 @@ fa2_status make_map(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int d, int
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * es,
                              static_cast<cuuint64_t>(d) * es * static_cast<cuuint64_t>(N)};
     cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
     CUtensorMapSwizzle sw = mn_major_f32       ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
                             : row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                             : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
                                                : CU_TENSOR_MAP_SWIZZLE_32B;
-    CUresult r = g_encode(m,
-                          dtype == FA2_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                          : dtype == FA2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                          3, const_cast<void*>(ptr), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+    return encode_cached(m,
+                         dtype == FA2_BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                         : dtype == FA2_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                         ptr, dims, strides, box, sw);
 }
 
 // [BH][n_pad][d] fp32 accumulator, reduce-added in boxes of box_cols columns x
@@ -123,12 +185,8 @@ fa2_status make_map_f32_reduce(CUtensorMap* m, void* ptr, int d, int n_pad, int 
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
                              static_cast<cuuint64_t>(d) * 4 * static_cast<cuuint64_t>(n_pad)};
     cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(kTileRows), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapSwizzle sw = box_cols * 4 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? FA2_OK : FA2_ERR_CUDA;
+    return encode_cached(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, ptr, dims, strides, box, sw);
 }
 
 template <int ES, int D>
@@ -143,12 +201,22 @@ fa2_status make_maps_mnmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, i
     return make_map(m, ptr, dtype, D, N, BH, G::kBoxMN, G::kRowBMN, G::kF32);
 }
 
+// The dynamic shared memory limit of a kernel is raised once per device.
+std::mutex g_attr_mutex;
+std::vector<std::pair<const void*, int>> g_attr_done;
+
 template <class Kernel>
 fa2_status set_smem(Kernel k, int bytes) {
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-                   cudaSuccess
-               ? FA2_OK
-               : FA2_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA2_ERR_CUDA;
+    const void* fn = reinterpret_cast<const void*>(k);
+    std::lock_guard<std::mutex> lock(g_attr_mutex);
+    for (const auto& e : g_attr_done)
+        if (e.first == fn && e.second == dev) return FA2_OK;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return FA2_ERR_CUDA;
+    g_attr_done.emplace_back(fn, dev);
+    return FA2_OK;
 }
 
 // The two-query-tile forward serves 16-bit inputs.  fp32 (TF32) inputs use the
@@ -187,18 +255,19 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
     p.block_mask = block_mask;
+    p.head_group = heads_per_group(BH, (p.n_tiles + 1) / 2);
     if constexpr (use_two_tile_forward<ES, D>()) {
         // Two query tiles per CTA (softmax of one overlaps the MMAs of the other).
         using Cfg2 = Fwd2Cfg<ES, D, F16>;
         auto kern = block_mask ? fa2_fwd2_kernel<ES, D, F16, true> : fa2_fwd2_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
         const unsigned pairs = static_cast<unsigned>((p.n_tiles + 1) / 2);
-        kern<<<pairs * static_cast<unsigned>(BH), Cfg2::kThreads, Cfg2::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+        launch_pdl(kern, dim3(pairs * static_cast<unsigned>(BH)), dim3(Cfg2::kThreads), Cfg2::kSmemBytes, stream, mq, mk, mv, mo, p);
     } else {
         auto kern = fa2_fwd_kernel<ES, D>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mo, p);
+        launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, mq, mk, mv, mo, p);
     }
     return cudaGetLastError() == cudaSuccess ? FA2_OK : FA2_ERR_CUDA;
 }
@@ -245,7 +314,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     const long long rows = static_cast<long long>(BH) * ws.n_pad;
     if (!mark(0)) return FA2_ERR_CUDA;
     constexpr int kPreRows = BwdPreCfg<D>::kRowsPerBlock;
-    fa2_bwd_pre_kernel<D, F16><<<static_cast<unsigned>((rows + kPreRows - 1) / kPreRows), 256, 0, stream>>>(
+    launch_pdl(fa2_bwd_pre_kernel<D, F16>, dim3(static_cast<unsigned>((rows + kPreRows - 1) / kPreRows)), dim3(256), 0, stream, 
         static_cast<const T*>(o), static_cast<const T*>(dout), lse, l2, dvec, N, ws.n_pad, rows, dq_acc);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     CUtensorMap mq, mk, mv, mdo, mdk, mdv, mdq;
@@ -279,17 +348,18 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     p.kv_splits = ws.kv_splits;
     p.part = ws.kv_splits > 1 ? reinterpret_cast<float*>(ws_base + ws.part_off) : nullptr;
     p.item0 = 0;
-    // One-pass backward: heads in groups whose (key tile, head) items make about
-    // two waves of the SMs, so the CTAs resident together share L2.
-    p.head_group = std::max(1, std::min(p.BH_kv, (2 * 148 + p.n_tiles_k - 1) / p.n_tiles_k));
+    // Work items in groups of heads (grouped_item), set per launch below.
+    const int hg_q = heads_per_group(BH, p.n_tiles);                        // query-tile pass
+    const int hg_kv = heads_per_group(p.BH_kv * p.kv_splits, p.n_tiles_k);  // key-tile passes
     if (one_pass) {
         // 2. dQ and D of the query tiles whose rows see a single key tile (causal:
         // query tile 0 of every head, the pass's last BH work items).
         if (causal) {
             auto kern = fa2_bwd_dq_kernel<ES, D, F16, false>;
             if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
-            p.item0 = (p.n_tiles - 1) * BH;
-            kern<<<static_cast<unsigned>(BH), Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+            p.item0 = (p.n_tiles - 1) * BH;   // the last BH items of the plain order
+            p.head_group = BH;
+            launch_pdl(kern, dim3(static_cast<unsigned>(BH)), dim3(Cfg::kThreadsDq), Cfg::kDqSmemBytes, stream, mq, mk, mv, mdo, mdq, p);
             p.item0 = 0;
             if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
         }
@@ -298,14 +368,15 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
         // dQ = scale * dQ_acc rounded once.
         using FC = BwdFusedCfg<ES, D, F16>;
         auto kern = fa2_bwd_fused_kernel<ES, D, F16>;
+        p.head_group = hg_kv;
         if ((st = set_smem(kern, FC::kSmemBytes)) != FA2_OK) return st;
         const unsigned grid_f = static_cast<unsigned>(p.n_tiles_k) * static_cast<unsigned>(p.BH_kv);
         CUtensorMap macc;
         if ((st = make_map_f32_reduce(&macc, dq_acc, D, ws.n_pad, BH, FC::kCW)) != FA2_OK) return st;
-        kern<<<grid_f, FC::kThreads, FC::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, macc, p);
+        launch_pdl(kern, dim3(grid_f), dim3(FC::kThreads), FC::kSmemBytes, stream, mq, mk, mv, mdo, mdk, mdv, macc, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
         const long long groups8 = static_cast<long long>(BH) * N * D / 8;
-        fa2_bwd_dq_finalize_kernel<F16><<<static_cast<unsigned>((groups8 + 255) / 256), 256, 0, stream>>>(
+        launch_pdl(fa2_bwd_dq_finalize_kernel<F16>, dim3(static_cast<unsigned>((groups8 + 255) / 256)), dim3(256), 0, stream, 
             dq_acc, static_cast<uint16_t*>(dq), N, ws.n_pad, D, groups8, causal ? kTileRows : 0, scale);
         if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
         return FA2_OK;
@@ -321,18 +392,20 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     {
         auto kern = block_mask ? fa2_bwd_dq_kernel<ES, D, F16, true> : fa2_bwd_dq_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kDqSmemBytes)) != FA2_OK) return st;
-        kern<<<grid, Cfg::kThreadsDq, Cfg::kDqSmemBytes, stream>>>(mq, mk, mv, mdo, mdq, p);
+        p.head_group = hg_q;
+        launch_pdl(kern, dim3(grid), dim3(Cfg::kThreadsDq), Cfg::kDqSmemBytes, stream, mq, mk, mv, mdo, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     }
     // 3. dK, dV: key/value-tile-outer pass (+ the sum of a split group's partials).
     {
         auto kern = block_mask ? fa2_bwd_dkdv_kernel<ES, D, F16, true> : fa2_bwd_dkdv_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
-        kern<<<grid_kv, Cfg::kThreads, Cfg::kSmemBytes, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+        p.head_group = hg_kv;
+        launch_pdl(kern, dim3(grid_kv), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, mq, mk, mv, mdo, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
         if (p.kv_splits > 1) {
             const size_t groups4 = 2 * static_cast<size_t>(p.BH_kv) * Nk * D / 4;
-            fa2_bwd_kv_reduce_kernel<F16><<<static_cast<unsigned>((groups4 + 255) / 256), 256, 0, stream>>>(
+            launch_pdl(fa2_bwd_kv_reduce_kernel<F16>, dim3(static_cast<unsigned>((groups4 + 255) / 256)), dim3(256), 0, stream, 
                 p.part, static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), p.kv_splits, p.BH_kv, Nk,
                 p.n_tiles_k * kTileRows, D, scale);
             if (cudaGetLastError() != cudaSuccess) return FA2_ERR_CUDA;
@@ -368,13 +441,13 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     float* kr = reinterpret_cast<float*>(ws_base + ws.k_off);
     float* vr = reinterpret_cast<float*>(ws_base + ws.v_off);
     float* dor = reinterpret_cast<float*>(ws_base + ws.do_off);
-    fa2_bwd32_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(
+    launch_pdl(fa2_bwd32_pre_kernel<D>, dim3(static_cast<unsigned>((rows + 7) / 8)), dim3(256), 0, stream, 
         static_cast<const float*>(q), static_cast<const float*>(o), static_cast<const float*>(dout),
         lse, qr, dor, l2, dvec, N, ws.n_pad, rows);
     const size_t kv4 = static_cast<size_t>(B) * H_kv * Nk * D / 4;  // D is a multiple of 4
     const unsigned round_grid = static_cast<unsigned>((kv4 + 255) / 256 < 4096 ? (kv4 + 255) / 256 : 4096);
-    fa2_round_tf32_kernel<<<round_grid, 256, 0, stream>>>(static_cast<const float4*>(k), reinterpret_cast<float4*>(kr), kv4);
-    fa2_round_tf32_kernel<<<round_grid, 256, 0, stream>>>(static_cast<const float4*>(v), reinterpret_cast<float4*>(vr), kv4);
+    launch_pdl(fa2_round_tf32_kernel, dim3(round_grid), dim3(256), 0, stream, static_cast<const float4*>(k), reinterpret_cast<float4*>(kr), kv4);
+    launch_pdl(fa2_round_tf32_kernel, dim3(round_grid), dim3(256), 0, stream, static_cast<const float4*>(v), reinterpret_cast<float4*>(vr), kv4);
     if (cudaGetLastError() != cudaSuccess || !mark(1)) return FA2_ERR_CUDA;
     q = qr;
     k = kr;
@@ -425,7 +498,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             return st;
         auto kern = fa2_bwd32_dq_kernel<D>;
         if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
-        kern<<<grid, Cfg::kThreads, Cfg::kSmemQ, stream>>>(mq, mdo, mkk, mkmn, mvk, mdq, p);
+        launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemQ, stream, mq, mdo, mkk, mkmn, mvk, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     }
     {
@@ -438,7 +511,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             return st;
         auto kern = fa2_bwd32_dkdv_kernel<D>;
         if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
-        kern<<<grid_kv, Cfg::kThreads, Cfg::kSmemKV, stream>>>(mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
+        launch_pdl(kern, dim3(grid_kv), dim3(Cfg::kThreads), Cfg::kSmemKV, stream, mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
     }
     return FA2_OK;

@@ -135,6 +135,10 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ 
                    const float* __restrict__ lse, float* __restrict__ l2,
                    float* __restrict__ dvec, int N, int n_pad, long long rows_total,
                    float* __restrict__ dq_acc = nullptr) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using C = BwdPreCfg<D>;
     const int sub = threadIdx.x % C::kTPR;
     const long long row = static_cast<long long>(blockIdx.x) * C::kRowsPerBlock + threadIdx.x / C::kTPR;
@@ -192,7 +196,7 @@ struct BwdParams {
     int kv_splits;         // dK/dV pass CTAs per (key tile, key/value head)
     float* part;           // fp32 partial dK, dV when kv_splits > 1
     int item0;             // dQ pass: work item of the first CTA (a launch may cover a suffix)
-    int head_group;        // one-pass backward: key/value heads per group of work items
+    int head_group;        // heads (dK/dV pass: key/value heads x splits) per group of work items
 };
 
 template <int ES, int D, bool F16 = false>
@@ -244,6 +248,10 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                     const BwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = BwdCfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int RS = Cfg::kRing;
@@ -281,9 +289,8 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // tiles j..T-1 (causal) of each of the `group` query heads sharing this
     // key/value head, whose dK and dV sum over all of them; small j carries
     // the most work and is issued first.
-    const int item = blockIdx.x;
-    const int kv_tile = item / (p.BH_kv * p.kv_splits);
-    const int item_r = item - kv_tile * p.BH_kv * p.kv_splits;
+    int kv_tile, item_r;
+    grouped_item(blockIdx.x, p.n_tiles_k, p.BH_kv * p.kv_splits, p.head_group, kv_tile, item_r);
     const int split = item_r / p.BH_kv;                 // which share of the group's steps
     const int bh = item_r - split * p.BH_kv;            // key/value head
     const int i_begin = p.causal ? kv_tile : 0;
@@ -714,6 +721,10 @@ __global__ void __launch_bounds__(256)
 fa2_bwd_kv_reduce_kernel(const float* __restrict__ part, uint16_t* __restrict__ dk,
                          uint16_t* __restrict__ dv, int splits, int BH_kv, int Nk, int nk_pad, int d,
                          float scale) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     const size_t per = static_cast<size_t>(BH_kv) * Nk * d / 4;   // 4-column groups per tensor
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= 2 * per) return;
@@ -755,6 +766,10 @@ __global__ void __launch_bounds__(352, 1)
 fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = BwdCfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int RK = Cfg::kRingK;
@@ -785,9 +800,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Work item: causal query tile i sees key tiles 0..i; longest first.  A
     // launch may cover only the last items (item0 > 0: the single-tile query
     // tiles ahead of the one-pass backward).
-    const int item = blockIdx.x + p.item0;
-    const int rank = item / p.BH;
-    const int bh = item - rank * p.BH;
+    int rank, bh;
+    grouped_item(blockIdx.x + p.item0, p.n_tiles, p.BH, p.head_group, rank, bh);
     const int q_tile = p.causal ? (p.n_tiles - 1 - rank) : rank;
     // Key tiles this query tile sees (causal: key index <= query index).
     const int n_kv_lim = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;

@@ -88,6 +88,10 @@ fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ o,
                      const float* __restrict__ dout, const float* __restrict__ lse,
                      float* __restrict__ qr, float* __restrict__ dor, float* __restrict__ l2,
                      float* __restrict__ dvec, int N, int n_pad, long long rows_total) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows_total) return;
@@ -119,6 +123,10 @@ fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ o,
 // TF32-rounded copy of an fp32 tensor (k or v: [B * H_kv][N][d]), n4 float4s.
 __global__ void __launch_bounds__(256)
 fa2_round_tf32_kernel(const float4* __restrict__ in, float4* __restrict__ out, size_t n4) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
          i += static_cast<size_t>(gridDim.x) * blockDim.x) {
         float4 x = in[i];
@@ -227,6 +235,10 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                       const __grid_constant__ CUtensorMap tm_dok, const __grid_constant__ CUtensorMap tm_domn,
                       const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                       const BwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = Bwd32Cfg<D>;
     using G = typename Cfg::G;
     constexpr int W = Cfg::kWkv;
@@ -476,6 +488,10 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_kk, const __grid_constant__ CUtensorMap tm_kmn,
                     const __grid_constant__ CUtensorMap tm_vk, const __grid_constant__ CUtensorMap tm_dq,
                     const BwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = Bwd32Cfg<D>;
     using G = typename Cfg::G;
     constexpr int W = Cfg::kWq;

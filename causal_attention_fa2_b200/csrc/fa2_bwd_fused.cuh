@@ -117,6 +117,10 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                      const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = BwdFusedCfg<ES, D, F16>;
     using G = typename Cfg::G;
     using GS = typename Cfg::GS;
@@ -145,16 +149,12 @@ fa2_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: (key tile j, key/value head).  Heads are taken in groups of
-    // p.head_group so that the CTAs resident together touch few heads' dQ
-    // accumulator, Q and dO (they stay in L2); inside a group key tile 0 (the
-    // most query tiles under the causal rule) comes first.
-    const int per_group = p.head_group * p.n_tiles_k;
-    const int hgroup = blockIdx.x / per_group;
-    const int in_group = blockIdx.x - hgroup * per_group;
-    const int heads_here = min(p.head_group, p.BH_kv - hgroup * p.head_group);
-    const int kv_tile = in_group / heads_here;
-    const int bh = hgroup * p.head_group + (in_group - kv_tile * heads_here);   // key/value head
+    // Work item: (key tile j, key/value head), in groups of p.head_group heads
+    // (grouped_item: the CTAs resident together share those heads' Q, dO and dQ
+    // accumulator in L2); inside a group key tile 0, which the most query tiles
+    // see under the causal rule, comes first.
+    int kv_tile, bh;                                     // bh: key/value head
+    grouped_item(blockIdx.x, p.n_tiles_k, p.BH_kv, p.head_group, kv_tile, bh);
     const int i_begin = p.causal ? kv_tile : 0;
     const int kv_row0 = kv_tile * kTileRows;
     const int n_q = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;
@@ -601,6 +601,10 @@ template <bool F16>
 __global__ void __launch_bounds__(256)
 fa2_bwd_dq_finalize_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq, int N, int n_pad,
                            int d, long long groups8, int skip_rows, float scale) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= groups8) return;
     const long long e = i * 8;                            // element of dq, [BH][N][d]

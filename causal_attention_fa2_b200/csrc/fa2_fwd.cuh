@@ -60,6 +60,7 @@ struct FwdParams {
     float scale_log2;      // scale * log2(e)
     unsigned long long timeout_ns;
     const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
+    int head_group;        // two-tile forward: heads per group of work items (grouped_item)
 };
 
 template <int ES, int D>
@@ -102,6 +103,10 @@ __global__ void __launch_bounds__(FwdCfg<ES, D>::kThreads, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                const FwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = FwdCfg<ES, D>;
     using G = typename Cfg::G;
     constexpr int KST = Cfg::kKSt;

@@ -260,6 +260,10 @@ __global__ void __launch_bounds__(384, 1)
 fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const FwdParams p) {
+    // Programmatic dependent launch: the next kernel may be scheduled now; wait for
+    // the previous kernel of the stream before touching global memory.
+    ptx::pdl_launch_dependents();
+    ptx::pdl_wait();
     using Cfg = Fwd2Cfg<ES, D, F16>;
     using G = typename Cfg::G;
     constexpr int ST = Cfg::kStages;
@@ -288,9 +292,8 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // Work item: a pair of adjacent query tiles (2t, 2t+1) of one head;
     // causal pairs are issued longest first.
     const int n_pairs = (p.n_tiles + 1) >> 1;
-    const int item = blockIdx.x;
-    const int rank = item / p.BH;
-    const int bh = item - rank * p.BH;
+    int rank, bh;
+    grouped_item(blockIdx.x, n_pairs, p.BH, p.head_group, rank, bh);
     const int pair = p.causal ? (n_pairs - 1 - rank) : rank;
     const int tile[2] = {2 * pair, 2 * pair + 1};
     const bool has_b = tile[1] < p.n_tiles;

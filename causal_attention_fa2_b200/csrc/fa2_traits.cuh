@@ -35,6 +35,29 @@ __host__ __device__ inline int kv_head_of(int bh, int H, int H_kv, int group) {
     return (bh / H) * H_kv + (bh % H) / group;
 }
 
+// Work items of a (rank, head) grid in groups of `hg` heads: the items of a
+// group cover its heads at every rank, rank-major inside the group, so the CTAs
+// resident together read the K/V (or Q/dO) of few heads, which stay in L2;
+// inside a group the lowest rank (the longest item under the causal rule, as
+// the callers number ranks) comes first.  hg >= n_heads is the plain rank-major
+// order.
+__host__ __device__ inline void grouped_item(int item, int n_rank, int n_heads, int hg, int& rank, int& head) {
+    const int per_group = hg * n_rank;
+    const int g = item / per_group;
+    const int in_group = item - g * per_group;
+    const int heads_here = (n_heads - g * hg) < hg ? (n_heads - g * hg) : hg;
+    rank = in_group / heads_here;
+    head = g * hg + (in_group - rank * heads_here);
+}
+
+// Heads per group for grouped_item: groups of about 600 items (four waves of
+// 148 SMs), the heads split evenly over the groups.
+inline int heads_per_group(int n_heads, int n_rank) {
+    const long long items = static_cast<long long>(n_heads) * n_rank;
+    const int groups = static_cast<int>((items + 599) / 600);
+    return groups <= 1 ? n_heads : (n_heads + groups - 1) / groups;
+}
+
 // Block-sparse attention ("Notes on flashattention", section "Block-sparse
 // Flashattention"): a byte per (query tile, key tile) pair of kTileRows x
 // kTileRows blocks, row-major with one row per query tile; zero blocks are
