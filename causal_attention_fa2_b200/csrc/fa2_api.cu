@@ -33,6 +33,7 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait
 // FA2_BWD_ONE_PASS does).
 constexpr bool kOnePassDefault = false;
 constexpr int kMaxDevices = 64;
+constexpr int kSmCount = 148;   // streaming multiprocessors of a B200
 constexpr int kMaxN = 1 << 24;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -255,14 +256,17 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
     p.block_mask = block_mask;
-    p.head_group = heads_per_group(BH, (p.n_tiles + 1) / 2);
+    // Two query tiles per CTA (the softmax of one overlaps the MMAs of the
+    // other), unless the pairs would leave SMs idle: then one tile per CTA.
+    const long long pair_items = static_cast<long long>((p.n_tiles + 1) / 2) * BH;
+    p.one_tile = pair_items < kSmCount ? 1 : 0;
+    const int n_items = p.one_tile ? p.n_tiles : (p.n_tiles + 1) / 2;
+    p.head_group = heads_per_group(BH, n_items);
     if constexpr (use_two_tile_forward<ES, D>()) {
-        // Two query tiles per CTA (softmax of one overlaps the MMAs of the other).
         using Cfg2 = Fwd2Cfg<ES, D, F16>;
         auto kern = block_mask ? fa2_fwd2_kernel<ES, D, F16, true> : fa2_fwd2_kernel<ES, D, F16, false>;
         if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
-        const unsigned pairs = static_cast<unsigned>((p.n_tiles + 1) / 2);
-        launch_pdl(kern, dim3(pairs * static_cast<unsigned>(BH)), dim3(Cfg2::kThreads), Cfg2::kSmemBytes, stream, mq, mk, mv, mo, p);
+        launch_pdl(kern, dim3(static_cast<unsigned>(n_items) * static_cast<unsigned>(BH)), dim3(Cfg2::kThreads), Cfg2::kSmemBytes, stream, mq, mk, mv, mo, p);
     } else {
         auto kern = fa2_fwd_kernel<ES, D>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;

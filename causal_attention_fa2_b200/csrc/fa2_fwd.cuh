@@ -61,6 +61,7 @@ struct FwdParams {
     unsigned long long timeout_ns;
     const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
     int head_group;        // two-tile forward: heads per group of work items (grouped_item)
+    int one_tile;          // two-tile forward: one query tile per CTA (small grids)
 };
 
 template <int ES, int D>

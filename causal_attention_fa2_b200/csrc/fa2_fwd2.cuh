@@ -289,13 +289,14 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Work item: a pair of adjacent query tiles (2t, 2t+1) of one head;
-    // causal pairs are issued longest first.
-    const int n_pairs = (p.n_tiles + 1) >> 1;
+    // Work item: a pair of adjacent query tiles (2t, 2t+1) of one head, or (when
+    // pairs would leave SMs idle, p.one_tile) a single query tile t with no
+    // tile B; causal items are issued longest first.
+    const int n_items = p.one_tile ? p.n_tiles : (p.n_tiles + 1) >> 1;
     int rank, bh;
-    grouped_item(blockIdx.x, n_pairs, p.BH, p.head_group, rank, bh);
-    const int pair = p.causal ? (n_pairs - 1 - rank) : rank;
-    const int tile[2] = {2 * pair, 2 * pair + 1};
+    grouped_item(blockIdx.x, n_items, p.BH, p.head_group, rank, bh);
+    const int pair = p.causal ? (n_items - 1 - rank) : rank;
+    const int tile[2] = {p.one_tile ? pair : 2 * pair, p.one_tile ? p.n_tiles : 2 * pair + 1};
     const bool has_b = tile[1] < p.n_tiles;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
     constexpr bool sparse = SPARSE;
