@@ -203,17 +203,9 @@ template <int ES, int D, bool F16 = false>
 struct BwdCfg {
     using G = TileGeom<ES, D, F16>;
     static_assert(ES == 2, "the backward kernels are written for 16-bit inputs");
-    // Warp 0 TMA producer, warp 1 MMA issuer, then the elementwise groups of
-    // four warps (dK/dV pass: kGroupsKV of them, each owning 128 / kGroupsKV
-    // score columns; dQ pass: two); the dQ pass adds a second MMA issuer.
-    // Four groups (a thread's share of P^T and dP^T halved) measured 2-4 %
-    // slower on the whole dK/dV pass than two at d = 80 and 128, so two it is.
-    static constexpr int kGroupsKV = 2;
-    static constexpr int kColsKV = 128 / kGroupsKV;
-    static constexpr int kThreads = 64 + 128 * kGroupsKV;
-    // Registers are granted per SM sub-partition: with 18 warps five share one,
-    // so a four-group block is compiled as if it had 20 warps (96 registers).
-    static constexpr int kLaunchKV = kGroupsKV == 4 ? 640 : kThreads;
+    // Warp 0 TMA producer, warp 1 MMA issuer, warps 2-9 the two elementwise
+    // groups; the dQ pass adds warp 10 as a second MMA issuer.
+    static constexpr int kThreads = 320;
     static constexpr int kThreadsDq = 352;
     static constexpr int kTile = G::kTileBytesK;
     // 227 KB minus the alignment pad and the static shared memory.
@@ -237,13 +229,11 @@ struct BwdCfg {
 };
 
 // TMEM column, relative to the score (or dP) block, of k-step kk of the
-// 16-bit P (or dS) A operand when the elementwise groups own `cols` columns
-// each.  The group that owns columns [cols g, cols g + cols) writes its values,
-// packed two per column, to the first cols / 2 of them, so the k-steps of its
-// columns read there and no group waits for another.
-template <int cols = 64>
+// 16-bit P (or dS) A operand.  The group that owns columns [64g, 64g + 64)
+// writes its 64 values, packed two per column, to the first 32 of them, so
+// k-steps 4g .. 4g+3 read there and neither group waits for the other.
 __host__ __device__ constexpr uint32_t a_col(int kk) {
-    return static_cast<uint32_t>((kk / (cols / 16)) * cols + (kk % (cols / 16)) * 8);
+    return static_cast<uint32_t>((kk / 4) * 64 + (kk % 4) * 8);
 }
 
 // ------------------------------------------------------------------ dK / dV pass
@@ -253,7 +243,7 @@ __host__ __device__ constexpr uint32_t a_col(int kk) {
 //   dK += dS^T(i) Q(i)      (A = dS^T from TMEM)    ; dP^T(i+1) = V dO(i+1)^T
 // while the groups compute P^T(i+1) and dS^T(i+1).
 template <int ES, int D, bool F16 = false, bool SPARSE = false>
-__global__ void __launch_bounds__(BwdCfg<ES, D, F16>::kLaunchKV, 1)
+__global__ void __launch_bounds__(320, 1)
 fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
@@ -266,8 +256,6 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     using G = typename Cfg::G;
     constexpr int RS = Cfg::kRing;
     constexpr int TB = Cfg::kTile;
-    constexpr int NW = 4 * Cfg::kGroupsKV;               // elementwise warps
-    constexpr int QC = Cfg::kColsKV;                     // query columns a group owns
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full;
@@ -277,9 +265,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     // Per-warp copies of the current query tile's L*log2(e) and D values for
-    // the warp's QC query columns (double-buffered; each warp syncs itself).
-    __shared__ __align__(16) float sL2[NW][2][QC];
-    __shared__ __align__(16) float sDv[NW][2][QC];
+    // the warp's 64 query columns (double-buffered; each warp syncs itself).
+    __shared__ __align__(16) float sL2[8][2][64];
+    __shared__ __align__(16) float sDv[8][2][64];
     // Block-sparse: the query tiles whose block with this key tile is set.
     __shared__ uint16_t s_q[SPARSE ? kMaxMaskTiles : 1];
     __shared__ int s_nq;
@@ -332,8 +320,8 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         ptx::mbar_init(&bar_s_full, 1);
         ptx::mbar_init(&bar_dp_full, 1);
-        ptx::mbar_init(&bar_p_ready, NW);
-        ptx::mbar_init(&bar_ds_ready, NW);
+        ptx::mbar_init(&bar_p_ready, 8);
+        ptx::mbar_init(&bar_ds_ready, 8);
         ptx::mbar_init(&bar_dkv_full, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::fence_mbar_init();
@@ -453,7 +441,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t da = do_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + a_col<QC>(kk), desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_f16_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + a_col(kk), desc_mnmajor<G>(da, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_do_empty[it % RS]);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
@@ -462,12 +450,12 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t qa = q_addr(it);
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsRows; ++kk)
-                    ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col<QC>(kk), desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(qa, kk), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 if (hilo_of(q_tile_of(it))) {
-                    // dK_j += dS^T_lo Q_i: the low parts sit QC / 2 columns after the high parts.
+                    // dK_j += dS^T_lo Q_i: the low parts sit 32 columns after the high parts.
 #pragma unroll
                     for (int kk = 0; kk < G::kStepsRows; ++kk)
-                        ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col<QC>(kk) + QC / 2, desc_mnmajor<G>(qa, kk), idesc_kv, 1u);
+                        ptx::mma_f16_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + a_col(kk) + 32, desc_mnmajor<G>(qa, kk), idesc_kv, 1u);
                 }
                 ptx::mma_commit(&bar_q_empty[it % RS]);
                 if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
@@ -480,29 +468,23 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
     } else {
-        // ------------------------------------------------ elementwise groups
-        // Group g (warps 2 + 4g .. 5 + 4g) owns query columns [QC g, QC g + QC)
-        // of the score tile; thread t of a group owns key row t (TMEM lane t).
-        // A row's QC values are handled in chunks of 32 columns.
-        constexpr int kCh = QC / 32;                      // 32-column chunks per row
+        // ------------------------------------------------ two P / dS groups
+        const int g = (warp - 2) >> 2;                  // query columns [64g, 64g+64)
         const int wi = warp - 2;
-        const int g = wi >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // key row inside the tile
-        const int qc0 = QC * g;
+        const int qc0 = 64 * g;
         const bool key_valid = kv_row0 + r < p.Nk;
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
-        // Offset of step it's L / D values for this group's query columns.
+        // Offset of step it's L / D values for this group's 64 query columns.
         auto vec_base = [&](int it) {
             return static_cast<size_t>(q_head_of(it)) * p.n_pad + static_cast<size_t>(q_tile_of(it)) * kTileRows + qc0;
         };
-        float nl2[kCh], nd[kCh];
-#pragma unroll
-        for (int m = 0; m < kCh; ++m) { nl2[m] = 0.f; nd[m] = 0.f; }
+        float nl2[2] = {0.f, 0.f}, nd[2] = {0.f, 0.f};
         if (n_it > 0) {
 #pragma unroll
-            for (int m = 0; m < kCh; ++m) {
+            for (int m = 0; m < 2; ++m) {
                 nl2[m] = p.l2[vec_base(0) + lane + 32 * m];
                 nd[m] = p.dvec[vec_base(0) + lane + 32 * m];
             }
@@ -512,7 +494,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const int i = q_tile_of(it);
             const int b = it & 1;
 #pragma unroll
-            for (int m = 0; m < kCh; ++m) {
+            for (int m = 0; m < 2; ++m) {
                 sL2[wi][b][lane + 32 * m] = nl2[m];
                 sDv[wi][b][lane + 32 * m] = nd[m];
             }
@@ -520,7 +502,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (it + 1 < n_it) {
                 const size_t nb = vec_base(it + 1);
 #pragma unroll
-                for (int m = 0; m < kCh; ++m) {
+                for (int m = 0; m < 2; ++m) {
                     nl2[m] = p.l2[nb + lane + 32 * m];
                     nd[m] = p.dvec[nb + lane + 32 * m];
                 }
@@ -529,17 +511,16 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14)
             if (!ptx::mbar_wait(&bar_s_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            uint32_t pk[QC / 2];                           // this group's P^T row, 16-bit pairs
+            uint32_t pk[32];                               // this group's P^T row, bf16 pairs
             {
-                uint32_t us[QC];
-#pragma unroll
-                for (int h = 0; h < kCh; ++h)
-                    ptx::tmem_ld32(lane_base + Cfg::kColS + qc0 + 32 * h, *reinterpret_cast<uint32_t(*)[32]>(us + 32 * h));
+                uint32_t us[64];
+                ptx::tmem_ld32(lane_base + Cfg::kColS + qc0, *reinterpret_cast<uint32_t(*)[32]>(us));
+                ptx::tmem_ld32(lane_base + Cfg::kColS + qc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(us + 32));
                 ptx::tmem_wait_ld();
                 const float2 sl2v = make_float2(sl2, sl2);
                 if (diag || !key_valid) {
 #pragma unroll
-                    for (int c = 0; c < QC; c += 4) {
+                    for (int c = 0; c < 64; c += 4) {
                         const float4 lv = *reinterpret_cast<const float4*>(&sL2[wi][b][c]);
                         const float2 a0 = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, make_float2(-lv.x, -lv.y));
                         const float2 a1 = ptx::fma2(make_float2(__uint_as_float(us[c + 2]), __uint_as_float(us[c + 3])), sl2v, make_float2(-lv.z, -lv.w));
@@ -552,7 +533,7 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 } else {
 #pragma unroll
-                    for (int c = 0; c < QC; c += 4) {
+                    for (int c = 0; c < 64; c += 4) {
                         const float4 lv = *reinterpret_cast<const float4*>(&sL2[wi][b][c]);
                         const float2 a0 = ptx::fma2(make_float2(__uint_as_float(us[c]), __uint_as_float(us[c + 1])), sl2v, make_float2(-lv.x, -lv.y));
                         const float2 a1 = ptx::fma2(make_float2(__uint_as_float(us[c + 2]), __uint_as_float(us[c + 3])), sl2v, make_float2(-lv.z, -lv.w));
@@ -561,11 +542,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             }
-            // P^T -> this group's own score columns [qc0, qc0 + QC / 2) (already read,
-            // so no wait on another group), A operand of dV += P^T dO.
-#pragma unroll
-            for (int h = 0; h < kCh; ++h)
-                ptx::tmem_st16(lane_base + Cfg::kColS + qc0 + 16 * h, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16 * h));
+            // P^T -> this group's own score columns [64g, 64g + 32) (already read,
+            // so no wait on the other group), A operand of dV += P^T dO.
+            ptx::tmem_st32(lane_base + Cfg::kColS + qc0, pk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
@@ -576,49 +555,71 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (ok) ptx::mbar_arrive(&bar_p_ready);
             }
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
-            // ---- dS^T = P^T o (dP^T - D)   (Eq. 17), chunk by chunk of 32 columns:
-            // the packed result of chunk h goes to the group's dP^T columns
-            // [qc0 + 16h, + 16), which held values already read.  On single-tile
-            // steps (hilo_of) dS^T goes to the dK MMA as hi + lo 16-bit parts, the lo
-            // parts at [qc0 + QC / 2 + 16h, + 16): stored once chunk h's columns there
-            // have been read (QC = 64: the first chunk's lo waits for the second load).
+            // ---- dS^T = P^T o (dP^T - D)   (Eq. 17)
             if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            const bool hilo = hilo_of(i);
-            uint32_t lo_keep[16];
+            if (hilo_of(i)) {
+                // dS^T = hi + lo, both rounded to the 16-bit type: hi into the group's
+                // first 32 dP^T columns, lo into the next 32 (the issuer's second dK
+                // group reads them).  Columns are overwritten only after they are read.
+                uint32_t lo_a[16];
+                {
+                    uint32_t ud[32], hi[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0, ud);
+                    ptx::tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kCh; ++h) {
-                uint32_t ud[32], hi[16], lo[16];
-                ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32 * h, ud);
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[c >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])),
+                                                                  make_float2(-sDv[wi][b][c], -sDv[wi][b][c + 1])));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo_a[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0, hi);          // hi, values 0..31
+                }
+                {
+                    uint32_t ud[32], hi[16], lo[16];
+                    ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32, ud);
+                    ptx::tmem_wait_ld();
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 32, lo_a);     // lo, values 0..31
+#pragma unroll
+                    for (int c = 0; c < 32; c += 2) {
+                        float2 pp, hv;
+                        G::unpack2(pk[(32 + c) >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c]), __uint_as_float(ud[c + 1])),
+                                                                  make_float2(-sDv[wi][b][32 + c], -sDv[wi][b][33 + c])));
+                        hi[c >> 1] = G::pack2(ds.x, ds.y);
+                        G::unpack2(hi[c >> 1], hv.x, hv.y);
+                        lo[c >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
+                    }
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 16, hi);     // hi, values 32..63
+                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 48, lo);     // lo, values 32..63
+                }
+            } else {
+            uint32_t dk[32];                               // this group's dS^T row, bf16 pairs
+            {
+                uint32_t ud[64];
+                ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0, *reinterpret_cast<uint32_t(*)[32]>(ud));
+                ptx::tmem_ld32(lane_base + Cfg::kColDP + qc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ud + 32));
                 ptx::tmem_wait_ld();
-                if (hilo && kCh == 2 && h == 1)
-                    ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + QC / 2, lo_keep);   // lo, chunk 0
 #pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 dv4 = *reinterpret_cast<const float4*>(&sDv[wi][b][32 * h + c]);
-                    const float2 nd2[2] = {make_float2(-dv4.x, -dv4.y), make_float2(-dv4.z, -dv4.w)};
+                for (int c = 0; c < 64; c += 4) {
+                    const float4 dv4 = *reinterpret_cast<const float4*>(&sDv[wi][b][c]);
+                    const float2 nd[2] = {make_float2(-dv4.x, -dv4.y), make_float2(-dv4.z, -dv4.w)};
 #pragma unroll
-                    for (int e = 0; e < 4; e += 2) {
+                    for (int h = 0; h < 4; h += 2) {
                         float2 pp;
-                        G::unpack2(pk[(32 * h + c + e) >> 1], pp.x, pp.y);
-                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c + e]), __uint_as_float(ud[c + e + 1])), nd2[e >> 1]));
-                        hi[(c + e) >> 1] = G::pack2(ds.x, ds.y);
-                        if (hilo) {
-                            float2 hv;
-                            G::unpack2(hi[(c + e) >> 1], hv.x, hv.y);
-                            lo[(c + e) >> 1] = G::pack2(ds.x - hv.x, ds.y - hv.y);
-                        }
+                        G::unpack2(pk[(c + h) >> 1], pp.x, pp.y);
+                        const float2 ds = ptx::mul2(pp, ptx::add2(make_float2(__uint_as_float(ud[c + h]), __uint_as_float(ud[c + h + 1])), nd[h >> 1]));
+                        dk[(c + h) >> 1] = G::pack2(ds.x, ds.y);
                     }
                 }
-                ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + 16 * h, hi);
-                if (hilo) {
-                    if (kCh == 2 && h == 0) {
-#pragma unroll
-                        for (int w = 0; w < 16; ++w) lo_keep[w] = lo[w];
-                    } else {
-                        ptx::tmem_st16(lane_base + Cfg::kColDP + qc0 + QC / 2 + 16 * h, lo);
-                    }
-                }
+            }
+            // dS^T -> this group's own dP^T columns [128 + 64g, ... + 32), A operand
+            // of dK += dS^T Q.
+            ptx::tmem_st32(lane_base + Cfg::kColDP + qc0, dk);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -632,10 +633,9 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) { ok = false; break; }
         }
         // ---------------- epilogue: dV (group 0) / dK (group 1) -> shared memory -> TMA store
-        // (zeros when no query reaches this key tile); other groups are done.
+        // (zeros when no query reaches this key tile).
         if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
-        if (g >= 2) {
-        } else if (p.kv_splits > 1) {
+        if (p.kv_splits > 1) {
             // Split group: this CTA's fp32 partial sums, one key row per thread, to
             // part[dK = 0 / dV = 1][split][head][row][d]; the reduction pass scales
             // dK, sums the splits in order and rounds.
