@@ -45,8 +45,10 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each
 # bf16 d=128 kernel on the 10B head shape, from one ncu capture of the current
 # kernel build; None where no capture of the current build exists.
-FWD_TRAFFIC_BYTES = 208_496_896   # 185.7 MB read + 22.8 MB written (12-warp forward)
-FUSED_TRAFFIC_BYTES = None        # no capture of the one-pass backward yet
+FWD_TRAFFIC_BYTES = 209_842_944   # 186.0 MB read + 23.8 MB written
+DKDV_TRAFFIC_BYTES = 204_046_336  # 153.5 MB read + 50.5 MB written (two-pass dK/dV pass)
+DQ_TRAFFIC_BYTES = 178_731_264    # 154.2 MB read + 24.6 MB written (two-pass dQ pass)
+FUSED_TRAFFIC_BYTES = None        # no capture of the one-pass backward's current build
 TRAFFIC_WORKLOAD = "10b-b1h36-n4096-d128"
 
 
@@ -607,7 +609,8 @@ def main():
         elif w.dtype != "fp32":
             names = (f"fa2_fwd2_kernel<{w.dtype},d={w.d}>", f"fa2_bwd_dkdv_kernel<{w.dtype},d={w.d}>",
                      f"fa2_bwd_dq_kernel<{w.dtype},d={w.d}>")
-            traffic = (None, None, None)
+            traffic = ((FWD_TRAFFIC_BYTES, DKDV_TRAFFIC_BYTES, DQ_TRAFFIC_BYTES)
+                       if w.name == TRAFFIC_WORKLOAD else (None, None, None))
             flops_k = (8 * pc4, 2 * pc4)
         else:
             names = (f"fa2_fwd_kernel<fp32,d={w.d}>", f"fa2_bwd32_dkdv_kernel<d={w.d}>",
