@@ -224,8 +224,11 @@ struct BwdCfg {
     static_assert(kRingK >= 2 && kRingV >= 2, "shared memory too small for the dQ rings");
     static constexpr int kDqSmemBytes = 1024 + (2 + kRingK + kRingV) * kTile;
     static constexpr uint32_t kTmemCols = 512;
-    // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
+    // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP (even key tiles) | dQ |
+    // dP (odd key tiles); dQ takes at most 128 columns.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
+    static constexpr uint32_t kColDP1 = 384;
+    static_assert(G::kNOut <= 128, "dQ must fit between the two dP buffers");
 };
 
 // TMEM column, relative to the score (or dP) block, of k-step kk of the
@@ -756,11 +759,12 @@ fa2_bwd_kv_reduce_kernel(const float* __restrict__ part, uint16_t* __restrict__ 
 
 // One CTA per (query tile i, head).  Per key tile j the tensor core runs
 //   S(j) = Q K_j^T ; dP(j) = dO V_j^T ; dQ += dS(j) K_j   (A = dS from TMEM)
-// from two issuing threads: S(j+1) as soon as both groups have read S(j),
-// and dP(j+1) right after dQ(j), so the groups' exponentials overlap the
-// tensor core.  A thread that waits on an mbarrier after committing MMAs
-// stalls until those MMAs are done; with two issuers the other one's MMAs
-// keep the tensor core busy meanwhile.
+// from two issuing threads: S(j+1) as soon as both groups have read S(j), and
+// dP into two TMEM buffers, dP(j+2) right after dQ(j) (which reads dS(j) from
+// the same buffer), so dP(j+1) is ready when the groups finish P(j+1).  A
+// thread that waits on an mbarrier after committing MMAs stalls until those
+// MMAs are done; with two issuers the other one's MMAs keep the tensor core
+// busy meanwhile.
 template <int ES, int D, bool F16 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(352, 1)
 fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -779,7 +783,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_qdo_full;
     __shared__ uint64_t bar_k_full[RK], bar_k_empty[RK], bar_v_full[RV], bar_v_empty[RV];
-    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready;
+    __shared__ uint64_t bar_s_full, bar_dp_full[2], bar_s_read, bar_ds_ready;
     __shared__ uint64_t bar_dq_done, bar_drain[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
@@ -827,7 +831,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             ptx::mbar_init(&bar_v_empty[s], 1);
         }
         ptx::mbar_init(&bar_s_full, 1);
-        ptx::mbar_init(&bar_dp_full, 1);
+        ptx::mbar_init(&bar_dp_full[0], 1);
+        ptx::mbar_init(&bar_dp_full[1], 1);
         ptx::mbar_init(&bar_s_read, 8);
         ptx::mbar_init(&bar_ds_ready, 8);
         ptx::mbar_init(&bar_dq_done, 1);
@@ -853,6 +858,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // see is in that tile, so those rows take D from the tile's own P and dP and
     // their dS goes to the dQ MMA as two 16-bit parts (see the groups below).
     const bool single = n_kv == 1;
+    // TMEM columns of key tile j's dP (and, written over it, dS) buffer.
+    auto dp_col = [](int j) { return (j & 1) ? Cfg::kColDP1 : Cfg::kColDP; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -892,11 +899,11 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     } else if (warp == 1 || warp == 10) {
         // ------------------------------------------------ MMA issuers
         // Issuer 0 (warp 1): S(j) for every key tile, each as soon as both
-        // groups have read S(j-1).  Issuer 1 (warp 10): dP(0); per key tile j
-        // dQ += dS(j) K_j, then dP(j+1) (it overwrites dS(j)).  A wait stalls
-        // only the thread whose MMAs precede it, so one issuer's MMAs keep the
-        // tensor core busy while the other waits.  K_j's slot is released by
-        // both S(j) and dQ(j); V_j's by dP(j).
+        // groups have read S(j-1).  Issuer 1 (warp 10): dP(0), dP(1); per key
+        // tile j dQ += dS(j) K_j, then dP(j+2) (it overwrites dS(j)).  A wait
+        // stalls only the thread whose MMAs precede it, so one issuer's MMAs
+        // keep the tensor core busy while the other waits.  K_j's slot is
+        // released by both S(j) and dQ(j); V_j's by dP(j).
         const int role = warp == 1 ? 0 : 1;
         if (lane == 0 && (!SPARSE || n_kv > 0)) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, 128, false, false);
@@ -927,12 +934,13 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t va = v_addr(j);
 #pragma unroll
                     for (int kk = 0; kk < G::kStepsD; ++kk)
-                        ptx::mma_f16_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk), idesc_s, kk > 0 ? 1u : 0u);
-                    ptx::mma_commit(&bar_dp_full);
+                        ptx::mma_f16_ss(tmem + dp_col(j), desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk), idesc_s, kk > 0 ? 1u : 0u);
+                    ptx::mma_commit(&bar_dp_full[j & 1]);
                     ptx::mma_commit(&bar_v_empty[j % RV]);
                     return true;
                 };
                 if (ok) ok = issue_dp(0);
+                if (ok && n_kv > 1) ok = issue_dp(1);
                 for (int j = 0; ok && j < n_kv; ++j) {
                     // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
                     if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo) || !wait_k(j)) { ok = false; break; }
@@ -940,7 +948,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const uint32_t ka = k_addr(j);
 #pragma unroll
                     for (int kk = 0; kk < G::kStepsRows; ++kk)
-                        ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + a_col(kk), desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                        ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + dp_col(j) + a_col(kk), desc_mnmajor<G>(ka, kk), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
                     if (single) {
                         // dQ += dS_lo K_j: the low parts sit 32 columns after the high parts.
 #pragma unroll
@@ -948,7 +956,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             ptx::mma_f16_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + a_col(kk) + 32, desc_mnmajor<G>(ka, kk), idesc_dq, 1u);
                     }
                     ptx::mma_commit(&bar_k_empty[j % RK]);
-                    if (j + 1 < n_kv && !issue_dp(j + 1)) { ok = false; break; }
+                    if (j + 2 < n_kv && !issue_dp(j + 2)) { ok = false; break; }
                 }
                 if (ok) ptx::mma_commit(&bar_dq_done);
             }
@@ -987,7 +995,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const int kv_valid = p.Nk - kv * kTileRows - kc0;
             uint32_t pk[32];
             bool got = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_s_full, 0, &abort_flag, tmo) &&
-                                                   ptx::mbar_wait(&bar_dp_full, 0, &abort_flag, tmo));
+                                                   ptx::mbar_wait(&bar_dp_full[0], 0, &abort_flag, tmo));
             float part = 0.f;
             if (got) {
                 ptx::tc_fence_after();
@@ -1098,13 +1106,14 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
-            if (!ptx::mbar_wait(&bar_dp_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar_dp_full[j & 1], (j >> 1) & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
+            const uint32_t dpc = dp_col(j);
             uint32_t dk[32];
             {
                 uint32_t ud[64];
-                ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0, *reinterpret_cast<uint32_t(*)[32]>(ud));
-                ptx::tmem_ld32(lane_base + Cfg::kColDP + kc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ud + 32));
+                ptx::tmem_ld32(lane_base + dpc + kc0, *reinterpret_cast<uint32_t(*)[32]>(ud));
+                ptx::tmem_ld32(lane_base + dpc + kc0 + 32, *reinterpret_cast<uint32_t(*)[32]>(ud + 32));
                 ptx::tmem_wait_ld();
                 const float2 ndv = make_float2(-dr, -dr);
 #pragma unroll
@@ -1115,8 +1124,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     dk[c >> 1] = G::pack2(ds.x, ds.y);
                 }
             }
-            // dS -> this group's own dP columns [128 + 64g, ... + 32), already read.
-            ptx::tmem_st32(lane_base + Cfg::kColDP + kc0, dk);
+            // dS -> this group's own columns of the dP buffer [64g, 64g + 32), already read.
+            ptx::tmem_st32(lane_base + dpc + kc0, dk);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
