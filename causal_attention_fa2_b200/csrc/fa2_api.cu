@@ -571,12 +571,10 @@ fa2_status check_keys(int B, int H_kv, int Nk) {
     return FA2_OK;
 }
 
-// Block mask (optional): 16-bit inputs only, at most kMaxMaskTiles tiles per side.
-fa2_status check_block_mask(const uint8_t* block_mask, int N, int Nk, fa2_dtype dtype) {
+// Block mask (optional): 16-bit inputs only; any number of tiles per side.
+fa2_status check_block_mask(const uint8_t* block_mask, fa2_dtype dtype) {
     if (!block_mask) return FA2_OK;
     if (dtype == FA2_FP32) return FA2_ERR_UNSUPPORTED_DTYPE;
-    if ((N + kTileRows - 1) / kTileRows > kMaxMaskTiles || (Nk + kTileRows - 1) / kTileRows > kMaxMaskTiles)
-        return FA2_ERR_BAD_SHAPE;
     return FA2_OK;
 }
 
@@ -587,7 +585,7 @@ fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, fl
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
-    if ((st = check_block_mask(block_mask, N, Nk, dtype)) != FA2_OK) return st;
+    if ((st = check_block_mask(block_mask, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
@@ -615,7 +613,7 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
-    if ((st = check_block_mask(block_mask, N, Nk, dtype)) != FA2_OK) return st;
+    if ((st = check_block_mask(block_mask, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||

@@ -299,10 +299,10 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int i_begin = p.causal ? kv_tile : 0;
     const int kv_row0 = kv_tile * kTileRows;
     constexpr bool sparse = SPARSE;
+    const int n_col = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;   // candidate query tiles
+    auto blk_set = [&](int t) { return __ldg(p.block_mask + static_cast<size_t>(i_begin + t) * p.n_tiles_k + kv_tile) != 0; };
     if (sparse && warp == 0) {
-        const int n = warp_compact(s_q, p.n_tiles > i_begin ? p.n_tiles - i_begin : 0,
-            [&](int t) { return p.block_mask[static_cast<size_t>(i_begin + t) * p.n_tiles_k + kv_tile] != 0; },
-            [&](int t) { return i_begin + t; });
+        const int n = warp_compact(s_q, n_col, blk_set, [&](int t) { return i_begin + t; });
         bool before = false;
         if (p.causal && kv_tile < p.n_tiles) {
             const uint8_t* row = p.block_mask + static_cast<size_t>(kv_tile) * p.n_tiles_k;
@@ -341,7 +341,10 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // Query tiles per query head; none when no query reaches this key tile
     // (causal with keys longer than queries, or an empty block column): then
     // dK = dV = 0 is written.
-    const int n_q = sparse ? s_nq : (p.n_tiles > i_begin ? p.n_tiles - i_begin : 0);
+    const int n_q = sparse ? s_nq : n_col;
+    // Past kMaxMaskTiles steps (or 16-bit tile indices) each thread walks the column.
+    const bool walk = sparse && (n_q > kMaxMaskTiles || p.n_tiles > 0xFFFF);
+    MaskWalk walker;
     // (query head, query tile) steps of the group, this CTA taking the split-th
     // of kv_splits consecutive shares.
     const int n_all = n_q * p.group;
@@ -351,7 +354,8 @@ fa2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // Step it: global step it0 + it = (query head) * n_q + (query tile index).
     auto q_tile_of = [&](int it) {
         const int g = (it0 + it) % n_q;
-        return sparse ? static_cast<int>(s_q[g]) : i_begin + g;
+        if (!sparse) return i_begin + g;
+        return walk ? i_begin + walker.at(g, n_col, blk_set) : static_cast<int>(s_q[g]);
     };
     auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + (it0 + it) / n_q; };
     // Steps whose query tile sees this key tile only (causal: query tile 0, or
@@ -783,7 +787,11 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_qdo_full;
     __shared__ uint64_t bar_k_full[RK], bar_k_empty[RK], bar_v_full[RV], bar_v_empty[RV];
-    __shared__ uint64_t bar_s_full, bar_dp_full[2], bar_s_read, bar_ds_ready;
+    // dP and dS of key tile j live in buffer j % 2, and so do their barriers: with
+    // dP(j+1) issued before dQ(j) a warp may finish dS(j+1) while another still
+    // works on dS(j), so one dS barrier would mix their arrivals.  (No warp gets
+    // two key tiles ahead: S(j+2) is issued only after every warp read S(j+1).)
+    __shared__ uint64_t bar_s_full, bar_dp_full[2], bar_s_read, bar_ds_ready[2];
     __shared__ uint64_t bar_dq_done, bar_drain[2];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
@@ -810,10 +818,10 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Key tiles this query tile sees (causal: key index <= query index).
     const int n_kv_lim = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
     constexpr bool sparse = SPARSE;
+    const uint8_t* mask_row = sparse ? p.block_mask + static_cast<size_t>(q_tile) * p.n_tiles_k : nullptr;
+    auto blk_set = [&](int j) { return __ldg(mask_row + j) != 0; };
     if (sparse && warp == 0) {
-        const uint8_t* row = p.block_mask + static_cast<size_t>(q_tile) * p.n_tiles_k;
-        const int n = warp_compact(s_kv, n_kv_lim, [&](int j) { return row[j] != 0; },
-                                   [&](int j) { return j; });
+        const int n = warp_compact(s_kv, n_kv_lim, blk_set, [&](int j) { return j; });
         if (lane == 0) s_nkv = n;
     }
     const int q_row0 = q_tile * kTileRows;
@@ -834,7 +842,8 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ptx::mbar_init(&bar_dp_full[0], 1);
         ptx::mbar_init(&bar_dp_full[1], 1);
         ptx::mbar_init(&bar_s_read, 8);
-        ptx::mbar_init(&bar_ds_ready, 8);
+        ptx::mbar_init(&bar_ds_ready[0], 8);
+        ptx::mbar_init(&bar_ds_ready[1], 8);
         ptx::mbar_init(&bar_dq_done, 1);
         ptx::mbar_init(&bar_drain[0], 1);
         ptx::mbar_init(&bar_drain[1], 1);
@@ -852,7 +861,13 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Key-tile steps; none for an empty block row, whose dQ is written as 0
     // (nothing is loaded, so the Q slot can stage the zeros).
     const int n_kv = sparse ? s_nkv : n_kv_lim;
-    auto kv_of = [&](int j) { return sparse ? static_cast<int>(s_kv[j]) : j; };
+    // Past kMaxMaskTiles steps (or 16-bit tile indices) each thread walks the row.
+    const bool walk = sparse && (n_kv > kMaxMaskTiles || p.n_tiles_k > 0xFFFF);
+    MaskWalk walker;
+    auto kv_of = [&](int j) {
+        if (!sparse) return j;
+        return walk ? walker.at(j, n_kv_lim, blk_set) : static_cast<int>(s_kv[j]);
+    };
     // A query tile that sees one key tile only (causal: the first query tile;
     // or a single key tile; or a block row with one block): every key its rows
     // see is in that tile, so those rows take D from the tile's own P and dP and
@@ -943,7 +958,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (ok && n_kv > 1) ok = issue_dp(1);
                 for (int j = 0; ok && j < n_kv; ++j) {
                     // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
-                    if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo) || !wait_k(j)) { ok = false; break; }
+                    if (!ptx::mbar_wait(&bar_ds_ready[j & 1], (j >> 1) & 1, &abort_flag, tmo) || !wait_k(j)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t ka = k_addr(j);
 #pragma unroll
@@ -1068,7 +1083,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+                if (lane == 0) ptx::mbar_arrive(&bar_ds_ready[0]);
             }
         }
         for (int j = 0; !single && j < n_kv; ++j) {
@@ -1129,7 +1144,7 @@ fa2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready[j & 1]);
         }
         // ---------------- epilogue (group 0): dQ * scale -> shared memory -> TMA store.
         if (g == 0) {

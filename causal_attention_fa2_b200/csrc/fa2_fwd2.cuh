@@ -73,6 +73,15 @@ struct Fwd2Cfg {
     static __device__ __forceinline__ uint32_t col_o(int t) { return 256u + 128u * t; }
 };
 
+// Block-sparse: the mask rows of a CTA's two query tiles, and the largest key
+// tile each may see (causal limit; -1 for a missing tile B).
+struct PairRows {
+    const uint8_t* row[2];
+    int lim[2];
+    __device__ __forceinline__ bool on(int t, int j) const { return j <= lim[t] && __ldg(row[t] + j) != 0; }
+    __device__ __forceinline__ bool any(int j) const { return on(0, j) || on(1, j); }
+};
+
 // One softmax warpgroup: processes query tile `t` (0 = A, 1 = B) for key
 // tiles 0 .. n_kv-1, then writes its O tile and L rows.
 template <int ES, int D, bool F16, bool SPARSE>
@@ -80,6 +89,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
                                              int bh, uint32_t tmem, uint8_t* sQt,
                                              uint64_t* bar_s_full, uint64_t* bar_p_full,
                                              uint64_t* bar_o_done, const uint16_t* kv_list,
+                                             const PairRows* pr, bool walk,
                                              volatile uint32_t* abort_flag,
                                              const CUtensorMap* tm_o) {
     using Cfg = Fwd2Cfg<ES, D, F16>;
@@ -97,11 +107,21 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
     float m_raw = -INFINITY;    // reference max of raw scores
     float l = 0.f;
     bool ok = true;
+    MaskWalk walker;
     for (int j = 0; j < n_kv; ++j) {
         // Key tile of step j, and (block-sparse) whether its block is set for this
         // query tile: a step the other tile needs but this one does not is masked.
-        const int kv = SPARSE ? (kv_list[j] & 0x3FFF) : j;
-        const bool blk_on = !SPARSE || ((kv_list[j] >> (14 + t)) & 1);
+        int kv = j;
+        bool blk_on = true;
+        if constexpr (SPARSE) {
+            if (walk) {
+                kv = walker.at(j, p.n_tiles_k, [&](int x) { return pr->any(x); });
+                blk_on = pr->on(t, kv);
+            } else {
+                kv = kv_list[j] & 0x3FFF;
+                blk_on = (kv_list[j] >> (14 + t)) & 1;
+            }
+        }
         if (!ptx::mbar_wait(bar_s_full, j & 1, abort_flag, tmo)) { ok = false; break; }
         ptx::tc_fence_after();
         float s[128];
@@ -276,9 +296,11 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     // Block-sparse: the pair's key tiles, in order, with bit 14 / 15 set when
-    // the block of query tile A / B is set; s_cnt = steps of tile A, of the pair.
+    // the block of query tile A / B is set (the first kMaxMaskTiles steps);
+    // s_cnt = steps of tile A, of the pair.
     __shared__ uint16_t s_kv[SPARSE ? kMaxMaskTiles : 1];
     __shared__ int s_cnt[2];
+    __shared__ PairRows s_pr;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -300,23 +322,25 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const bool has_b = tile[1] < p.n_tiles;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
     constexpr bool sparse = SPARSE;
+    // Key tiles of the pair: those whose block is set for tile A or tile B (and,
+    // causal, at or below that tile).  Tile A visits the prefix up to its own
+    // diagonal; steps whose block is set only for B are masked for A.
     if (sparse && warp == 0) {
-        // Key tiles of the pair: those whose block is set for tile A or tile B
-        // (and, causal, at or below that tile).  Tile A visits the prefix up to
-        // its own diagonal; steps whose block is set only for B are masked for A.
-        const uint8_t* row_a = p.block_mask + static_cast<size_t>(tile[0]) * p.n_tiles_k;
-        const uint8_t* row_b = p.block_mask + static_cast<size_t>(has_b ? tile[1] : tile[0]) * p.n_tiles_k;
-        auto on_a = [&](int j) { return (!p.causal || j <= tile[0]) && row_a[j] != 0; };
-        auto on_b = [&](int j) { return has_b && (!p.causal || j <= tile[1]) && row_b[j] != 0; };
-        auto any = [&](int j) { return on_a(j) || on_b(j); };
-        const int n_pair = warp_compact(s_kv, p.n_tiles_k, any,
-            [&](int j) { return j | (on_a(j) ? 0x4000 : 0) | (on_b(j) ? 0x8000 : 0); });
+        PairRows pr;
+        const int last = p.n_tiles_k - 1;
+        pr.row[0] = p.block_mask + static_cast<size_t>(tile[0]) * p.n_tiles_k;
+        pr.row[1] = p.block_mask + static_cast<size_t>(has_b ? tile[1] : tile[0]) * p.n_tiles_k;
+        pr.lim[0] = p.causal ? min(tile[0], last) : last;
+        pr.lim[1] = has_b ? (p.causal ? min(tile[1], last) : last) : -1;
+        if (lane == 0) s_pr = pr;
+        const int n_pair = warp_compact(s_kv, p.n_tiles_k, [&](int j) { return pr.any(j); },
+            [&](int j) { return j | (pr.on(0, j) ? 0x4000 : 0) | (pr.on(1, j) ? 0x8000 : 0); });
         int n_a = n_pair;
         if (p.causal) {
             n_a = 0;
             for (int base = 0; base <= tile[0] && base < p.n_tiles_k; base += 32) {
                 const int j = base + lane;
-                n_a += __popc(__ballot_sync(0xffffffffu, j <= tile[0] && j < p.n_tiles_k && any(j)));
+                n_a += __popc(__ballot_sync(0xffffffffu, j <= tile[0] && j < p.n_tiles_k && pr.any(j)));
             }
         }
         if (lane == 0) { s_cnt[0] = n_a; s_cnt[1] = n_pair; }
@@ -360,7 +384,14 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
     const bool load_q[2] = {n_kv_t[0] > 0, n_kv_t[1] > 0};
-    auto kv_of = [&](int j) { return sparse ? (s_kv[j] & 0x3FFF) : j; };
+    // The shared-memory list holds kMaxMaskTiles steps of 14-bit key tiles;
+    // beyond that each thread walks the mask rows itself.
+    const bool walk = sparse && (s_cnt[1] > kMaxMaskTiles || p.n_tiles_k > 0x4000);
+    MaskWalk walker;
+    auto kv_of = [&](int j) {
+        if (!sparse) return j;
+        return walk ? walker.at(j, p.n_tiles_k, [&](int x) { return s_pr.any(x); }) : static_cast<int>(s_kv[j] & 0x3FFF);
+    };
 
     // Each warpgroup changes its register count inside its own branch, so the
     // compiler allocates each role's code for the count that role runs with.
@@ -502,7 +533,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Every existing query tile writes O and L, also one without key steps.
         if (SPARSE ? tile[t] < p.n_tiles : n_kv_t[t] > 0) {
             fwd2_softmax<ES, D, F16, SPARSE>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
-                                &bar_p_full[t], &bar_o_done[t], s_kv,
+                                &bar_p_full[t], &bar_o_done[t], s_kv, &s_pr, walk,
                                 &abort_flag, &tm_o);
         }
     }

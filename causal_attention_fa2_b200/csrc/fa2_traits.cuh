@@ -61,13 +61,15 @@ inline int heads_per_group(int n_heads, int n_rank) {
 // Block-sparse attention ("Notes on flashattention", section "Block-sparse
 // Flashattention"): a byte per (query tile, key tile) pair of kTileRows x
 // kTileRows blocks, row-major with one row per query tile; zero blocks are
-// skipped.  A CTA compacts the tiles it visits into a shared-memory list of at
-// most kMaxMaskTiles entries, so masks cover at most that many tiles per side.
+// skipped.  A CTA compacts the tiles it visits into a shared-memory list of
+// kMaxMaskTiles 16-bit entries; a CTA whose tiles do not fit there (more steps,
+// or tile indices wider than the entries) walks the mask itself (MaskWalk).
 constexpr int kMaxMaskTiles = 512;
 
 // Warp-cooperative compaction (whole warp): writes, in increasing order, the
-// value val(t) of every t in [0, n) with keep(t) into list[], and returns the
-// count (the same in every lane).
+// value val(t) of every t in [0, n) with keep(t) into list[] (the first
+// kMaxMaskTiles of them), and returns the count of all of them (the same in
+// every lane).
 template <class Keep, class Val>
 __device__ __forceinline__ int warp_compact(uint16_t* list, int n, Keep keep, Val val) {
     const int lane = threadIdx.x & 31;
@@ -80,8 +82,27 @@ __device__ __forceinline__ int warp_compact(uint16_t* list, int n, Keep keep, Va
             list[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(val(t));
         count += __popc(bal);
     }
-    return count < kMaxMaskTiles ? count : kMaxMaskTiles;
+    return count;
 }
+
+// The s-th (s = 0, 1, 2, ...) index t in [0, n) with keep(t), found by walking
+// the mask from the previous answer: one thread's replacement for the
+// shared-memory list.  Steps are asked for in increasing order (asking for an
+// earlier step restarts the walk); a step past the last index gives n.
+struct MaskWalk {
+    int step = -1;   // step number of `pos`
+    int pos = -1;    // index of that step
+    template <class Keep>
+    __device__ __forceinline__ int at(int s, int n, Keep keep) {
+        if (s < step) { step = -1; pos = -1; }
+        while (step < s && pos < n) {
+            ++pos;
+            while (pos < n && !keep(pos)) ++pos;
+            ++step;
+        }
+        return pos < n ? pos : n;
+    }
+};
 
 // Device status codes the kernels record (same values as fa2_status).
 constexpr uint32_t kDevStatusTimeout = 8;

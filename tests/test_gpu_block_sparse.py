@@ -43,6 +43,15 @@ def _mask(kind, nq_t, nk_t, seed):
         return np.zeros((nq_t, nk_t), dtype=np.uint8)
     if kind == "ones":
         return np.ones((nq_t, nk_t), dtype=np.uint8)
+    if kind == "mostly_ones":                              # long rows / columns with a few holes
+        m = np.ones((nq_t, nk_t), dtype=np.uint8)
+        if nk_t > 8:
+            for i in range(nq_t):
+                m[i, rng.choice(nk_t, 3, replace=False)] = 0
+        if nq_t > 8:
+            for j in range(nk_t):
+                m[rng.choice(nq_t, 3, replace=False), j] = 0
+        return m
     raise ValueError(kind)
 
 
@@ -68,6 +77,12 @@ CASES = [
     (1, 2, 2, 768, 768, 64, "bf16", True, "pair_split"),
     (1, 2, 2, 768, 640, 16, "fp16", False, "pair_split"),
     (1, 2, 2, 384, 384, 32, "bf16", True, "empty"),
+    # More than 512 tiles on one side (520 x 128 rows), about 517 set blocks per
+    # row (forward, dQ pass) or per column (dK/dV pass): past the shared-memory
+    # tile list, the kernels walk the mask.
+    (1, 2, 2, 128, 520 * 128, 16, "bf16", False, "mostly_ones"),
+    (1, 2, 2, 520 * 128, 1024, 16, "bf16", False, "mostly_ones"),
+    (1, 2, 1, 200, 520 * 128 - 37, 32, "fp16", False, "mostly_ones"),
 ]
 
 
@@ -78,6 +93,14 @@ def test_block_sparse_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal, ki
     nq_t, nk_t = -(-N // BLOCK), -(-Nk // BLOCK)
     mask = _mask(kind, nq_t, nk_t, seed=N + Nk + d)
     q, k, v, do = _inputs(B, H, H_kv, N, Nk, d, dtype, seed=500 + N + Nk + d)
+    if N > 512 * BLOCK:
+        # Every dK, dV element here sums about 66 000 query rows, and its error
+        # follows the largest values (about 0.3 % of max |dK|, |dV| in the dense
+        # kernels as well, whose bits the mask walk reproduces for a mask of ones):
+        # with unit-variance dO those reach 15-20 and the error the absolute part
+        # of the bound.  dK and dV are linear in dO, so dO / 8 keeps the check
+        # element-wise at the same bound.
+        do = (do.float() / 8).to(do.dtype)
     scale = default_scale(d)
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     md = torch.from_numpy(mask).to(dev)
@@ -134,6 +157,31 @@ def test_all_ones_mask_is_bitwise_dense():
         torch.cuda.synchronize()
         assert torch.equal(o, o2) and torch.equal(lse, lse2)
         assert all(torch.equal(a, b) for a, b in zip(g, g2))
+
+
+@pytest.mark.parametrize("B,H,H_kv,N,Nk,d,causal", [
+    (1, 1, 1, 520 * 128, 520 * 128, 16, True),     # query-tile pairs, up to 520 steps per row / column
+    (1, 148, 1, 256, 520 * 128, 16, False),        # 148 query-tile pairs of 520 key tiles each
+])
+def test_all_ones_mask_past_the_tile_list_is_bitwise_dense(B, H, H_kv, N, Nk, d, causal):
+    """More than 512 tiles per side: the kernels walk a mask of ones and must
+    give the dense entry points' bits."""
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(N + Nk + H)
+    q, do = (torch.randn((B, H, N, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+    k, v = (torch.randn((B, H_kv, Nk, d), generator=g, device=dev).to(torch.bfloat16) for _ in range(2))
+    ones = torch.ones(-(-N // BLOCK), -(-Nk // BLOCK), dtype=torch.bool, device=dev)
+    o, lse = fa2.forward(q, k, v, causal=causal)
+    o2, lse2 = fa2.forward(q, k, v, causal=causal, block_mask=ones)
+    grads = fa2.backward(q, k, v, o, lse, do, causal=causal, mode="two-pass")
+    grads2 = fa2.backward(q, k, v, o, lse, do, causal=causal, block_mask=ones)
+    torch.cuda.synchronize()
+    assert fa2.last_device_status() == 0
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    for a, b in zip(grads, grads2):
+        assert torch.equal(a, b)
 
 
 def test_block_sparse_deterministic():
