@@ -113,8 +113,8 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tr
     q: contiguous CUDA tensor [B, H, N, d] (bf16, fp16 or fp32); k, v:
     [B, H_kv, Nk, d] with H a multiple of H_kv (grouped-query attention when
     H_kv < H: query head h uses key/value head h // (H // H_kv)); with
-    causal, key j is visible to query i iff j <= i.  ``block_mask`` (optional,
-    16-bit inputs): block-sparse attention, a CUDA bool / uint8 tensor
+    causal, key j is visible to query i iff j <= i.  ``block_mask`` (optional):
+    block-sparse attention, a CUDA bool / uint8 tensor
     [ceil(N / 128), ceil(Nk / 128)]; zero blocks of 128 x 128 rows are skipped,
     rows that see no key get O = 0 and L = -inf.
     Returns (o [B, H, N, d] in the input dtype, lse [B, H, N] float32).

@@ -268,7 +268,7 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
         if ((st = set_smem(kern, Cfg2::kSmemBytes)) != FA2_OK) return st;
         launch_pdl(kern, dim3(static_cast<unsigned>(n_items) * static_cast<unsigned>(BH)), dim3(Cfg2::kThreads), Cfg2::kSmemBytes, stream, mq, mk, mv, mo, p);
     } else {
-        auto kern = fa2_fwd_kernel<ES, D>;
+        auto kern = block_mask ? fa2_fwd_kernel<ES, D, true> : fa2_fwd_kernel<ES, D, false>;
         if ((st = set_smem(kern, Cfg::kSmemBytes)) != FA2_OK) return st;
         const unsigned grid = static_cast<unsigned>(p.n_tiles) * static_cast<unsigned>(BH);
         launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, mq, mk, mv, mo, p);
@@ -426,7 +426,8 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
                                int B, int H, int H_kv, int N, int Nk, int causal, float scale, uint8_t* ws_base,
                                const BwdWorkspace& ws, cudaStream_t stream, uint32_t* status,
-                               unsigned long long timeout_ns, void* const* events) {
+                               unsigned long long timeout_ns, void* const* events,
+                               const uint8_t* block_mask) {
     using Cfg = Bwd32Cfg<D>;
     using G = typename Cfg::G;
     constexpr fa2_dtype dt = FA2_FP32;
@@ -484,7 +485,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     p.scale_log2 = scale * 1.4426950408889634f;
     p.scale = scale;
     p.timeout_ns = timeout_ns;
-    p.block_mask = nullptr;                              // block-sparse: 16-bit inputs only
+    p.block_mask = block_mask;
     p.kv_splits = 1;                                     // fp32: one CTA per group
     p.part = nullptr;
     p.item0 = 0;
@@ -500,7 +501,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             (st = kmap(&mkk, k, W, BH_kv, Nk)) != FA2_OK || (st = mnmap(&mkmn, k, W, BH_kv, Nk)) != FA2_OK ||
             (st = kmap(&mvk, v, W, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdq, dq, kTileRows, BH, N)) != FA2_OK)
             return st;
-        auto kern = fa2_bwd32_dq_kernel<D>;
+        auto kern = block_mask ? fa2_bwd32_dq_kernel<D, true> : fa2_bwd32_dq_kernel<D, false>;
         if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
         launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemQ, stream, mq, mdo, mkk, mkmn, mvk, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
@@ -513,7 +514,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             (st = kmap(&mdok, dout, W, BH, N)) != FA2_OK || (st = mnmap(&mdomn, dout, W, BH, N)) != FA2_OK ||
             (st = kmap(&mdk, dk, kTileRows, BH_kv, Nk)) != FA2_OK || (st = kmap(&mdv, dv, kTileRows, BH_kv, Nk)) != FA2_OK)
             return st;
-        auto kern = fa2_bwd32_dkdv_kernel<D>;
+        auto kern = block_mask ? fa2_bwd32_dkdv_kernel<D, true> : fa2_bwd32_dkdv_kernel<D, false>;
         if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
         launch_pdl(kern, dim3(grid_kv), dim3(Cfg::kThreads), Cfg::kSmemKV, stream, mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
@@ -531,7 +532,8 @@ fa2_status launch_backward(const void* q, const void* k, const void* v, const vo
     case DD:                                                                                  \
         if (dtype == FA2_FP32)                                                                \
             return launch_backward32_t<DD>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, causal, \
-                                           scale, ws_base, ws, stream, status, timeout_ns, events); \
+                                           scale, ws_base, ws, stream, status, timeout_ns, events, \
+                                           block_mask);                                  \
         if (dtype == FA2_FP16)                                                                \
             return launch_backward_t<2, DD, true>(q, k, v, o, lse, dout, dq, dk, dv, B, H, H_kv, N, Nk, \
                                                   causal, scale, dtype, ws_base, ws, stream,    \
@@ -571,13 +573,6 @@ fa2_status check_keys(int B, int H_kv, int Nk) {
     return FA2_OK;
 }
 
-// Block mask (optional): 16-bit inputs only; any number of tiles per side.
-fa2_status check_block_mask(const uint8_t* block_mask, fa2_dtype dtype) {
-    if (!block_mask) return FA2_OK;
-    if (dtype == FA2_FP32) return FA2_ERR_UNSUPPORTED_DTYPE;
-    return FA2_OK;
-}
-
 fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int H, int H_kv, int N, int Nk, int d, int causal, float scale,
                         fa2_dtype dtype, fa2_stream_t stream, const uint8_t* block_mask = nullptr) {
@@ -585,7 +580,6 @@ fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, fl
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
-    if ((st = check_block_mask(block_mask, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse) return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
@@ -600,7 +594,8 @@ fa2_status forward_impl(const void* q, const void* k, const void* v, void* o, fl
     if (dtype == FA2_FP16)
         return dispatch_forward<2, true>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s,
                                          status, block_mask);
-    return dispatch_forward<4>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status);
+    return dispatch_forward<4>(d, q, k, v, o, lse, B, H, H_kv, N, Nk, causal, scale, dtype, s, status,
+                               block_mask);
 }
 
 fa2_status backward_impl(const void* q, const void* k, const void* v, const void* o,
@@ -613,7 +608,6 @@ fa2_status backward_impl(const void* q, const void* k, const void* v, const void
     if (st != FA2_OK) return st;
     if ((st = check_heads(H, H_kv)) != FA2_OK) return st;
     if ((st = check_keys(B, H_kv, Nk)) != FA2_OK) return st;
-    if ((st = check_block_mask(block_mask, dtype)) != FA2_OK) return st;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
         return FA2_ERR_NULL_PTR;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||

@@ -228,7 +228,9 @@ __device__ __forceinline__ void bwd32_stage_rows(uint32_t acc_col, int r, float 
 // that see key tile j stream through in sub-tiles of W rows.  Per sub-tile
 // the MMA issuer runs S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q,
 // issuing the next sub-tile's S^T right after dV and its dP^T right after dK.
-template <int D>
+// With a block mask (SPARSE) only the sub-tiles of query tiles whose block with
+// key tile j is set are visited, found by each thread walking the mask column.
+template <int D, bool SPARSE = false>
 __global__ void __launch_bounds__(192, 1)
 fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_constant__ CUtensorMap tm_qmn,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -253,6 +255,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_dkv_full, bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    __shared__ int s_cnt;                               // block-sparse: query sub-tiles per head
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -278,12 +281,22 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     const int kv_row0 = kv_tile * kTileRows;
     const int n_sub = (p.N + W - 1) / W;                // query sub-tiles
     const int sub_begin = p.causal ? kv_row0 / W : 0;
-    // Sub-tiles per query head; none when no query reaches this key tile
-    // (causal, keys longer than queries): then dK = dV = 0 is written.
-    const int n_q = n_sub > sub_begin ? n_sub - sub_begin : 0;
-    const int n_it = n_q * p.group;                     // (query head, sub-tile) steps
-    auto q_row_of = [&](int it) { return (sub_begin + it % n_q) * W; };
-    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
+    constexpr int R = kTileRows / W;                    // sub-tiles per 128-row tile
+    // Block-sparse: query tiles i_begin + t (t < n_col) whose block is set.
+    const int i_begin = p.causal ? kv_tile : 0;
+    const int n_col = p.n_tiles > i_begin ? p.n_tiles - i_begin : 0;
+    auto blk_set = [&](int t) {
+        return __ldg(p.block_mask + static_cast<size_t>(i_begin + t) * p.n_tiles_k + kv_tile) != 0;
+    };
+    if (SPARSE && warp == 0) {
+        int c = 0;
+        for (int base = 0; base < n_col; base += 32)
+            c += __popc(__ballot_sync(0xffffffffu, base + lane < n_col && blk_set(base + lane)));
+        // R sub-tiles per set query tile; the last query tile's end at n_sub.
+        const bool last = n_col > 0 && blk_set(n_col - 1);
+        if (lane == 0) s_cnt = c * R - (last ? p.n_tiles * R - n_sub : 0);
+    }
+    MaskWalk walker;
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -309,6 +322,17 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Sub-tiles per query head; none when no query reaches this key tile
+    // (causal, keys longer than queries; or an empty block column): then
+    // dK = dV = 0 is written.
+    const int n_q = SPARSE ? s_cnt : (n_sub > sub_begin ? n_sub - sub_begin : 0);
+    const int n_it = n_q * p.group;                     // (query head, sub-tile) steps
+    auto q_row_of = [&](int it) {
+        const int g = it % n_q;
+        if (!SPARSE) return (sub_begin + g) * W;
+        return ((i_begin + walker.at(g / R, n_col, blk_set)) * R + g % R) * W;
+    };
+    auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -482,7 +506,9 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 // query tile i sees stream through in sub-tiles of W rows.  Per sub-tile the
 // MMA issuer runs S = Q K^T, dP = dO V^T, dQ += dS K, issuing the next S as
 // soon as the warpgroup has read this one and the next dP right after dQ.
-template <int D>
+// With a block mask (SPARSE) only the sub-tiles of key tiles whose block with
+// query tile i is set are visited, found by each thread walking the mask row.
+template <int D, bool SPARSE = false>
 __global__ void __launch_bounds__(192, 1)
 fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_kk, const __grid_constant__ CUtensorMap tm_kmn,
@@ -505,6 +531,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready, bar_dq_done, bar_drain;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    __shared__ int s_cnt;                               // block-sparse: key sub-tiles
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -527,8 +554,23 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int q_row0 = q_tile * kTileRows;
     const int n_sub = (p.Nk + W - 1) / W;               // key sub-tiles
     const int lim = (q_row0 + kTileRows) / W;
-    const int n_kv = p.causal ? (lim < n_sub ? lim : n_sub) : n_sub;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
+    constexpr int R = kTileRows / W;                    // sub-tiles per 128-row tile
+    // Block-sparse: key tiles t < n_lim whose block with this query tile is set.
+    const int n_lim = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
+    const uint8_t* mask_row = SPARSE ? p.block_mask + static_cast<size_t>(q_tile) * p.n_tiles_k : nullptr;
+    auto blk_set = [&](int t) { return __ldg(mask_row + t) != 0; };
+    if (SPARSE && warp == 0) {
+        int c = 0;
+        for (int base = 0; base < n_lim; base += 32)
+            c += __popc(__ballot_sync(0xffffffffu, base + lane < n_lim && blk_set(base + lane)));
+        // R sub-tiles per set key tile; the last key tile's end at n_sub.
+        const bool last = n_lim == p.n_tiles_k && n_lim > 0 && blk_set(n_lim - 1);
+        if (lane == 0) s_cnt = c * R - (last ? p.n_tiles_k * R - n_sub : 0);
+    }
+    MaskWalk walker;
+    // Key sub-tile of step j.
+    auto kvs_of = [&](int j) { return SPARSE ? walker.at(j / R, n_lim, blk_set) * R + j % R : j; };
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -554,10 +596,12 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    // Key sub-tile steps; none for an empty block row, whose dQ is written as 0.
+    const int n_kv = SPARSE ? s_cnt : (p.causal ? (lim < n_sub ? lim : n_sub) : n_sub);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && n_kv > 0) {
             ptx::prefetch_tmap(&tm_kk);
             ptx::prefetch_tmap(&tm_kmn);
             ptx::prefetch_tmap(&tm_vk);
@@ -571,7 +615,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             for (int j = 0; j < n_kv; ++j) {
                 const int s = j % ST;
                 if (j >= ST && !ptx::mbar_wait(&bar_empty[s], ((j / ST) & 1) ^ 1, &abort_flag, tmo)) break;
-                const int row0 = j * W;
+                const int row0 = kvs_of(j) * W;
                 ptx::mbar_arrive_expect_tx(&bar_full[s], SB);
                 for (int b = 0; b < G::kNBoxK; ++b) {
                     ptx::tma_load_3d_hint(st_kk(s) + b * W * G::kRowBK, &tm_kk, &bar_full[s], b * G::kBoxK, row0, bh_kv, keep);
@@ -590,7 +634,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && n_kv > 0) {
             constexpr uint32_t idesc_s = ptx::instr_desc(G::kFmt, 128, W, false, false);
             constexpr uint32_t idesc_dq = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr = ptx::smem_addr(sQ);
@@ -652,7 +696,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float dr = p.dvec[vrow];                   // D_i (0 past N)
         bool ok = true;
         for (int j = 0; j < n_kv; ++j) {
-            const int k0 = j * W;
+            const int k0 = kvs_of(j) * W;
             const bool mask = p.causal && k0 + W - 1 > q_row0;   // some key follows some query
             const int kv_valid = p.Nk - k0;                         // key columns < Nk
             // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14), kept in registers
@@ -678,11 +722,12 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
         }
-        // ---------------- epilogue: dQ * scale -> sQ -> TMA store.
-        if (ok) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
+        // ---------------- epilogue: dQ * scale -> sQ -> TMA store (zeros when no
+        // key tile was visited; nothing was loaded into sQ then).
+        if (ok && n_kv > 0) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDQ, r, p.scale, sQ);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDQ, r, p.scale, sQ, n_kv == 0);
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");

@@ -99,7 +99,7 @@ __device__ __forceinline__ void round_tf32_smem(uint8_t* base, int bytes, int la
     __syncwarp();
 }
 
-template <int ES, int D>
+template <int ES, int D, bool SPARSE = false>
 __global__ void __launch_bounds__(FwdCfg<ES, D>::kThreads, 1)
 fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -122,6 +122,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint64_t bar_q_ready, bar_k_ready[KST], bar_v_ready[VST];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
+    __shared__ int s_cnt;                      // block-sparse: key tiles of this query tile
     uint64_t* const q_go = G::kF32 ? &bar_q_ready : &bar_q_full;
     uint64_t* const k_go = G::kF32 ? bar_k_ready : bar_k_full;
     uint64_t* const v_go = G::kF32 ? bar_v_ready : bar_v_full;
@@ -140,10 +141,20 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int tile_rank = item / p.BH;
     const int bh = item - tile_rank * p.BH;
     const int q_tile = p.causal ? (p.n_tiles - 1 - tile_rank) : tile_rank;
-    // Key tiles this query tile sees (causal: key index <= query index).
-    const int n_kv = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
+    // Key tiles this query tile sees (causal: key index <= query index); with a
+    // block mask, those whose block is set, found by each thread walking the
+    // mask row (no shared-memory list here: the fp32 tiles fill shared memory).
+    const int n_kv_lim = p.causal ? min(q_tile + 1, p.n_tiles_k) : p.n_tiles_k;
     const int q_row0 = q_tile * kTileRows;
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
+    const uint8_t* mask_row = SPARSE ? p.block_mask + static_cast<size_t>(q_tile) * p.n_tiles_k : nullptr;
+    auto blk_set = [&](int j) { return __ldg(mask_row + j) != 0; };
+    if (SPARSE && warp == 0) {
+        int c = 0;
+        for (int base = 0; base < n_kv_lim; base += 32)
+            c += __popc(__ballot_sync(0xffffffffu, base + lane < n_kv_lim && blk_set(base + lane)));
+        if (lane == 0) s_cnt = c;
+    }
 
     if (threadIdx.x == 0) {
         abort_flag = 0u;
@@ -167,10 +178,15 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
+    const int n_kv = SPARSE ? s_cnt : n_kv_lim;
+    MaskWalk walker;
+    auto kv_of = [&](int j) { return SPARSE ? walker.at(j, n_kv_lim, blk_set) : j; };
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
+        // (nothing for a query tile without key tiles: its epilogue stages zeros
+        // in the Q slot, which no copy or rounding may touch then)
+        if (lane == 0 && n_kv > 0) {
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_k);
             ptx::prefetch_tmap(&tm_v);
@@ -184,14 +200,14 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 uint8_t* dk = sK + ks * G::kTileBytesK;
                 ptx::mbar_arrive_expect_tx(&bar_k_full[ks], G::kTileBytesK);
                 for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, j * kTileRows, bh_kv);
+                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, kv_of(j) * kTileRows, bh_kv);
                 k_issued = j + 1;
                 const int vs = j % VST;
                 if (j >= VST && !ptx::mbar_wait(&bar_v_empty[vs], ((j / VST) & 1) ^ 1, &abort_flag, tmo)) break;
                 uint8_t* dv = sV + vs * G::kTileBytesMN;
                 ptx::mbar_arrive_expect_tx(&bar_v_full[vs], G::kTileBytesMN);
                 for (int b = 0; b < G::kNBoxMN; ++b)
-                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, j * kTileRows, bh_kv);
+                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, kv_of(j) * kTileRows, bh_kv);
                 v_issued = j + 1;
             }
             if (abort_flag) {
@@ -206,7 +222,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && n_kv > 0) {
             constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr = ptx::smem_addr(sQ);
@@ -282,8 +298,9 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             // Mask: causal diagonal tile (key > query), or keys past N.
-            const bool diag = p.causal && (j == q_tile);
-            const int kv_valid = p.Nk - j * kTileRows;
+            const int kv = kv_of(j);
+            const bool diag = p.causal && (kv == q_tile);
+            const int kv_valid = p.Nk - kv * kTileRows;
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 128; ++c) {
@@ -347,16 +364,19 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_p_full[j & 1]);
         }
-        // ---------------- epilogue: O / l -> shared memory -> TMA store; L.
-        if (ok) ok = ptx::mbar_wait(&bar_o_done, (n_kv - 1) & 1, &abort_flag, tmo);
+        // ---------------- epilogue: O / l -> shared memory -> TMA store; L.  A query
+        // tile whose block row is empty writes O = 0 and L = -inf.
+        if (ok && n_kv > 0) ok = ptx::mbar_wait(&bar_o_done, (n_kv - 1) & 1, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
-            const float inv_l = 1.f / l;
+            const float inv_l = n_kv > 0 ? 1.f / l : 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < G::kNOut; c0 += 16) {
-                uint32_t u[16];
-                ptx::tmem_ld16(o_tmem + c0, u);
-                ptx::tmem_wait_ld();
+                uint32_t u[16] = {};
+                if (n_kv > 0) {
+                    ptx::tmem_ld16(o_tmem + c0, u);
+                    ptx::tmem_wait_ld();
+                }
                 if constexpr (G::kF32) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
@@ -388,7 +408,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             const int q_row = q_row0 + r;
             if (q_row < p.N)
-                p.lse[static_cast<size_t>(bh) * p.N + q_row] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+                p.lse[static_cast<size_t>(bh) * p.N + q_row] =
+                    n_kv > 0 ? (m_ref + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -401,7 +422,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
         // ------------------------------------------------ TF32 rounding (fp32 only)
         if constexpr (G::kF32) {
-            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            bool ok = n_kv > 0 && ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
             if (ok) {
                 round_tf32_smem(sQ, G::kTileBytesK, lane);
                 if (lane == 0) ptx::mbar_arrive(&bar_q_ready);

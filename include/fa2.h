@@ -195,11 +195,11 @@ fa2_status fa2_backward_ex(const void* q, const void* k, const void* v, const vo
  * A query row that sees no key (its block row is empty) gets O = 0 and
  * L = -inf; its dQ is 0 and it adds nothing to dK or dV.  Other arguments,
  * results and the workspace are those of fa2_forward_ex / fa2_backward_ex.
- * Any N and Nk the dense calls accept: a thread block keeps the tiles it
- * visits in a list of 512 entries and walks the mask itself when there are
- * more.  Errors: block_mask NULL -> FA2_ERR_NULL_PTR; FA2_FP32 inputs ->
- * FA2_ERR_UNSUPPORTED_DTYPE (16-bit inputs only).  A mask of all ones gives the
- * results of fa2_forward_ex / fa2_backward_ex.
+ * Every input type and any N and Nk the dense calls accept (a thread block
+ * keeps the tiles it visits in a list of 512 entries, 16-bit inputs, and walks
+ * the mask itself past that or for fp32 inputs).  Errors: block_mask NULL ->
+ * FA2_ERR_NULL_PTR.  A mask of all ones gives the results of fa2_forward_ex /
+ * fa2_backward_ex.
  */
 fa2_status fa2_forward_block_sparse(const void* q, const void* k, const void* v, void* o,
                                     float* lse, int B, int H, int H_kv, int N, int Nk, int d,

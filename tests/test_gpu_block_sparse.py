@@ -83,6 +83,13 @@ CASES = [
     (1, 2, 2, 128, 520 * 128, 16, "bf16", False, "mostly_ones"),
     (1, 2, 2, 520 * 128, 1024, 16, "bf16", False, "mostly_ones"),
     (1, 2, 1, 200, 520 * 128 - 37, 32, "fp16", False, "mostly_ones"),
+    # fp32 inputs (TF32 kernels, streamed in sub-tiles of W rows: every set block
+    # is visited as its 128 / W sub-tiles).
+    (1, 2, 2, 640, 640, 64, "fp32", True, "random"),
+    (1, 4, 2, 600, 700, 128, "fp32", False, "random"),
+    (1, 2, 2, 768, 768, 32, "fp32", True, "pair_split"),
+    (1, 2, 2, 700, 450, 16, "fp32", False, "band"),
+    (1, 2, 2, 384, 384, 80, "fp32", True, "empty"),
 ]
 
 
@@ -141,13 +148,14 @@ def test_block_sparse_parity(oracle_mod, B, H, H_kv, N, Nk, d, dtype, causal, ki
         assert (err <= bound).all(), (name, float(err.max()), int((err > bound).sum()))
 
 
-def test_all_ones_mask_is_bitwise_dense():
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_all_ones_mask_is_bitwise_dense(dtype):
     """A mask of ones gives the bits of the dense entry points (block masks
     take the two-pass backward, so the dense one runs with FA2_BWD_DETERMINISTIC)."""
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
     B, H, N, d = 1, 4, 700, 64
-    q, k, v, do = (t.to(dev) for t in _inputs(B, H, H, N, N, d, "bf16", seed=9))
+    q, k, v, do = (t.to(dev) for t in _inputs(B, H, H, N, N, d, dtype, seed=9))
     ones = torch.ones(-(-N // BLOCK), -(-N // BLOCK), dtype=torch.bool, device=dev)
     for causal in (True, False):
         o, lse = fa2.forward(q, k, v, causal=causal)
