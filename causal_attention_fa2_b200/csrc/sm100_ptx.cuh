@@ -160,12 +160,6 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
     return p;
 }
 
-__device__ __forceinline__ uint64_t policy_evict_first() {
-    uint64_t p;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-    return p;
-}
-
 // 3-D tiled store of one box from shared memory (bulk-group completion).
 // Elements of the box outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x,
@@ -199,11 +193,6 @@ __device__ __forceinline__ void tma_store_wait_all() {
 
 __device__ __forceinline__ void tma_store_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-
-// Wait until at most one committed bulk group still has to read its source.
-__device__ __forceinline__ void tma_store_wait_read_1() {
-    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy
@@ -398,15 +387,6 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t fmt, uint32_t M, uint
                                                   bool a_mn_major, bool b_mn_major) {
     return (1u << 4) | (fmt << 7) | (fmt << 10) | ((a_mn_major ? 1u : 0u) << 15) |
            ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) | ((M >> 4) << 24);
-}
-
-// ------------------------------------------------------------------ reductions
-
-// Fire-and-forget fp32 vector add into global memory (16-byte aligned).
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-                 "f"(c), "f"(d)
-                 : "memory");
 }
 
 // ------------------------------------------------------------------ numerics
