@@ -65,7 +65,9 @@ struct Bwd32Cfg {
             if (stages_for(q_stage(w)) >= 2) return w;
         return 16;
     }
-    static constexpr int kWkv = pick_kv();
+    // At most 64 query rows per dK/dV sub-tile: with 128 (d = 16, 32) a thread's
+    // P^T row of W fp32 values spilled, and the pass ran 10 % slower, same bits.
+    static constexpr int kWkv = pick_kv() > 64 ? 64 : pick_kv();
     static constexpr int kStKV = stages_for(kv_stage(kWkv));
     static constexpr int kWq = pick_q();
     static constexpr int kStQ = stages_for(q_stage(kWq));
