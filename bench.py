@@ -47,7 +47,7 @@ L2_FLUSH_BYTES = 256 << 20
 # kernel build; None where no capture of the current build exists.
 FWD_TRAFFIC_BYTES = 209_842_944   # 186.0 MB read + 23.8 MB written
 DKDV_TRAFFIC_BYTES = 204_046_336  # 153.5 MB read + 50.5 MB written (two-pass dK/dV pass)
-DQ_TRAFFIC_BYTES = 178_731_264    # 154.2 MB read + 24.6 MB written (two-pass dQ pass)
+DQ_TRAFFIC_BYTES = 178_741_248    # 154.2 MB read + 24.5 MB written (two-pass dQ pass)
 FUSED_TRAFFIC_BYTES = None        # no capture of the one-pass backward's current build
 TRAFFIC_WORKLOAD = "10b-b1h36-n4096-d128"
 
