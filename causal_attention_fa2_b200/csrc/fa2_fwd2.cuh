@@ -83,13 +83,13 @@ struct PairRows {
 };
 
 // One softmax warpgroup: processes query tile `t` (0 = A, 1 = B) for key
-// tiles 0 .. n_kv-1, then writes its O tile and L rows.
+// tiles 0 .. n_kv-1 (block-sparse: its own n_kv set blocks), then writes its O
+// tile and L rows.
 template <int ES, int D, bool F16, bool SPARSE>
 __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_tile, int n_kv,
                                              int bh, uint32_t tmem, uint8_t* sQt,
                                              uint64_t* bar_s_full, uint64_t* bar_p_full,
-                                             uint64_t* bar_o_done, const uint16_t* kv_list,
-                                             const PairRows* pr, bool walk,
+                                             uint64_t* bar_o_done, const PairRows* pr,
                                              volatile uint32_t* abort_flag,
                                              const CUtensorMap* tm_o) {
     using Cfg = Fwd2Cfg<ES, D, F16>;
@@ -111,17 +111,11 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
     for (int j = 0; j < n_kv; ++j) {
         // Key tile of step j, and (block-sparse) whether its block is set for this
         // query tile: a step the other tile needs but this one does not is masked.
+        // (block-sparse: step j is the j-th key tile whose block is set for this
+        // query tile; the pair's other tile may take steps in between)
         int kv = j;
-        bool blk_on = true;
-        if constexpr (SPARSE) {
-            if (walk) {
-                kv = walker.at(j, p.n_tiles_k, [&](int x) { return pr->any(x); });
-                blk_on = pr->on(t, kv);
-            } else {
-                kv = kv_list[j] & 0x3FFF;
-                blk_on = (kv_list[j] >> (14 + t)) & 1;
-            }
-        }
+        const bool blk_on = true;
+        if constexpr (SPARSE) kv = walker.at(j, p.n_tiles_k, [&](int x) { return pr->on(t, x); });
         if (!ptx::mbar_wait(bar_s_full, j & 1, abort_flag, tmo)) { ok = false; break; }
         ptx::tc_fence_after();
         float s[128];
@@ -297,9 +291,9 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __shared__ volatile uint32_t abort_flag;
     // Block-sparse: the pair's key tiles, in order, with bit 14 / 15 set when
     // the block of query tile A / B is set (the first kMaxMaskTiles steps);
-    // s_cnt = steps of tile A, of the pair.
+    // s_cnt = set blocks of tile A, of tile B, of the pair.
     __shared__ uint16_t s_kv[SPARSE ? kMaxMaskTiles : 1];
-    __shared__ int s_cnt[2];
+    __shared__ int s_cnt[3];
     __shared__ PairRows s_pr;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
@@ -323,8 +317,8 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int bh_kv = kv_head_of(bh, p.H, p.H_kv, p.group);
     constexpr bool sparse = SPARSE;
     // Key tiles of the pair: those whose block is set for tile A or tile B (and,
-    // causal, at or below that tile).  Tile A visits the prefix up to its own
-    // diagonal; steps whose block is set only for B are masked for A.
+    // causal, at or below that tile).  The producer streams their union; each
+    // tile takes MMAs and softmax steps for its own set blocks only.
     if (sparse && warp == 0) {
         PairRows pr;
         const int last = p.n_tiles_k - 1;
@@ -335,15 +329,13 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (lane == 0) s_pr = pr;
         const int n_pair = warp_compact(s_kv, p.n_tiles_k, [&](int j) { return pr.any(j); },
             [&](int j) { return j | (pr.on(0, j) ? 0x4000 : 0) | (pr.on(1, j) ? 0x8000 : 0); });
-        int n_a = n_pair;
-        if (p.causal) {
-            n_a = 0;
-            for (int base = 0; base <= tile[0] && base < p.n_tiles_k; base += 32) {
-                const int j = base + lane;
-                n_a += __popc(__ballot_sync(0xffffffffu, j <= tile[0] && j < p.n_tiles_k && pr.any(j)));
-            }
+        int own[2] = {0, 0};
+        for (int base = 0; base < p.n_tiles_k; base += 32) {
+            const int j = base + lane;
+            own[0] += __popc(__ballot_sync(0xffffffffu, j < p.n_tiles_k && pr.on(0, j)));
+            own[1] += __popc(__ballot_sync(0xffffffffu, j < p.n_tiles_k && pr.on(1, j)));
         }
-        if (lane == 0) { s_cnt[0] = n_a; s_cnt[1] = n_pair; }
+        if (lane == 0) { s_cnt[0] = own[0]; s_cnt[1] = own[1]; s_cnt[2] = n_pair; }
     }
 
     if (threadIdx.x == 0) {
@@ -357,7 +349,9 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         for (int t = 0; t < 2; ++t) {
             ptx::mbar_init(&bar_s_full[t], 1);
-            ptx::mbar_init(&bar_p_full[t], 5);   // 4 softmax warps + the load watcher
+            // 4 softmax warps + the load watcher (block-sparse: the issuer checks
+            // the loads itself)
+            ptx::mbar_init(&bar_p_full[t], SPARSE ? 4 : 5);
             ptx::mbar_init(&bar_o_done[t], 1);
         }
         ptx::mbar_init(&bar_drain, 1);
@@ -372,25 +366,33 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     ptx::tc_fence_after();
     const uint32_t tmem = tmem_slot;
     const uint64_t tmo = p.timeout_ns;
-    // Key-tile steps each query tile takes (causal: key index <= query index);
-    // tile A's steps are a prefix of tile B's.
+    // Key-tile steps each query tile takes (causal: key index <= query index;
+    // dense: tile A's steps are a prefix of tile B's; block-sparse: each tile's
+    // own set blocks) and the steps the producer streams (their union).
     int n_kv_t[2];
     if (sparse) {
         n_kv_t[0] = s_cnt[0];
-        n_kv_t[1] = has_b ? s_cnt[1] : 0;
+        n_kv_t[1] = s_cnt[1];
     } else {
         n_kv_t[0] = p.causal ? min(tile[0] + 1, p.n_tiles_k) : p.n_tiles_k;
         n_kv_t[1] = has_b ? (p.causal ? min(tile[1] + 1, p.n_tiles_k) : p.n_tiles_k) : 0;
     }
-    const int n_kv = n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1];
+    const int n_kv = sparse ? s_cnt[2] : (n_kv_t[0] > n_kv_t[1] ? n_kv_t[0] : n_kv_t[1]);
     const bool load_q[2] = {n_kv_t[0] > 0, n_kv_t[1] > 0};
     // The shared-memory list holds kMaxMaskTiles steps of 14-bit key tiles;
     // beyond that each thread walks the mask rows itself.
-    const bool walk = sparse && (s_cnt[1] > kMaxMaskTiles || p.n_tiles_k > 0x4000);
+    const bool walk = sparse && (s_cnt[2] > kMaxMaskTiles || p.n_tiles_k > 0x4000);
+
     MaskWalk walker;
     auto kv_of = [&](int j) {
         if (!sparse) return j;
         return walk ? walker.at(j, p.n_tiles_k, [&](int x) { return s_pr.any(x); }) : static_cast<int>(s_kv[j] & 0x3FFF);
+    };
+    // Block-sparse: which query tiles take union step j (bit t for tile t).
+    auto step_bits = [&](int j) -> unsigned {
+        if (!walk) return (s_kv[j] >> 14) & 3u;
+        const int kv = kv_of(j);
+        return (s_pr.on(0, kv) ? 1u : 0u) | (s_pr.on(1, kv) ? 2u : 0u);
     };
 
     // Each warpgroup changes its register count inside its own branch, so the
@@ -475,11 +477,59 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mma_commit(&bar_o_done[t]);
                 return true;
             };
+            if constexpr (SPARSE) {
+                // Union step j: first the PV of each tile's previous step (step j-1,
+                // still in the V ring), then S of the tiles whose block j is set; a
+                // tile's PV always precedes its next S, which overwrites its P.  The
+                // loads are checked here (a tile may skip steps, so no P barrier
+                // covers them).
+                int local[2] = {0, 0};         // steps issued per tile
+                int pend[2] = {-1, -1};        // union step whose PV is still due
+                auto flush = [&](int t) -> bool {
+                    if (pend[t] < 0) return true;
+                    const int l = local[t] - 1, jv = pend[t];
+                    if (!ptx::mbar_wait(&bar_p_full[t], l & 1, &abort_flag, tmo)) return false;
+                    if (!ptx::mbar_wait(&bar_v_full[jv % ST], (jv / ST) & 1, &abort_flag, tmo)) return false;
+                    ptx::tc_fence_after();
+                    const uint32_t v_addr = ptx::smem_addr(sV + (jv % ST) * G::kTileBytesMN);
+#pragma unroll
+                    for (int kk = 0; kk < G::kStepsRows; ++kk) {
+                        const uint64_t b = desc_mnmajor<G>(v_addr, kk);
+                        const uint32_t acc = (l > 0 || kk > 0) ? 1u : 0u;
+                        if constexpr (G::kF32)
+                            ptx::mma_tf32_ts(tmem + Cfg::col_o(t), tmem + Cfg::col_s(t) + kk * 8, b, idesc_pv, acc);
+                        else
+                            ptx::mma_f16_ts(tmem + Cfg::col_o(t), tmem + Cfg::col_s(t) + kk * 8, b, idesc_pv, acc);
+                    }
+                    ptx::mma_commit(&bar_o_done[t]);
+                    pend[t] = -1;
+                    return true;
+                };
+                for (int j = 0; ok && j < n_kv; ++j) {
+                    const unsigned bits = step_bits(j);
+                    ok = ptx::mbar_wait(&bar_k_full[j % ST], (j / ST) & 1, &abort_flag, tmo);
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (!flush(t)) { ok = false; break; }
+                        if ((bits >> t) & 1u) {
+                            ptx::tc_fence_after();
+                            issue_s(t, j);
+                            pend[t] = j;
+                            ++local[t];
+                        }
+                    }
+                    if (!ok) break;
+                    ptx::mma_commit(&bar_k_empty[j % ST]);
+                    if (j > 0) ptx::mma_commit(&bar_v_empty[(j - 1) % ST]);
+                }
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (!flush(t)) ok = false;
+                if (ok) ptx::mma_commit(&bar_v_empty[(n_kv - 1) % ST]);
+            } else {
             // Prologue: S_A(0), S_B(0).
             if (ok) ok = ptx::mbar_wait(&bar_k_full[0], 0, &abort_flag, tmo);
             if (ok) {
                 ptx::tc_fence_after();
-                if (!SPARSE || n_kv_t[0] > 0) issue_s(0, 0);
+                issue_s(0, 0);
                 if (n_kv_t[1] > 0) issue_s(1, 0);
                 ptx::mma_commit(&bar_k_empty[0]);
             }
@@ -500,6 +550,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 ptx::mma_commit(&bar_v_empty[j % ST]);
                 if (j + 1 < n_kv) ptx::mma_commit(&bar_k_empty[(j + 1) % ST]);
             }
+            }
             if (!ok) {
                 ptx::mma_commit(&bar_drain);
                 ptx::mbar_wait_drain(&bar_drain, 0, 20000000ull);
@@ -512,7 +563,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // fifth arrival to P_t(j)'s barrier, so that the issuer's wait on P
         // covers the loads too.  Off every critical path: it runs ahead of the
         // softmax groups by up to one phase.
-        if (lane == 0 && (!SPARSE || n_kv > 0)) {
+        if (lane == 0 && !SPARSE) {
             bool ok = true;
             for (int j = 0; ok && j < n_kv; ++j) {
                 for (int t = 0; t < 2 && ok; ++t) {
@@ -533,8 +584,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Every existing query tile writes O and L, also one without key steps.
         if (SPARSE ? tile[t] < p.n_tiles : n_kv_t[t] > 0) {
             fwd2_softmax<ES, D, F16, SPARSE>(p, t, tile[t], n_kv_t[t], bh, tmem, sQ[t], &bar_s_full[t],
-                                &bar_p_full[t], &bar_o_done[t], s_kv, &s_pr, walk,
-                                &abort_flag, &tm_o);
+                                &bar_p_full[t], &bar_o_done[t], &s_pr, &abort_flag, &tm_o);
         }
     }
 
