@@ -197,9 +197,10 @@ fa2_status make_maps_kmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, in
 }
 
 template <int ES, int D>
-fa2_status make_maps_mnmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int N, int BH) {
+fa2_status make_maps_mnmajor(CUtensorMap* m, const void* ptr, fa2_dtype dtype, int N, int BH,
+                             int box_rows = kTileRows) {
     using G = TileGeom<ES, D>;
-    return make_map(m, ptr, dtype, D, N, BH, G::kBoxMN, G::kRowBMN, G::kF32);
+    return make_map(m, ptr, dtype, D, N, BH, G::kBoxMN, G::kRowBMN, G::kF32, box_rows);
 }
 
 // The dynamic shared memory limit of a kernel is raised once per device.
@@ -239,7 +240,9 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     fa2_status st;
     if ((st = make_maps_kmajor<ES, D>(&mq, q, dtype, N, BH)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mk, k, dtype, Nk, BH_kv)) != FA2_OK) return st;
-    if ((st = make_maps_mnmajor<ES, D>(&mv, v, dtype, Nk, BH_kv)) != FA2_OK) return st;
+    // V in the one-tile kernel arrives in parts of kVPartRows keys.
+    constexpr int v_rows = use_two_tile_forward<ES, D>() ? kTileRows : Cfg::kVPartRows;
+    if ((st = make_maps_mnmajor<ES, D>(&mv, v, dtype, Nk, BH_kv, v_rows)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mo, o, dtype, N, BH)) != FA2_OK) return st;
     FwdParams p;
     p.lse = lse;

@@ -87,15 +87,32 @@ struct FwdCfg {
         1024 + G::kTileBytesK * (1 + kKSt) + G::kTileBytesMN * kVSt;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kOCol = 256;
+    // fp32 when only one K stage fits (d = 128): K and V move through their
+    // rings in parts, each with its own full / ready / empty barriers (K: one
+    // 32-column box; V: four quarters of 32 keys), so a part is loaded, rounded and
+    // fed to its MMAs while the next one is still on its way; whole-tile
+    // hand-offs left the tensor pipe idle while each 64 KB tile was loaded and
+    // rounded.  With two or more stages (d <= 80) the parts' extra waits cost
+    // more than they overlap (measured 16 % slower at d = 64).
+    static constexpr bool kParted = kRoundSplit && kKSt == 1;
+    static constexpr int kKParts = kParted ? G::kNBoxK : 1;
+    static constexpr int kVParts = kParted ? 4 : 1;   // 4 measured 3-4 % faster than 2, 7 % than 1
+    static constexpr int kKPartBytes = G::kTileBytesK / kKParts;
+    static constexpr int kVPartBytes = G::kTileBytesMN / kVParts;
+    static constexpr int kVPartRows = kTileRows / kVParts;
+    static constexpr int kKStepsPart = kParted ? G::kBoxK / G::kKStep : G::kStepsD;  // QK^T steps per K part
+    static constexpr int kVStepsPart = G::kStepsRows / kVParts;                          // PV steps per V part
+    static_assert(kKParts * kKStepsPart >= G::kStepsD, "K parts miss a contraction step");
+    static_assert(kVParts * kVStepsPart == G::kStepsRows, "V parts miss a contraction step");
 };
 
 // Rounds BYTES bytes of fp32 values in shared memory to TF32 in place (one
 // warp), then makes the writes visible to the tensor core's operand reads.
-// Tiles of 32 KB and more go in batches of eight 16-byte loads per lane, so
-// the warp runs near shared-memory bandwidth instead of one load latency per
-// vector; smaller tiles keep the plain strided loop (the batched form, and a
-// fully unrolled one, measured 10-40 % slower at d <= 32).
-template <int BYTES>
+// BATCHED (fp32, d >= 64): batches of eight 16-byte loads per lane, so the
+// warp runs near shared-memory bandwidth instead of one load latency per
+// vector; otherwise the plain strided loop (the batched form, and a fully
+// unrolled one, measured 10-40 % slower at d <= 32).
+template <int BYTES, bool BATCHED>
 __device__ __forceinline__ void round_tf32_smem(uint8_t* base, int lane) {
     float4* p4 = reinterpret_cast<float4*>(base);
     auto rna = [](float4 x) {
@@ -105,7 +122,7 @@ __device__ __forceinline__ void round_tf32_smem(uint8_t* base, int lane) {
         x.w = __uint_as_float(ptx::to_tf32_rna(x.w));
         return x;
     };
-    if constexpr (BYTES >= 32768) {
+    if constexpr (BATCHED) {
         constexpr int kUnroll = 8;
         static_assert(BYTES % (16 * 32 * kUnroll) == 0, "tile not a whole number of rounding batches");
 #pragma unroll 1
@@ -136,14 +153,18 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     using G = typename Cfg::G;
     constexpr int KST = Cfg::kKSt;
     constexpr int VST = Cfg::kVSt;
+    constexpr int KP = Cfg::kKParts;
+    constexpr int VP = Cfg::kVParts;
+    constexpr int KS = KST * KP;       // K part slots: part b of stage ks is slot ks * KP + b
+    constexpr int VS = VST * VP;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_q_full;
-    __shared__ uint64_t bar_k_full[KST], bar_k_empty[KST];
-    __shared__ uint64_t bar_v_full[VST], bar_v_empty[VST];
+    __shared__ uint64_t bar_k_full[KS], bar_k_empty[KS];
+    __shared__ uint64_t bar_v_full[VS], bar_v_empty[VS];
     __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done, bar_drain;
     // fp32: tiles released by the rounding warp (the MMA issuer waits on these).
-    __shared__ uint64_t bar_q_ready, bar_k_ready[KST], bar_v_ready[VST];
+    __shared__ uint64_t bar_q_ready, bar_k_ready[KS], bar_v_ready[VS];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     __shared__ int s_cnt;                      // block-sparse: key tiles of this query tile
@@ -183,12 +204,12 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (threadIdx.x == 0) {
         abort_flag = 0u;
         ptx::mbar_init(&bar_q_full, 1);
-        for (int s = 0; s < KST; ++s) { ptx::mbar_init(&bar_k_full[s], 1); ptx::mbar_init(&bar_k_empty[s], 1); }
-        for (int s = 0; s < VST; ++s) { ptx::mbar_init(&bar_v_full[s], 1); ptx::mbar_init(&bar_v_empty[s], 1); }
+        for (int s = 0; s < KS; ++s) { ptx::mbar_init(&bar_k_full[s], 1); ptx::mbar_init(&bar_k_empty[s], 1); }
+        for (int s = 0; s < VS; ++s) { ptx::mbar_init(&bar_v_full[s], 1); ptx::mbar_init(&bar_v_empty[s], 1); }
         for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bar_s_full[b], 1); ptx::mbar_init(&bar_p_full[b], 4); }
         ptx::mbar_init(&bar_q_ready, 1);
-        for (int s = 0; s < KST; ++s) ptx::mbar_init(&bar_k_ready[s], 1);
-        for (int s = 0; s < VST; ++s) ptx::mbar_init(&bar_v_ready[s], 1);
+        for (int s = 0; s < KS; ++s) ptx::mbar_init(&bar_k_ready[s], 1);
+        for (int s = 0; s < VS; ++s) ptx::mbar_init(&bar_v_ready[s], 1);
         ptx::mbar_init(&bar_o_done, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::fence_mbar_init();
@@ -217,31 +238,59 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::mbar_arrive_expect_tx(&bar_q_full, G::kTileBytesK);
             for (int b = 0; b < G::kNBoxK; ++b)
                 ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full, b * G::kBoxK, q_row0, bh);
-            int k_issued = 0, v_issued = 0;
-            for (int j = 0; j < n_kv; ++j) {
-                const int ks = j % KST;
-                if (j >= KST && !ptx::mbar_wait(&bar_k_empty[ks], ((j / KST) & 1) ^ 1, &abort_flag, tmo)) break;
-                uint8_t* dk = sK + ks * G::kTileBytesK;
-                ptx::mbar_arrive_expect_tx(&bar_k_full[ks], G::kTileBytesK);
-                for (int b = 0; b < G::kNBoxK; ++b)
-                    ptx::tma_load_3d(dk + b * kTileRows * G::kRowBK, &tm_k, &bar_k_full[ks], b * G::kBoxK, kv_of(j) * kTileRows, bh_kv);
-                k_issued = j + 1;
-                const int vs = j % VST;
-                if (j >= VST && !ptx::mbar_wait(&bar_v_empty[vs], ((j / VST) & 1) ^ 1, &abort_flag, tmo)) break;
-                uint8_t* dv = sV + vs * G::kTileBytesMN;
-                ptx::mbar_arrive_expect_tx(&bar_v_full[vs], G::kTileBytesMN);
-                for (int b = 0; b < G::kNBoxMN; ++b)
-                    ptx::tma_load_3d(dv + b * kTileRows * G::kRowBMN, &tm_v, &bar_v_full[vs], b * G::kBoxMN, kv_of(j) * kTileRows, bh_kv);
-                v_issued = j + 1;
+            // K parts and V parts are issued as their slots free up, each ring on
+            // its own (a V slot still in use does not hold back the next K part).
+            MaskWalk walk_k, walk_v;
+            const int k_tot = n_kv * KP, v_tot = n_kv * VP;
+            int kn = 0, vn = 0;                     // parts issued
+            uint32_t spins = 0;
+            uint64_t t_idle = 0;
+            while (kn < k_tot || vn < v_tot) {
+                bool moved = false;
+                if (kn < k_tot) {
+                    const int j = kn / KP, b = kn - j * KP, sl = (j % KST) * KP + b;
+                    if (j < KST || ptx::mbar_test_wait(&bar_k_empty[sl], ((j / KST) & 1) ^ 1)) {
+                        const int kv = SPARSE ? walk_k.at(j, n_kv_lim, blk_set) : j;
+                        uint8_t* dk = sK + (j % KST) * G::kTileBytesK;
+                        constexpr int kBoxes = G::kNBoxK / KP;
+                        ptx::mbar_arrive_expect_tx(&bar_k_full[sl], Cfg::kKPartBytes);
+                        for (int bb = b * kBoxes; bb < (b + 1) * kBoxes; ++bb)
+                            ptx::tma_load_3d(dk + bb * kTileRows * G::kRowBK, &tm_k, &bar_k_full[sl], bb * G::kBoxK, kv * kTileRows, bh_kv);
+                        ++kn;
+                        moved = true;
+                    }
+                }
+                if (vn < v_tot) {
+                    const int j = vn / VP, h = vn - j * VP, sl = (j % VST) * VP + h;
+                    if (j < VST || ptx::mbar_test_wait(&bar_v_empty[sl], ((j / VST) & 1) ^ 1)) {
+                        const int kv = SPARSE ? walk_v.at(j, n_kv_lim, blk_set) : j;
+                        uint8_t* dv = sV + (j % VST) * G::kTileBytesMN + h * Cfg::kVPartBytes;
+                        ptx::mbar_arrive_expect_tx(&bar_v_full[sl], Cfg::kVPartBytes);
+                        for (int c = 0; c < G::kNBoxMN; ++c)
+                            ptx::tma_load_3d(dv + c * Cfg::kVPartRows * G::kRowBMN, &tm_v, &bar_v_full[sl], c * G::kBoxMN,
+                                             kv * kTileRows + h * Cfg::kVPartRows, bh_kv);
+                        ++vn;
+                        moved = true;
+                    }
+                }
+                if (moved) {
+                    spins = 0;
+                } else if (spins++ == 0) {
+                    t_idle = ptx::globaltimer_ns();
+                } else if ((spins & 63u) == 0) {
+                    // Bounded, as every wait here: give up on abort or after the timeout.
+                    if (abort_flag) break;
+                    if (ptx::globaltimer_ns() - t_idle > tmo) { abort_flag = 1u; break; }
+                }
             }
             if (abort_flag) {
                 // Let copies already in flight land before the CTA exits.
                 constexpr uint64_t kDrainNs = 20000000ull;
                 ptx::mbar_wait_drain(&bar_q_full, 0, kDrainNs);
-                for (int t = k_issued - 1; t >= 0 && t >= k_issued - KST; --t)
-                    ptx::mbar_wait_drain(&bar_k_full[t % KST], (t / KST) & 1, kDrainNs);
-                for (int t = v_issued - 1; t >= 0 && t >= v_issued - VST; --t)
-                    ptx::mbar_wait_drain(&bar_v_full[t % VST], (t / VST) & 1, kDrainNs);
+                for (int t = kn - 1; t >= 0 && t >= kn - KS; --t)
+                    ptx::mbar_wait_drain(&bar_k_full[((t / KP) % KST) * KP + t % KP], ((t / KP) / KST) & 1, kDrainNs);
+                for (int t = vn - 1; t >= 0 && t >= vn - VS; --t)
+                    ptx::mbar_wait_drain(&bar_v_full[((t / VP) % VST) * VP + t % VP], ((t / VP) / VST) & 1, kDrainNs);
             }
         }
     } else if (warp == 1) {
@@ -254,39 +303,50 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             auto issue_pv = [&](int jj) -> bool {
                 if (!ptx::mbar_wait(&bar_p_full[jj & 1], (jj >> 1) & 1, &abort_flag, tmo)) return false;
                 const int vs = jj % VST;
-                if (!ptx::mbar_wait(&v_go[vs], (jj / VST) & 1, &abort_flag, tmo)) return false;
-                ptx::tc_fence_after();
-                const uint32_t v_addr = ptx::smem_addr(sV + vs * G::kTileBytesMN);
                 const uint32_t p_tmem = tmem + (jj & 1) * 128;
+                for (int h = 0; h < VP; ++h) {
+                    const int sl = vs * VP + h;
+                    if (!ptx::mbar_wait(&v_go[sl], (jj / VST) & 1, &abort_flag, tmo)) return false;
+                    ptx::tc_fence_after();
+                    const uint32_t v_addr = ptx::smem_addr(sV + vs * G::kTileBytesMN + h * Cfg::kVPartBytes);
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsRows; ++kk) {
-                    const uint64_t bdesc = desc_mnmajor<G>(v_addr, kk);
-                    if constexpr (G::kF32)
-                        ptx::mma_tf32_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                    else
-                        ptx::mma_f16_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    for (int k2 = 0; k2 < Cfg::kVStepsPart; ++k2) {
+                        const int kk = h * Cfg::kVStepsPart + k2;
+                        const uint64_t bdesc = desc_mnmajor<G>(v_addr, k2, Cfg::kVPartRows);
+                        if constexpr (G::kF32)
+                            ptx::mma_tf32_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                        else
+                            ptx::mma_f16_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    ptx::mma_commit(&bar_v_empty[sl]);
                 }
                 ptx::mma_commit(&bar_o_done);
-                ptx::mma_commit(&bar_v_empty[vs]);
                 return true;
             };
             for (int j = 0; ok && j < n_kv; ++j) {
                 const int ks = j % KST;
-                if (!ptx::mbar_wait(&k_go[ks], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                ptx::tc_fence_after();
                 const uint32_t k_addr = ptx::smem_addr(sK + ks * G::kTileBytesK);
                 const uint32_t s_tmem = tmem + (j & 1) * 128;
+                for (int b = 0; b < KP; ++b) {
+                    const int sl = ks * KP + b;
+                    if (!ptx::mbar_wait(&k_go[sl], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                    ptx::tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk) {
-                    const uint64_t adesc = desc_kmajor<G>(q_addr, kk);
-                    const uint64_t bdesc = desc_kmajor<G>(k_addr, kk);
-                    if constexpr (G::kF32)
-                        ptx::mma_tf32_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-                    else
-                        ptx::mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                    for (int k2 = 0; k2 < Cfg::kKStepsPart; ++k2) {
+                        const int kk = b * Cfg::kKStepsPart + k2;
+                        if (kk < G::kStepsD) {
+                            const uint64_t adesc = desc_kmajor<G>(q_addr, kk);
+                            const uint64_t bdesc = desc_kmajor<G>(k_addr, kk);
+                            if constexpr (G::kF32)
+                                ptx::mma_tf32_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                            else
+                                ptx::mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                    }
+                    ptx::mma_commit(&bar_k_empty[sl]);
                 }
+                if (!ok) break;
                 ptx::mma_commit(&bar_s_full[j & 1]);
-                ptx::mma_commit(&bar_k_empty[ks]);
                 if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
             }
             if (ok) ok = issue_pv(n_kv - 1);
@@ -446,31 +506,37 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
         // ------------------------------------------------ TF32 rounding (fp32 only)
         if constexpr (G::kF32) {
-            // warp 6: Q and the K tiles (and the V tiles unless warp 7 has them).
+            // warp 6: Q and the K parts (and the V tiles unless warp 7 has them).
+            constexpr bool kB = Cfg::kRoundSplit;
             if (warp == 6) {
                 bool ok = n_kv > 0 && ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
                 if (ok) {
-                    round_tf32_smem<G::kTileBytesK>(sQ, lane);
+                    round_tf32_smem<G::kTileBytesK, kB>(sQ, lane);
                     if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
                 }
                 for (int j = 0; ok && j < n_kv; ++j) {
                     const int ks = j % KST;
-                    if (!ptx::mbar_wait(&bar_k_full[ks], (j / KST) & 1, &abort_flag, tmo)) break;
-                    round_tf32_smem<G::kTileBytesK>(sK + ks * G::kTileBytesK, lane);
-                    if (lane == 0) ptx::mbar_arrive(&bar_k_ready[ks]);
+                    for (int b = 0; ok && b < KP; ++b) {
+                        if (!ptx::mbar_wait(&bar_k_full[ks * KP + b], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                        round_tf32_smem<Cfg::kKPartBytes, kB>(sK + ks * G::kTileBytesK + b * Cfg::kKPartBytes, lane);
+                        if (lane == 0) ptx::mbar_arrive(&bar_k_ready[ks * KP + b]);
+                    }
                     if constexpr (!Cfg::kRoundSplit) {
                         const int vs = j % VST;
-                        if (!ptx::mbar_wait(&bar_v_full[vs], (j / VST) & 1, &abort_flag, tmo)) break;
-                        round_tf32_smem<G::kTileBytesMN>(sV + vs * G::kTileBytesMN, lane);
+                        if (!ok || !ptx::mbar_wait(&bar_v_full[vs], (j / VST) & 1, &abort_flag, tmo)) break;
+                        round_tf32_smem<G::kTileBytesMN, kB>(sV + vs * G::kTileBytesMN, lane);
                         if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs]);
                     }
                 }
             } else if constexpr (Cfg::kRoundSplit) {
-                for (int j = 0; j < n_kv; ++j) {
+                bool ok = true;
+                for (int j = 0; ok && j < n_kv; ++j) {
                     const int vs = j % VST;
-                    if (!ptx::mbar_wait(&bar_v_full[vs], (j / VST) & 1, &abort_flag, tmo)) break;
-                    round_tf32_smem<G::kTileBytesMN>(sV + vs * G::kTileBytesMN, lane);
-                    if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs]);
+                    for (int h = 0; h < VP; ++h) {
+                        if (!ptx::mbar_wait(&bar_v_full[vs * VP + h], (j / VST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                        round_tf32_smem<Cfg::kVPartBytes, kB>(sV + vs * G::kTileBytesMN + h * Cfg::kVPartBytes, lane);
+                        if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs * VP + h]);
+                    }
                 }
             }
         }
