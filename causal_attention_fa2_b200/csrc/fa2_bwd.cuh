@@ -197,6 +197,7 @@ struct BwdParams {
     float* part;           // fp32 partial dK, dV when kv_splits > 1
     int item0;             // dQ pass: work item of the first CTA (a launch may cover a suffix)
     int head_group;        // heads (dK/dV pass: key/value heads x splits) per group of work items
+    const float* k32;      // fp32 dK/dV pass at d = 128: TF32-rounded K, [BH_kv][Nk][D]
 };
 
 template <int ES, int D, bool F16 = false>

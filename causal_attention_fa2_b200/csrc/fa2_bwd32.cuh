@@ -47,8 +47,15 @@ struct Bwd32Cfg {
     __host__ __device__ static constexpr int tile_k(int rows) { return G::kNBoxK * rows * G::kRowBK; }
     __host__ __device__ static constexpr int tile_mn(int rows) { return G::kNBoxMN * rows * G::kRowBMN; }
     static constexpr int kResident = 2 * tile_k(kTileRows);
-    __host__ __device__ static constexpr int stages_for(int stage_bytes) {
-        const int s = (kBudget - kResident) / stage_bytes;
+    // dK/dV pass at d = 128: K sits in tensor memory (the S^T = K Q^T MMA reads
+    // its A operand there), so only V is resident in shared memory and the
+    // streamed query rows come in sub-tiles of 32 rows instead of 16.  The pass
+    // is bound by the tcgen05 pipe, and the narrow S^T / dP^T MMAs (N = W) are
+    // most of its instructions: W = 32 halves them per query row.
+    static constexpr bool kKInTmem = (D == 128);
+    static constexpr int kResidentKV = (kKInTmem ? 1 : 2) * tile_k(kTileRows);
+    __host__ __device__ static constexpr int stages_for(int stage_bytes, int resident = kResident) {
+        const int s = (kBudget - resident) / stage_bytes;
         return s > 4 ? 4 : s;
     }
     // dK/dV pass, per stage: W query rows of Q and of dO, each K-major and MN-major.
@@ -57,7 +64,7 @@ struct Bwd32Cfg {
     __host__ __device__ static constexpr int q_stage(int w) { return 2 * tile_k(w) + tile_mn(w); }
     __host__ __device__ static constexpr int pick_kv() {
         for (int w = kTileRows; w > 16; w /= 2)
-            if (stages_for(kv_stage(w)) >= 2) return w;
+            if (stages_for(kv_stage(w), kResidentKV) >= 2) return w;
         return 16;
     }
     __host__ __device__ static constexpr int pick_q() {
@@ -68,15 +75,18 @@ struct Bwd32Cfg {
     // At most 64 query rows per dK/dV sub-tile: with 128 (d = 16, 32) a thread's
     // P^T row of W fp32 values spilled, and the pass ran 10 % slower, same bits.
     static constexpr int kWkv = pick_kv() > 64 ? 64 : pick_kv();
-    static constexpr int kStKV = stages_for(kv_stage(kWkv));
+    static constexpr int kStKV = stages_for(kv_stage(kWkv), kResidentKV);
     static constexpr int kWq = pick_q();
     static constexpr int kStQ = stages_for(q_stage(kWq));
     static_assert(kStKV >= 2 && kStQ >= 2, "shared memory too small for two pipeline stages");
-    static constexpr int kSmemKV = 1024 + kResident + kStKV * kv_stage(kWkv);
+    static constexpr int kSmemKV = 1024 + kResidentKV + kStKV * kv_stage(kWkv);
     static constexpr int kSmemQ = 1024 + kResident + kStQ * q_stage(kWq);
     static constexpr uint32_t kTmemCols = 512;
     // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
+    // dK/dV pass with K in tensor memory: S^T | dP^T | K | dV | dK.
+    static constexpr uint32_t kColDPkv = kKInTmem ? 64 : kColDP, kColKT = 128;
+    static_assert(!kKInTmem || kWkv <= 64, "S^T and dP^T must fit below the K columns");
 };
 
 // ------------------------------------------------------------------ pre-processing
@@ -255,15 +265,19 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full, bar_full[ST], bar_empty[ST];
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_dkv_full, bar_drain;
+    __shared__ uint64_t bar_kt_ready;                   // K written to tensor memory (KT)
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     __shared__ int s_cnt;                               // block-sparse: query sub-tiles per head
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* sK = smem;
-    uint8_t* sV = sK + TK;
+    constexpr bool KT = Cfg::kKInTmem;
+    uint8_t* sK = smem;                                 // unused when K is in tensor memory
+    uint8_t* sV = KT ? smem : sK + TK;
     uint8_t* sStage = sV + TK;
+    // dK is staged for its store where K was, or in the (then idle) first stage.
+    uint8_t* sDK = KT ? sStage : sK;
     // Stage s: Q (K-major) | dO (K-major) | Q (MN-major) | dO (MN-major).
     auto st_qk = [&](int s) { return sStage + s * SB; };
     auto st_dok = [&](int s) { return sStage + s * SB + SK; };
@@ -313,6 +327,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         ptx::mbar_init(&bar_ds_ready, 4);
         ptx::mbar_init(&bar_dkv_full, 1);
         ptx::mbar_init(&bar_drain, 1);
+        ptx::mbar_init(&bar_kt_ready, 4);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -343,9 +358,9 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             ptx::prefetch_tmap(&tm_qmn);
             ptx::prefetch_tmap(&tm_dok);
             ptx::prefetch_tmap(&tm_domn);
-            ptx::mbar_arrive_expect_tx(&bar_kv_full, 2 * TK);
+            ptx::mbar_arrive_expect_tx(&bar_kv_full, (KT ? 1 : 2) * TK);
             for (int b = 0; b < G::kNBoxK; ++b) {
-                ptx::tma_load_3d(sK + b * kTileRows * G::kRowBK, &tm_k, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
+                if (!KT) ptx::tma_load_3d(sK + b * kTileRows * G::kRowBK, &tm_k, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
                 ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
             }
             int issued = 0;
@@ -386,8 +401,12 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 ptx::tc_fence_after();
                 const uint32_t qa = ptx::smem_addr(st_qk(s));
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < G::kStepsD; ++kk) {
+                    if constexpr (KT)
+                        ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColKT + kk * G::kKStep, desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                }
                 ptx::mma_commit(&bar_s_full);
                 return true;
             };
@@ -396,10 +415,11 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 const uint32_t da = ptx::smem_addr(st_dok(it % ST));
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                    ptx::mma_tf32_ss(tmem + Cfg::kColDPkv, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 ptx::mma_commit(&bar_dp_full);
             };
             bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
+            if (KT && ok) ok = ptx::mbar_wait(&bar_kt_ready, 0, &abort_flag, tmo);
             if (ok) ok = issue_s(0);
             if (ok) issue_dp(0);
             for (int it = 0; ok && it < n_it; ++it) {
@@ -418,7 +438,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 const uint32_t qmn = ptx::smem_addr(st_qmn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDP + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPkv + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_empty[s]);
                 if (it + 1 < n_it) issue_dp(it + 1);
             }
@@ -437,6 +457,30 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
         const float sl2 = p.scale_log2;
         bool ok = true;
+        if constexpr (KT) {
+            // K row r (TF32-rounded copy) into tensor memory; zeros past Nk.
+            if (n_it > 0) {
+                const float4* krow = reinterpret_cast<const float4*>(
+                    p.k32 + (static_cast<size_t>(bh) * p.Nk + (key_valid ? kv_row0 + r : 0)) * D);
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 x = key_valid ? __ldg(krow + c0 / 4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        u[4 * q4 + 0] = __float_as_uint(x.x);
+                        u[4 * q4 + 1] = __float_as_uint(x.y);
+                        u[4 * q4 + 2] = __float_as_uint(x.z);
+                        u[4 * q4 + 3] = __float_as_uint(x.w);
+                    }
+                    ptx::tmem_st32(lane_base + Cfg::kColKT + c0, u);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_kt_ready);
+            }
+        }
         for (int it = 0; it < n_it; ++it) {
             const int q0 = q_row_of(it);
             const size_t qv = static_cast<size_t>(q_head_of(it)) * p.n_pad + q0;
@@ -469,7 +513,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             // ---- dS^T = P^T o (dP^T - D)   (Eq. 17), in place over dP^T
             if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            bwd32_ds_inplace<W>(lane_base + Cfg::kColDP, pu, [&](int c) { return __ldg(dvq + c); });
+            bwd32_ds_inplace<W>(lane_base + Cfg::kColDPkv, pu, [&](int c) { return __ldg(dvq + c); });
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
@@ -479,14 +523,14 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         if (ok) {
             ptx::tc_fence_after();
             bwd32_stage_rows<G>(lane_base + Cfg::kColDV, r, 1.f, sV, n_it == 0);
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sK, n_it == 0);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sDK, n_it == 0);
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (ok && threadIdx.x == 64) {
             for (int bx = 0; bx < G::kNBoxK; ++bx) {
                 ptx::tma_store_3d(&tm_dv, sV + bx * kTileRows * G::kRowBK, bx * G::kBoxK, kv_row0, bh);
-                ptx::tma_store_3d(&tm_dk, sK + bx * kTileRows * G::kRowBK, bx * G::kBoxK, kv_row0, bh);
+                ptx::tma_store_3d(&tm_dk, sDK + bx * kTileRows * G::kRowBK, bx * G::kBoxK, kv_row0, bh);
             }
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
