@@ -334,7 +334,7 @@ fa2_status launch_backward_t(const void* q, const void* k, const void* v, const 
     if ((st = make_maps_kmajor<ES, D>(&mdv, dv, dtype, Nk, BH_kv)) != FA2_OK) return st;
     if ((st = make_maps_kmajor<ES, D>(&mdq, dq, dtype, N, BH)) != FA2_OK) return st;
     BwdParams p;
-    p.k32 = nullptr;
+    p.k32 = p.q32 = p.do32 = nullptr;
     p.l2 = l2;
     p.dvec = dvec;
     p.status = status;
@@ -492,6 +492,8 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
     p.block_mask = block_mask;
     p.kv_splits = 1;                                     // fp32: one CTA per group
     p.k32 = kr;
+    p.q32 = qr;
+    p.do32 = dor;
     p.part = nullptr;
     p.item0 = 0;
     p.head_group = 1;

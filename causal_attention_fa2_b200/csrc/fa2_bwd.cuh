@@ -198,6 +198,8 @@ struct BwdParams {
     int item0;             // dQ pass: work item of the first CTA (a launch may cover a suffix)
     int head_group;        // heads (dK/dV pass: key/value heads x splits) per group of work items
     const float* k32;      // fp32 dK/dV pass at d = 128: TF32-rounded K, [BH_kv][Nk][D]
+    const float* q32;      // fp32 dQ pass at d = 128: TF32-rounded Q and dO, [BH][N][D]
+    const float* do32;
 };
 
 template <int ES, int D, bool F16 = false>

@@ -54,6 +54,11 @@ struct Bwd32Cfg {
     // most of its instructions: W = 32 halves them per query row.
     static constexpr bool kKInTmem = (D == 128);
     static constexpr int kResidentKV = (kKInTmem ? 1 : 2) * tile_k(kTileRows);
+    // dQ pass at d = 128, likewise: Q and dO in tensor memory (the A operands of
+    // S = Q K^T and dP = dO V^T), nothing resident in shared memory, and key
+    // sub-tiles of 64 rows instead of 32.
+    static constexpr bool kQInTmem = (D == 128);
+    static constexpr int kResidentQ = kQInTmem ? 0 : 2 * tile_k(kTileRows);
     __host__ __device__ static constexpr int stages_for(int stage_bytes, int resident = kResident) {
         const int s = (kBudget - resident) / stage_bytes;
         return s > 4 ? 4 : s;
@@ -69,7 +74,7 @@ struct Bwd32Cfg {
     }
     __host__ __device__ static constexpr int pick_q() {
         for (int w = kTileRows; w > 16; w /= 2)
-            if (stages_for(q_stage(w)) >= 2) return w;
+            if (stages_for(q_stage(w), kResidentQ) >= 2) return w;
         return 16;
     }
     // At most 64 query rows per dK/dV sub-tile: with 128 (d = 16, 32) a thread's
@@ -77,16 +82,20 @@ struct Bwd32Cfg {
     static constexpr int kWkv = pick_kv() > 64 ? 64 : pick_kv();
     static constexpr int kStKV = stages_for(kv_stage(kWkv), kResidentKV);
     static constexpr int kWq = pick_q();
-    static constexpr int kStQ = stages_for(q_stage(kWq));
+    static constexpr int kStQ = stages_for(q_stage(kWq), kResidentQ);
     static_assert(kStKV >= 2 && kStQ >= 2, "shared memory too small for two pipeline stages");
     static constexpr int kSmemKV = 1024 + kResidentKV + kStKV * kv_stage(kWkv);
-    static constexpr int kSmemQ = 1024 + kResident + kStQ * q_stage(kWq);
+    static constexpr int kSmemQ = 1024 + kResidentQ + kStQ * q_stage(kWq);
     static constexpr uint32_t kTmemCols = 512;
     // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
     // dK/dV pass with K in tensor memory: S^T | dP^T | K | dV | dK.
     static constexpr uint32_t kColDPkv = kKInTmem ? 64 : kColDP, kColKT = 128;
     static_assert(!kKInTmem || kWkv <= 64, "S^T and dP^T must fit below the K columns");
+    // dQ pass with Q and dO in tensor memory: S | dP | dQ | Q | dO.
+    static constexpr uint32_t kColDPq = kQInTmem ? 64 : kColDP, kColDQq = kQInTmem ? 128 : kColDQ;
+    static constexpr uint32_t kColQT = 256, kColDOT = 384;
+    static_assert(!kQInTmem || kWq <= 64, "S and dP must fit below the dQ columns");
 };
 
 // ------------------------------------------------------------------ pre-processing
@@ -575,15 +584,19 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_qdo_full, bar_full[ST], bar_empty[ST];
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready, bar_dq_done, bar_drain;
+    __shared__ uint64_t bar_qt_ready;                   // Q and dO written to tensor memory (QT)
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     __shared__ int s_cnt;                               // block-sparse: key sub-tiles
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* sQ = smem;
+    constexpr bool QT = Cfg::kQInTmem;
+    uint8_t* sQ = smem;                                 // unused when Q, dO are in tensor memory
     uint8_t* sDO = sQ + TK;
-    uint8_t* sStage = sDO + TK;
+    uint8_t* sStage = QT ? smem : sDO + TK;
+    // dQ is staged for its store where Q was, or in the (then idle) first stage.
+    uint8_t* sDQ = QT ? sStage : sQ;
     // Stage s: K (K-major) | V (K-major) | K (MN-major).
     auto st_kk = [&](int s) { return sStage + s * SB; };
     auto st_vk = [&](int s) { return sStage + s * SB + SK; };
@@ -631,6 +644,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(&bar_ds_ready, 4);
         ptx::mbar_init(&bar_dq_done, 1);
         ptx::mbar_init(&bar_drain, 1);
+        ptx::mbar_init(&bar_qt_ready, 4);
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -652,10 +666,12 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::prefetch_tmap(&tm_kmn);
             ptx::prefetch_tmap(&tm_vk);
             const uint64_t keep = ptx::policy_evict_last();
-            ptx::mbar_arrive_expect_tx(&bar_qdo_full, 2 * TK);
-            for (int b = 0; b < G::kNBoxK; ++b) {
-                ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
-                ptx::tma_load_3d(sDO + b * kTileRows * G::kRowBK, &tm_do, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
+            if (!QT) {
+                ptx::mbar_arrive_expect_tx(&bar_qdo_full, 2 * TK);
+                for (int b = 0; b < G::kNBoxK; ++b) {
+                    ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
+                    ptx::tma_load_3d(sDO + b * kTileRows * G::kRowBK, &tm_do, &bar_qdo_full, b * G::kBoxK, q_row0, bh);
+                }
             }
             int issued = 0;
             for (int j = 0; j < n_kv; ++j) {
@@ -673,7 +689,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             if (abort_flag) {
                 constexpr uint64_t kDrainNs = 20000000ull;
-                ptx::mbar_wait_drain(&bar_qdo_full, 0, kDrainNs);
+                if (!QT) ptx::mbar_wait_drain(&bar_qdo_full, 0, kDrainNs);
                 for (int t = issued - 1; t >= 0 && t >= issued - ST; --t)
                     ptx::mbar_wait_drain(&bar_full[t % ST], (t / ST) & 1, kDrainNs);
             }
@@ -692,8 +708,12 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tc_fence_after();
                 const uint32_t ka = ptx::smem_addr(st_kk(s));
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < G::kStepsD; ++kk) {
+                    if constexpr (QT)
+                        ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColQT + kk * G::kKStep, desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                }
                 ptx::mma_commit(&bar_s_full);
                 return true;
             };
@@ -701,11 +721,16 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             auto issue_dp = [&](int j) {
                 const uint32_t va = ptx::smem_addr(st_vk(j % ST));
 #pragma unroll
-                for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < G::kStepsD; ++kk) {
+                    if constexpr (QT)
+                        ptx::mma_tf32_ts(tmem + Cfg::kColDPq, tmem + Cfg::kColDOT + kk * G::kKStep, desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                    else
+                        ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                }
                 ptx::mma_commit(&bar_dp_full);
             };
-            bool ok = ptx::mbar_wait(&bar_qdo_full, 0, &abort_flag, tmo);
+            bool ok = QT ? ptx::mbar_wait(&bar_qt_ready, 0, &abort_flag, tmo)
+                         : ptx::mbar_wait(&bar_qdo_full, 0, &abort_flag, tmo);
             if (ok) ok = issue_s(0);
             if (ok) issue_dp(0);
             for (int j = 0; ok && j < n_kv; ++j) {
@@ -720,7 +745,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t kmn = ptx::smem_addr(st_kmn(j % ST));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDQ, tmem + Cfg::kColDP + kk * G::kKStep, desc_mnmajor<G>(kmn, kk, W), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDQq, tmem + Cfg::kColDPq + kk * G::kKStep, desc_mnmajor<G>(kmn, kk, W), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_empty[j % ST]);
                 if (j + 1 < n_kv) issue_dp(j + 1);
             }
@@ -741,6 +766,35 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float l2r = p.l2[vrow];                    // L_i * log2(e) (+inf past N)
         const float dr = p.dvec[vrow];                   // D_i (0 past N)
         bool ok = true;
+        if constexpr (QT) {
+            // Q and dO row r (TF32-rounded copies) into tensor memory; zeros past N.
+            if (n_kv > 0) {
+                const bool row_valid = q_row0 + r < p.N;
+                const size_t row_off = (static_cast<size_t>(bh) * p.N + (row_valid ? q_row0 + r : 0)) * D;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const float4* src = reinterpret_cast<const float4*>((t == 0 ? p.q32 : p.do32) + row_off);
+                    const uint32_t col = t == 0 ? Cfg::kColQT : Cfg::kColDOT;
+#pragma unroll
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t u[32];
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4) {
+                            const float4 x = row_valid ? __ldg(src + c0 / 4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                            u[4 * q4 + 0] = __float_as_uint(x.x);
+                            u[4 * q4 + 1] = __float_as_uint(x.y);
+                            u[4 * q4 + 2] = __float_as_uint(x.z);
+                            u[4 * q4 + 3] = __float_as_uint(x.w);
+                        }
+                        ptx::tmem_st32(lane_base + col + c0, u);
+                    }
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_qt_ready);
+            }
+        }
         for (int j = 0; j < n_kv; ++j) {
             const int k0 = kvs_of(j) * W;
             const bool mask = p.causal && k0 + W - 1 > q_row0;   // some key follows some query
@@ -763,7 +817,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
             if (!ptx::mbar_wait(&bar_dp_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            bwd32_ds_inplace<W>(lane_base + Cfg::kColDP, pu, [&](int) { return dr; });
+            bwd32_ds_inplace<W>(lane_base + Cfg::kColDPq, pu, [&](int) { return dr; });
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
@@ -773,13 +827,13 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (ok && n_kv > 0) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDQ, r, p.scale, sQ, n_kv == 0);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDQq, r, p.scale, sDQ, n_kv == 0);
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (ok && threadIdx.x == 64) {
             for (int bx = 0; bx < G::kNBoxK; ++bx)
-                ptx::tma_store_3d(&tm_dq, sQ + bx * kTileRows * G::kRowBK, bx * G::kBoxK, q_row0, bh);
+                ptx::tma_store_3d(&tm_dq, sDQ + bx * kTileRows * G::kRowBK, bx * G::kBoxK, q_row0, bh);
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
         }
