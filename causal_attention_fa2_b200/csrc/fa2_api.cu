@@ -259,6 +259,7 @@ fa2_status launch_forward(const void* q, const void* k, const void* v, void* o, 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.timeout_ns = kDefaultTimeoutNs;
     p.block_mask = block_mask;
+    p.q32 = ES == 4 ? static_cast<const float*>(q) : nullptr;
     // Two query tiles per CTA (the softmax of one overlaps the MMAs of the
     // other), unless the pairs would leave SMs idle: then one tile per CTA.
     const long long pair_items = static_cast<long long>((p.n_tiles + 1) / 2) * BH;

@@ -62,6 +62,7 @@ struct FwdParams {
     float scale_log2;      // scale * log2(e)
     unsigned long long timeout_ns;
     const uint8_t* block_mask;  // [n_tiles][n_tiles_k] block mask, or nullptr (dense)
+    const float* q32;      // fp32 inputs at d = 128: q itself, [BH][N][D] (read row by row)
     int head_group;        // two-tile forward: heads per group of work items (grouped_item)
     int one_tile;          // two-tile forward: one query tile per CTA (small grids)
 };
@@ -75,7 +76,14 @@ struct FwdCfg {
     static constexpr bool kRoundSplit = G::kF32 && D >= 64;
     static constexpr int kThreads = G::kF32 ? (kRoundSplit ? 256 : 224) : 192;
     static constexpr int kBudget = 227 * 1024 - 2048;
-    static constexpr int kFree = kBudget - G::kTileBytesK;
+    // fp32 at d = 128: Q sits in tensor memory (columns 384-511, beside the two
+    // score buffers and O), written there rounded by the softmax threads; S =
+    // Q K^T reads its A operand from TMEM, and the 64 KB of shared memory this
+    // frees gives K a second ring stage.
+    static constexpr bool kQInTmem = G::kF32 && D == 128;
+    static constexpr uint32_t kQCol = 384;
+    static constexpr int kQBytes = kQInTmem ? 0 : G::kTileBytesK;   // Q staged in shared memory
+    static constexpr int kFree = kBudget - kQBytes;
     // Ring depths for K and V (at most 4 each), as many as fit.
     static constexpr int kKV = G::kTileBytesK + G::kTileBytesMN;
     static constexpr int kPairs = kFree / kKV;
@@ -84,17 +92,17 @@ struct FwdCfg {
     static constexpr int kVSt = kKSt0;
     static_assert(kVSt >= 1, "shared memory too small for one K/V stage");
     static constexpr int kSmemBytes =
-        1024 + G::kTileBytesK * (1 + kKSt) + G::kTileBytesMN * kVSt;
+        1024 + kQBytes + G::kTileBytesK * kKSt + G::kTileBytesMN * kVSt;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kOCol = 256;
-    // fp32 when only one K stage fits (d = 128): K and V move through their
-    // rings in parts, each with its own full / ready / empty barriers (K: one
-    // 32-column box; V: four quarters of 32 keys), so a part is loaded, rounded and
-    // fed to its MMAs while the next one is still on its way; whole-tile
-    // hand-offs left the tensor pipe idle while each 64 KB tile was loaded and
-    // rounded.  With two or more stages (d <= 80) the parts' extra waits cost
-    // more than they overlap (measured 16 % slower at d = 64).
-    static constexpr bool kParted = kRoundSplit && kKSt == 1;
+    // fp32 at d = 128, where one V stage is all that fits: K and V move through
+    // their rings in parts, each with its own full / ready / empty barriers (K:
+    // one 32-column box; V: four quarters of 32 keys), so a part is loaded,
+    // rounded and fed to its MMAs while the next one is still on its way;
+    // whole-tile hand-offs left the tensor pipe idle while each 64 KB tile was
+    // loaded and rounded.  At d <= 80 the parts' extra waits cost more than they
+    // overlap (measured 16 % slower at d = 64, 15 % at d = 80).
+    static constexpr bool kParted = G::kF32 && D == 128;
     static constexpr int kKParts = kParted ? G::kNBoxK : 1;
     static constexpr int kVParts = kParted ? 4 : 1;   // 4 measured 3-4 % faster than 2, 7 % than 1
     static constexpr int kKPartBytes = G::kTileBytesK / kKParts;
@@ -174,8 +182,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t* sQ = smem;
-    uint8_t* sK = sQ + G::kTileBytesK;
+    constexpr bool QT = Cfg::kQInTmem;
+    uint8_t* sQ = smem;                        // unused when Q is in tensor memory
+    uint8_t* sK = sQ + Cfg::kQBytes;
+    // O is staged for its store in the Q slot, or in K stage 0 (idle by then).
+    uint8_t* sO = QT ? sK : sQ;
     uint8_t* sV = sK + KST * G::kTileBytesK;
 
     const int warp = threadIdx.x >> 5;
@@ -207,7 +218,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int s = 0; s < KS; ++s) { ptx::mbar_init(&bar_k_full[s], 1); ptx::mbar_init(&bar_k_empty[s], 1); }
         for (int s = 0; s < VS; ++s) { ptx::mbar_init(&bar_v_full[s], 1); ptx::mbar_init(&bar_v_empty[s], 1); }
         for (int b = 0; b < 2; ++b) { ptx::mbar_init(&bar_s_full[b], 1); ptx::mbar_init(&bar_p_full[b], 4); }
-        ptx::mbar_init(&bar_q_ready, 1);
+        ptx::mbar_init(&bar_q_ready, QT ? 4 : 1);   // QT: one arrival per softmax warp
         for (int s = 0; s < KS; ++s) ptx::mbar_init(&bar_k_ready[s], 1);
         for (int s = 0; s < VS; ++s) ptx::mbar_init(&bar_v_ready[s], 1);
         ptx::mbar_init(&bar_o_done, 1);
@@ -235,9 +246,11 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::prefetch_tmap(&tm_q);
             ptx::prefetch_tmap(&tm_k);
             ptx::prefetch_tmap(&tm_v);
-            ptx::mbar_arrive_expect_tx(&bar_q_full, G::kTileBytesK);
-            for (int b = 0; b < G::kNBoxK; ++b)
-                ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full, b * G::kBoxK, q_row0, bh);
+            if (!QT) {
+                ptx::mbar_arrive_expect_tx(&bar_q_full, G::kTileBytesK);
+                for (int b = 0; b < G::kNBoxK; ++b)
+                    ptx::tma_load_3d(sQ + b * kTileRows * G::kRowBK, &tm_q, &bar_q_full, b * G::kBoxK, q_row0, bh);
+            }
             // K parts and V parts are issued as their slots free up, each ring on
             // its own (a V slot still in use does not hold back the next K part).
             MaskWalk walk_k, walk_v;
@@ -286,7 +299,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (abort_flag) {
                 // Let copies already in flight land before the CTA exits.
                 constexpr uint64_t kDrainNs = 20000000ull;
-                ptx::mbar_wait_drain(&bar_q_full, 0, kDrainNs);
+                if (!QT) ptx::mbar_wait_drain(&bar_q_full, 0, kDrainNs);
                 for (int t = kn - 1; t >= 0 && t >= kn - KS; --t)
                     ptx::mbar_wait_drain(&bar_k_full[((t / KP) % KST) * KP + t % KP], ((t / KP) / KST) & 1, kDrainNs);
                 for (int t = vn - 1; t >= 0 && t >= vn - VS; --t)
@@ -335,12 +348,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int k2 = 0; k2 < Cfg::kKStepsPart; ++k2) {
                         const int kk = b * Cfg::kKStepsPart + k2;
                         if (kk < G::kStepsD) {
-                            const uint64_t adesc = desc_kmajor<G>(q_addr, kk);
                             const uint64_t bdesc = desc_kmajor<G>(k_addr, kk);
-                            if constexpr (G::kF32)
-                                ptx::mma_tf32_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                            if constexpr (QT)
+                                ptx::mma_tf32_ts(s_tmem, tmem + Cfg::kQCol + kk * G::kKStep, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                            else if constexpr (G::kF32)
+                                ptx::mma_tf32_ss(s_tmem, desc_kmajor<G>(q_addr, kk), bdesc, idesc_qk, kk > 0 ? 1u : 0u);
                             else
-                                ptx::mma_f16_ss(s_tmem, adesc, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                                ptx::mma_f16_ss(s_tmem, desc_kmajor<G>(q_addr, kk), bdesc, idesc_qk, kk > 0 ? 1u : 0u);
                         }
                     }
                     ptx::mma_commit(&bar_k_empty[sl]);
@@ -366,6 +380,31 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         float m_ref = -INFINITY;                // reference max (log2 units)
         float l = 0.f;                          // running sum of 2^(t - m_ref)
         bool ok = true;
+        if constexpr (QT) {
+            // Query row r, rounded to TF32, into tensor memory; zeros past N.
+            if (n_kv > 0) {
+                const bool row_valid = q_row0 + r < p.N;
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.q32 + (static_cast<size_t>(bh) * p.N + (row_valid ? q_row0 + r : 0)) * D);
+#pragma unroll
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const float4 x = row_valid ? __ldg(src + c0 / 4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        u[4 * q4 + 0] = ptx::to_tf32_rna(x.x);
+                        u[4 * q4 + 1] = ptx::to_tf32_rna(x.y);
+                        u[4 * q4 + 2] = ptx::to_tf32_rna(x.z);
+                        u[4 * q4 + 3] = ptx::to_tf32_rna(x.w);
+                    }
+                    ptx::tmem_st32(lane_base + Cfg::kQCol + c0, u);
+                }
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
+            }
+        }
         for (int j = 0; j < n_kv; ++j) {
             if (!ptx::mbar_wait(&bar_s_full[j & 1], (j >> 1) & 1, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -471,7 +510,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * inv_l);
                             w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * inv_l);
                             w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * inv_l);
-                            *reinterpret_cast<uint4*>(sQ + kmajor_chunk_offset<G>(r, col)) = w;
+                            *reinterpret_cast<uint4*>(sO + kmajor_chunk_offset<G>(r, col)) = w;
                         }
                     }
                 } else {
@@ -485,7 +524,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             w.y = ptx::pack_bf16x2(f[2] * inv_l, f[3] * inv_l);
                             w.z = ptx::pack_bf16x2(f[4] * inv_l, f[5] * inv_l);
                             w.w = ptx::pack_bf16x2(f[6] * inv_l, f[7] * inv_l);
-                            *reinterpret_cast<uint4*>(sQ + kmajor_chunk_offset<G>(r, col)) = w;
+                            *reinterpret_cast<uint4*>(sO + kmajor_chunk_offset<G>(r, col)) = w;
                         }
                     }
                 }
@@ -499,7 +538,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         asm volatile("bar.sync 1, 128;" ::: "memory");
         if (ok && threadIdx.x == 64) {
             for (int b = 0; b < G::kNBoxK; ++b)
-                ptx::tma_store_3d(&tm_o, sQ + b * kTileRows * G::kRowBK, b * G::kBoxK, q_row0, bh);
+                ptx::tma_store_3d(&tm_o, sO + b * kTileRows * G::kRowBK, b * G::kBoxK, q_row0, bh);
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
         }
@@ -509,8 +548,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             // warp 6: Q and the K parts (and the V tiles unless warp 7 has them).
             constexpr bool kB = Cfg::kRoundSplit;
             if (warp == 6) {
-                bool ok = n_kv > 0 && ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
-                if (ok) {
+                bool ok = n_kv > 0 && (QT || ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo));
+                if (ok && !QT) {
                     round_tf32_smem<G::kTileBytesK, kB>(sQ, lane);
                     if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
                 }
