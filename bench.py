@@ -431,7 +431,7 @@ def main():
     args = ap.parse_args()
     if args.table:
         return run_table(args)
-    w = fa2_inputs.WORKLOADS[args.workload]
+    w = fa2_inputs.workload_by_name(args.workload)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -63,6 +63,19 @@ def sweep_workload(N: int, d: int, dtype: str) -> Workload:
     return Workload(f"sweep-b1h16-n{N}-d{d}-{dtype}", 1, 16, N, d, dtype, 1000 + N + d)
 
 
+def workload_by_name(name: str) -> Workload:
+    """A fixed workload, or a sweep point named as sweep_workload names it
+    ("sweep-b1h16-n<N>-d<d>-<dtype>")."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    parts = name.split("-")
+    if len(parts) == 5 and parts[0] == "sweep" and parts[1] == "b1h16" and parts[4] in DTYPES:
+        w = sweep_workload(int(parts[2][1:]), int(parts[3][1:]), parts[4])
+        if w.name == name:
+            return w
+    raise KeyError(f"unknown workload {name!r}")
+
+
 def sweep_workloads() -> List[Workload]:
     return [sweep_workload(N, d, dt) for dt in ("bf16", "fp32") for d in SWEEP_D for N in SWEEP_N]
 

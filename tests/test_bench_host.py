@@ -65,3 +65,13 @@ def test_single_tile_pairs(N, causal):
     k = np.arange(N)[None, :]
     brute = int(((k <= q) & (q < 128)).sum()) if causal else 0
     assert bench.single_tile_pairs(w) == 2 * 3 * brute
+
+
+def test_workload_by_name_covers_fixed_and_sweep_points():
+    for w in fa2_inputs.WORKLOADS.values():
+        assert fa2_inputs.workload_by_name(w.name) is w
+    for w in fa2_inputs.sweep_workloads():
+        assert fa2_inputs.workload_by_name(w.name) == w
+    for bad in ("sweep-b1h16-n4096-d128-int8", "sweep-b2h16-n4096-d128-fp32", "10b"):
+        with pytest.raises(KeyError):
+            fa2_inputs.workload_by_name(bad)
