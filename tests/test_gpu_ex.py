@@ -35,6 +35,9 @@ CASES = [
     (1, 2, 1, 170, 390, 32, "fp16", True),
     (1, 2, 2, 150, 400, 64, "fp32", True),
     (1, 2, 2, 260, 100, 128, "fp32", False),
+    # fp32 at d = 128 (operands in tensor memory) with grouped heads and ragged lengths
+    (1, 4, 2, 300, 257, 128, "fp32", True),
+    (1, 3, 1, 129, 300, 128, "fp32", False),
 ]
 
 
