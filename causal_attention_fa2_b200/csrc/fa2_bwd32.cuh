@@ -127,11 +127,19 @@ fa2_bwd32_pre_kernel(const float* __restrict__ q, const float* __restrict__ o,
     }
     const size_t base = (static_cast<size_t>(bh) * N + n) * D;
     float acc = 0.f;
-    for (int e = lane; e < D; e += 32) {
-        const float g = __uint_as_float(ptx::to_tf32_rna(dout[base + e]));
-        dor[base + e] = g;
-        qr[base + e] = __uint_as_float(ptx::to_tf32_rna(q[base + e]));
-        acc += o[base + e] * g;
+    // 16-byte accesses (D is a multiple of 4): a lane takes columns 4e .. 4e + 3.
+    const float4* q4 = reinterpret_cast<const float4*>(q + base);
+    const float4* o4 = reinterpret_cast<const float4*>(o + base);
+    const float4* g4 = reinterpret_cast<const float4*>(dout + base);
+    float4* qr4 = reinterpret_cast<float4*>(qr + base);
+    float4* dor4 = reinterpret_cast<float4*>(dor + base);
+    auto rna = [](float x) { return __uint_as_float(ptx::to_tf32_rna(x)); };
+    for (int e = lane; e < D / 4; e += 32) {
+        const float4 gv = __ldg(g4 + e), qv = __ldg(q4 + e), ov = __ldg(o4 + e);
+        const float4 g = make_float4(rna(gv.x), rna(gv.y), rna(gv.z), rna(gv.w));
+        dor4[e] = g;
+        qr4[e] = make_float4(rna(qv.x), rna(qv.y), rna(qv.z), rna(qv.w));
+        acc += ov.x * g.x + ov.y * g.y + ov.z * g.z + ov.w * g.w;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
