@@ -221,12 +221,12 @@ fa2_status set_smem(Kernel k, int bytes) {
     return FA2_OK;
 }
 
-// The two-query-tile forward serves 16-bit inputs.  fp32 (TF32) inputs use the
-// one-tile kernel, whose extra warp rounds every operand tile to TF32 in
-// shared memory (the rounding the backward pass's operand copies use too).
+// The two-query-tile forward serves 16-bit inputs, and fp32 (TF32) inputs up to
+// d = 64 (its warp 3 rounds their tiles).  fp32 at d = 80 and 128 uses the
+// one-tile kernel (two query tiles of fp32 leave too little shared memory).
 template <int ES, int D>
 constexpr bool use_two_tile_forward() {
-    return ES == 2 && Fwd2Cfg<ES, D>::kFits;
+    return (ES == 2 || D <= 64) && Fwd2Cfg<ES, D>::kFits;
 }
 
 template <int ES, int D, bool F16 = false>

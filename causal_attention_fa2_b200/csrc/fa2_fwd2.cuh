@@ -16,7 +16,11 @@
 //              runs PV_B(j) and S_B(j+1), and the other way round.
 //   warp 2     load watcher: adds the arrival that tells the issuer V_j and
 //              K_{j+1} have landed to the P-ready barrier, so the issuer waits
-//              on that barrier alone.  Warp 3 idles.
+//              on that barrier alone.
+//   warp 3     fp32 inputs: rounds each landed Q, K and V tile to TF32 in
+//              shared memory (round to nearest, as the one-tile kernel and the
+//              backward's operand copies do) and only then releases it; the
+//              issuer and the watcher wait on those releases.  Idle otherwise.
 //   warps 4-7  softmax warpgroup for tile A; warps 8-11 for tile B.  Thread t
 //              owns query row t of its tile (tensor-memory lane t).
 //   Warpgroup 0 (warps 0-3) runs with fewer registers and the softmax
@@ -190,7 +194,7 @@ __device__ __forceinline__ void fwd2_softmax(const FwdParams p, int t, int q_til
             if constexpr (G::kF32) {
                 uint32_t u[32];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) u[c] = __float_as_uint(s[c0 + c]);
+                for (int c = 0; c < 32; ++c) u[c] = ptx::to_tf32_rna(s[c0 + c]);
                 ptx::tmem_st32(s_tmem + c0, u);
             } else {
                 uint32_t u[16];
@@ -287,6 +291,11 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     __shared__ uint64_t bar_q_full;
     __shared__ uint64_t bar_k_full[ST], bar_k_empty[ST], bar_v_full[ST], bar_v_empty[ST];
     __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done[2], bar_drain;
+    // fp32: tiles released by the rounding warp (what the issuer and watcher wait on).
+    __shared__ uint64_t bar_q_ready, bar_k_ready[ST], bar_v_ready[ST];
+    uint64_t* const q_go = G::kF32 ? &bar_q_ready : &bar_q_full;
+    uint64_t* const k_go = G::kF32 ? bar_k_ready : bar_k_full;
+    uint64_t* const v_go = G::kF32 ? bar_v_ready : bar_v_full;
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     // Block-sparse: the pair's key tiles, in order, with bit 14 / 15 set when
@@ -355,6 +364,11 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             ptx::mbar_init(&bar_o_done[t], 1);
         }
         ptx::mbar_init(&bar_drain, 1);
+        ptx::mbar_init(&bar_q_ready, 1);
+        for (int s = 0; s < ST; ++s) {
+            ptx::mbar_init(&bar_k_ready[s], 1);
+            ptx::mbar_init(&bar_v_ready[s], 1);
+        }
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -447,7 +461,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             constexpr uint32_t idesc_qk = ptx::instr_desc(G::kFmt, 128, 128, false, false);
             constexpr uint32_t idesc_pv = ptx::instr_desc(G::kFmt, 128, G::kNOut, false, true);
             const uint32_t q_addr[2] = {ptx::smem_addr(sQ[0]), ptx::smem_addr(sQ[1])};
-            bool ok = ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            bool ok = ptx::mbar_wait(q_go, 0, &abort_flag, tmo);
             auto issue_s = [&](int t, int j) {
                 const uint32_t k_addr = ptx::smem_addr(sK + (j % ST) * G::kTileBytesK);
 #pragma unroll
@@ -489,7 +503,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     if (pend[t] < 0) return true;
                     const int l = local[t] - 1, jv = pend[t];
                     if (!ptx::mbar_wait(&bar_p_full[t], l & 1, &abort_flag, tmo)) return false;
-                    if (!ptx::mbar_wait(&bar_v_full[jv % ST], (jv / ST) & 1, &abort_flag, tmo)) return false;
+                    if (!ptx::mbar_wait(&v_go[jv % ST], (jv / ST) & 1, &abort_flag, tmo)) return false;
                     ptx::tc_fence_after();
                     const uint32_t v_addr = ptx::smem_addr(sV + (jv % ST) * G::kTileBytesMN);
 #pragma unroll
@@ -507,7 +521,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 };
                 for (int j = 0; ok && j < n_kv; ++j) {
                     const unsigned bits = step_bits(j);
-                    ok = ptx::mbar_wait(&bar_k_full[j % ST], (j / ST) & 1, &abort_flag, tmo);
+                    ok = ptx::mbar_wait(&k_go[j % ST], (j / ST) & 1, &abort_flag, tmo);
                     for (int t = 0; t < 2 && ok; ++t) {
                         if (!flush(t)) { ok = false; break; }
                         if ((bits >> t) & 1u) {
@@ -526,7 +540,7 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (ok) ptx::mma_commit(&bar_v_empty[(n_kv - 1) % ST]);
             } else {
             // Prologue: S_A(0), S_B(0).
-            if (ok) ok = ptx::mbar_wait(&bar_k_full[0], 0, &abort_flag, tmo);
+            if (ok) ok = ptx::mbar_wait(&k_go[0], 0, &abort_flag, tmo);
             if (ok) {
                 ptx::tc_fence_after();
                 issue_s(0, 0);
@@ -568,12 +582,34 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int j = 0; ok && j < n_kv; ++j) {
                 for (int t = 0; t < 2 && ok; ++t) {
                     if (j >= n_kv_t[t]) continue;
-                    ok = ptx::mbar_wait(&bar_v_full[j % ST], (j / ST) & 1, &abort_flag, tmo);
+                    ok = ptx::mbar_wait(&v_go[j % ST], (j / ST) & 1, &abort_flag, tmo);
                     if (ok && j + 1 < n_kv_t[t])
-                        ok = ptx::mbar_wait(&bar_k_full[(j + 1) % ST], ((j + 1) / ST) & 1, &abort_flag, tmo);
+                        ok = ptx::mbar_wait(&k_go[(j + 1) % ST], ((j + 1) / ST) & 1, &abort_flag, tmo);
                     if (ok && j > 0) ok = ptx::mbar_wait(&bar_p_full[t], (j - 1) & 1, &abort_flag, tmo);
                     if (ok) ptx::mbar_arrive(&bar_p_full[t]);
                 }
+            }
+        }
+    } else if (G::kF32 && warp == 3) {
+        // ------------------------------------------------ TF32 rounding (fp32 only)
+        // Only the Q slots that were loaded: an unloaded slot stages the zero
+        // epilogue of a query tile without key steps.
+        if constexpr (G::kF32) {
+            constexpr bool kB = D >= 64;
+            bool ok = (!SPARSE || n_kv > 0) && ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
+            if (ok) {
+                for (int t = 0; t < 2; ++t)
+                    if (load_q[t]) round_tf32_smem<G::kTileBytesK, kB>(sQ[t], lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int s = j % ST;
+                if (!ptx::mbar_wait(&bar_k_full[s], (j / ST) & 1, &abort_flag, tmo)) break;
+                round_tf32_smem<G::kTileBytesK, kB>(sK + s * G::kTileBytesK, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_k_ready[s]);
+                if (!ptx::mbar_wait(&bar_v_full[s], (j / ST) & 1, &abort_flag, tmo)) break;
+                round_tf32_smem<G::kTileBytesMN, kB>(sV + s * G::kTileBytesMN, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_v_ready[s]);
             }
         }
     }
