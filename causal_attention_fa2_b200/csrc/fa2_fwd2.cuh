@@ -595,6 +595,8 @@ fa2_fwd2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // Only the Q slots that were loaded: an unloaded slot stages the zero
         // epilogue of a query tile without key steps.
         if constexpr (G::kF32) {
+            // Batched rounding loop at d = 64, the plain one at d <= 32 (as in the
+            // one-tile kernel).
             constexpr bool kB = D >= 64;
             bool ok = (!SPARSE || n_kv > 0) && ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo);
             if (ok) {
