@@ -54,10 +54,11 @@ struct Bwd32Cfg {
     // most of its instructions: W = 32 halves them per query row.
     static constexpr bool kKInTmem = (D == 128);
     static constexpr int kResidentKV = (kKInTmem ? 1 : 2) * tile_k(kTileRows);
-    // dQ pass at d = 128, likewise: Q and dO in tensor memory (the A operands of
-    // S = Q K^T and dP = dO V^T), nothing resident in shared memory, and key
-    // sub-tiles of 64 rows instead of 32.
-    static constexpr bool kQInTmem = (D == 128);
+    // dQ pass at d = 64 and 128, likewise: Q and dO in tensor memory (the A
+    // operands of S = Q K^T and dP = dO V^T), nothing resident in shared memory,
+    // and key sub-tiles of 128 rows instead of 64 (d = 64), 64 instead of 32
+    // (d = 128).
+    static constexpr bool kQInTmem = (D == 64 || D == 128);
     static constexpr int kResidentQ = kQInTmem ? 0 : 2 * tile_k(kTileRows);
     __host__ __device__ static constexpr int stages_for(int stage_bytes, int resident = kResident) {
         const int s = (kBudget - resident) / stage_bytes;
@@ -93,9 +94,9 @@ struct Bwd32Cfg {
     static constexpr uint32_t kColDPkv = kKInTmem ? 64 : kColDP, kColKT = 128;
     static_assert(!kKInTmem || kWkv <= 64, "S^T and dP^T must fit below the K columns");
     // dQ pass with Q and dO in tensor memory: S | dP | dQ | Q | dO.
-    static constexpr uint32_t kColDPq = kQInTmem ? 64 : kColDP, kColDQq = kQInTmem ? 128 : kColDQ;
-    static constexpr uint32_t kColQT = 256, kColDOT = 384;
-    static_assert(!kQInTmem || kWq <= 64, "S and dP must fit below the dQ columns");
+    static constexpr uint32_t kColDPq = kQInTmem ? kWq : kColDP, kColDQq = kQInTmem ? 2 * kWq : kColDQ;
+    static constexpr uint32_t kColQT = 2 * kWq + G::kNOut, kColDOT = kColQT + G::kStepsD * G::kKStep;
+    static_assert(!kQInTmem || kColDOT + G::kStepsD * G::kKStep <= kTmemCols, "dQ pass columns exceed TMEM");
 };
 
 // ------------------------------------------------------------------ pre-processing
