@@ -80,12 +80,21 @@ struct Bwd32Cfg {
     }
     // At most 64 query rows per dK/dV sub-tile: with 128 (d = 16, 32) a thread's
     // P^T row of W fp32 values spilled, and the pass ran 10 % slower, same bits.
-    static constexpr int kWkv = pick_kv() > 64 ? 64 : pick_kv();
-    static constexpr int kStKV = stages_for(kv_stage(kWkv), kResidentKV);
+    // dK/dV pass at d = 128 (K in TMEM): sub-tiles of 64 query rows in a single
+    // stage whose four parts (Q and dO, each K-major and MN-major) are refilled
+    // one by one as soon as the one MMA group that reads each has finished, plus a
+    // second slot for Q K-major, the part each sub-tile needs first.  Two whole
+    // stages of 64 rows do not fit beside V; 32-row sub-tiles left the tcgen05
+    // instruction pipe the busiest unit of the pass.
+    static constexpr bool kPartStaged = kKInTmem;
+    static constexpr int kWkv = kPartStaged ? 64 : (pick_kv() > 64 ? 64 : pick_kv());
+    static constexpr int kStKV = kPartStaged ? 1 : stages_for(kv_stage(kWkv), kResidentKV);
     static constexpr int kWq = pick_q();
     static constexpr int kStQ = stages_for(q_stage(kWq), kResidentQ);
-    static_assert(kStKV >= 2 && kStQ >= 2, "shared memory too small for two pipeline stages");
-    static constexpr int kSmemKV = 1024 + kResidentKV + kStKV * kv_stage(kWkv);
+    static_assert((kPartStaged || kStKV >= 2) && kStQ >= 2, "shared memory too small for two pipeline stages");
+    static constexpr int kSmemKV = 1024 + kResidentKV +
+        (kPartStaged ? 3 * tile_k(kWkv) + 2 * tile_mn(kWkv) : kStKV * kv_stage(kWkv));
+    static_assert(kSmemKV <= 227 * 1024 - 1024, "dK/dV pass shared memory over the limit");
     static constexpr int kSmemQ = 1024 + kResidentQ + kStQ * q_stage(kWq);
     static constexpr uint32_t kTmemCols = 512;
     // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
@@ -284,6 +293,9 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     __shared__ uint64_t bar_kv_full, bar_full[ST], bar_empty[ST];
     __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_dkv_full, bar_drain;
     __shared__ uint64_t bar_kt_ready;                   // K written to tensor memory (KT)
+    // Part-staged (PP): full / empty barrier per part slot: Q K-major slots 0 and
+    // 1, then dO K-major, Q MN-major, dO MN-major.
+    __shared__ uint64_t bar_pf[5], bar_pe[5];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     __shared__ int s_cnt;                               // block-sparse: query sub-tiles per head
@@ -297,6 +309,16 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     // dK is staged for its store where K was, or in the (then idle) first stage.
     uint8_t* sDK = KT ? sStage : sK;
     // Stage s: Q (K-major) | dO (K-major) | Q (MN-major) | dO (MN-major).
+    // Part-staged: Q (K-major) slot 0 | slot 1 | dO (K-major) | Q (MN-major) | dO (MN-major).
+    constexpr bool PP = Cfg::kPartStaged;
+    constexpr int kPartQk = 0, kPartDok = 1, kPartQmn = 2, kPartDomn = 3;
+    auto pp_slot = [](int part, int it) { return part == kPartQk ? (it & 1) : part + 1; };
+    auto pp_phase = [](int part, int it) -> uint32_t { return static_cast<uint32_t>(part == kPartQk ? it >> 1 : it) & 1u; };
+    auto pp_addr = [&](int part, int it) -> uint8_t* {
+        return part == kPartQk ? sStage + (it & 1) * SK
+             : part == kPartDok ? sStage + 2 * SK
+             : part == kPartQmn ? sStage + 3 * SK : sStage + 3 * SK + SM;
+    };
     auto st_qk = [&](int s) { return sStage + s * SB; };
     auto st_dok = [&](int s) { return sStage + s * SB + SK; };
     auto st_qmn = [&](int s) { return sStage + s * SB + 2 * SK; };
@@ -346,6 +368,10 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         ptx::mbar_init(&bar_dkv_full, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::mbar_init(&bar_kt_ready, 4);
+        for (int b = 0; b < 5; ++b) {
+            ptx::mbar_init(&bar_pf[b], 1);
+            ptx::mbar_init(&bar_pe[b], 1);
+        }
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
@@ -362,11 +388,12 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     // dK = dV = 0 is written.
     const int n_q = SPARSE ? s_cnt : (n_sub > sub_begin ? n_sub - sub_begin : 0);
     const int n_it = n_q * p.group;                     // (query head, sub-tile) steps
-    auto q_row_of = [&](int it) {
+    auto q_row_walk = [&](MaskWalk& w, int it) {
         const int g = it % n_q;
         if (!SPARSE) return (sub_begin + g) * W;
-        return ((i_begin + walker.at(g / R, n_col, blk_set)) * R + g % R) * W;
+        return ((i_begin + w.at(g / R, n_col, blk_set)) * R + g % R) * W;
     };
+    auto q_row_of = [&](int it) { return q_row_walk(walker, it); };
     auto q_head_of = [&](int it) { return (bh / p.H_kv) * p.H + (bh % p.H_kv) * p.group + it / n_q; };
 
     if (warp == 0) {
@@ -381,6 +408,59 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 if (!KT) ptx::tma_load_3d(sK + b * kTileRows * G::kRowBK, &tm_k, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
                 ptx::tma_load_3d(sV + b * kTileRows * G::kRowBK, &tm_v, &bar_kv_full, b * G::kBoxK, kv_row0, bh);
             }
+            if constexpr (PP) {
+                // The four parts stream independently, each into its slot(s) as
+                // soon as the MMA group that last read the slot has finished.
+                MaskWalk walk[4];
+                int nxt[4] = {0, 0, 0, 0};              // sub-tiles issued, per part
+                uint32_t spins = 0;
+                uint64_t t_idle = 0;
+                while (nxt[0] < n_it || nxt[1] < n_it || nxt[2] < n_it || nxt[3] < n_it) {
+                    bool moved = false;
+#pragma unroll
+                    for (int part = 0; part < 4; ++part) {
+                        const int it = nxt[part];
+                        if (it >= n_it) continue;
+                        const int depth = part == kPartQk ? 2 : 1;
+                        const int b = pp_slot(part, it);
+                        if (it >= depth && !ptx::mbar_test_wait(&bar_pe[b], pp_phase(part, it) ^ 1u)) continue;
+                        const int row0 = q_row_walk(walk[part], it);
+                        const int qh = q_head_of(it);
+                        uint8_t* dst = pp_addr(part, it);
+                        if (part == kPartQk || part == kPartDok) {
+                            ptx::mbar_arrive_expect_tx(&bar_pf[b], SK);
+                            for (int bx = 0; bx < G::kNBoxK; ++bx)
+                                ptx::tma_load_3d(dst + bx * W * G::kRowBK, part == kPartQk ? &tm_qk : &tm_dok, &bar_pf[b],
+                                                 bx * G::kBoxK, row0, qh);
+                        } else {
+                            ptx::mbar_arrive_expect_tx(&bar_pf[b], SM);
+                            for (int bx = 0; bx < G::kNBoxMN; ++bx)
+                                ptx::tma_load_3d(dst + bx * W * G::kRowBMN, part == kPartQmn ? &tm_qmn : &tm_domn, &bar_pf[b],
+                                                 bx * G::kBoxMN, row0, qh);
+                        }
+                        nxt[part] = it + 1;
+                        moved = true;
+                    }
+                    if (moved) {
+                        spins = 0;
+                    } else if (spins++ == 0) {
+                        t_idle = ptx::globaltimer_ns();
+                    } else if ((spins & 63u) == 0) {
+                        // Bounded, as every wait here: give up on abort or after the timeout.
+                        if (abort_flag) break;
+                        if (ptx::globaltimer_ns() - t_idle > tmo) { abort_flag = 1u; break; }
+                    }
+                }
+                if (abort_flag) {
+                    constexpr uint64_t kDrainNs = 20000000ull;
+                    ptx::mbar_wait_drain(&bar_kv_full, 0, kDrainNs);
+                    for (int part = 0; part < 4; ++part) {
+                        const int depth = part == kPartQk ? 2 : 1;
+                        for (int t = nxt[part] - 1; t >= 0 && t >= nxt[part] - depth; --t)
+                            ptx::mbar_wait_drain(&bar_pf[pp_slot(part, t)], pp_phase(part, t), kDrainNs);
+                    }
+                }
+            } else {
             int issued = 0;
             for (int it = 0; it < n_it; ++it) {
                 const int s = it % ST;
@@ -404,6 +484,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 for (int t = issued - 1; t >= 0 && t >= issued - ST; --t)
                     ptx::mbar_wait_drain(&bar_full[t % ST], (t / ST) & 1, kDrainNs);
             }
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -413,11 +494,26 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             const uint32_t k_addr = ptx::smem_addr(sK);
             const uint32_t v_addr = ptx::smem_addr(sV);
             // S^T = K_j Q_i^T   (Eq. 13, transposed: rows are keys)
+            // Part-staged: wait for one part, and release it after its MMAs.
+            auto wait_part = [&](int part, int it) -> bool {
+                if constexpr (PP) {
+                    if (!ptx::mbar_wait(&bar_pf[pp_slot(part, it)], pp_phase(part, it), &abort_flag, tmo)) return false;
+                    ptx::tc_fence_after();
+                }
+                return true;
+            };
+            auto release_part = [&](int part, int it) {
+                if constexpr (PP) ptx::mma_commit(&bar_pe[pp_slot(part, it)]);
+            };
             auto issue_s = [&](int it) -> bool {
                 const int s = it % ST;
-                if (!ptx::mbar_wait(&bar_full[s], (it / ST) & 1, &abort_flag, tmo)) return false;
-                ptx::tc_fence_after();
-                const uint32_t qa = ptx::smem_addr(st_qk(s));
+                if constexpr (PP) {
+                    if (!wait_part(kPartQk, it)) return false;
+                } else {
+                    if (!ptx::mbar_wait(&bar_full[s], (it / ST) & 1, &abort_flag, tmo)) return false;
+                    ptx::tc_fence_after();
+                }
+                const uint32_t qa = ptx::smem_addr(PP ? pp_addr(kPartQk, it) : st_qk(s));
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (KT)
@@ -426,39 +522,48 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                         ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(&bar_s_full);
+                release_part(kPartQk, it);
                 return true;
             };
-            // dP^T = V_j dO_i^T   (Eq. 16, transposed); the stage is already full.
-            auto issue_dp = [&](int it) {
-                const uint32_t da = ptx::smem_addr(st_dok(it % ST));
+            // dP^T = V_j dO_i^T   (Eq. 16, transposed); the stage is already full
+            // (part-staged: its dO K-major part is waited for here).
+            auto issue_dp = [&](int it) -> bool {
+                if (!wait_part(kPartDok, it)) return false;
+                const uint32_t da = ptx::smem_addr(PP ? pp_addr(kPartDok, it) : st_dok(it % ST));
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk)
                     ptx::mma_tf32_ss(tmem + Cfg::kColDPkv, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 ptx::mma_commit(&bar_dp_full);
+                release_part(kPartDok, it);
+                return true;
             };
             bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
             if (KT && ok) ok = ptx::mbar_wait(&bar_kt_ready, 0, &abort_flag, tmo);
             if (ok) ok = issue_s(0);
-            if (ok) issue_dp(0);
+            if (ok) ok = issue_dp(0);
             for (int it = 0; ok && it < n_it; ++it) {
                 const int s = it % ST;
                 // dV_j += P^T dO_i   (Eq. 15); P^T read from the score columns.
                 if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t dmn = ptx::smem_addr(st_domn(s));
+                if (!wait_part(kPartDomn, it)) { ok = false; break; }
+                const uint32_t dmn = ptx::smem_addr(PP ? pp_addr(kPartDomn, it) : st_domn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
                     ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                release_part(kPartDomn, it);
                 if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
                 if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t qmn = ptx::smem_addr(st_qmn(s));
+                if (!wait_part(kPartQmn, it)) { ok = false; break; }
+                const uint32_t qmn = ptx::smem_addr(PP ? pp_addr(kPartQmn, it) : st_qmn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
                     ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPkv + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar_empty[s]);
-                if (it + 1 < n_it) issue_dp(it + 1);
+                if constexpr (PP) release_part(kPartQmn, it);
+                else ptx::mma_commit(&bar_empty[s]);
+                if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
             }
             if (ok) {
                 ptx::mma_commit(&bar_dkv_full);
