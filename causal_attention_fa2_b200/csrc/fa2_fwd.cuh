@@ -13,11 +13,11 @@
 // query are excluded (set to -inf, which is what the handout's -1e6 offset
 // amounts to once exponentiated).
 //
-// The library runs this kernel for fp32 inputs at d = 80 and 128, where two
-// fp32 query tiles per CTA (fa2_fwd2.cuh) leave too little shared memory.
+// The kernel serves fp32 inputs (TF32 MMAs) from d = 64 up; the library runs
+// it at d = 80 and 128, where two fp32 query tiles per CTA (fa2_fwd2.cuh, which
+// also serves every 16-bit input) leave too little shared memory.
 //
-// B200 mapping (one CTA per (query tile, head); 6 warps, 7 or 8 for fp32
-// inputs, warp-specialised):
+// B200 mapping (one CTA per (query tile, head); 8 warps, warp-specialised):
 //   warp 0    TMA producer: Q_i once, then K_j and V_j into two rings of
 //             shared-memory stages guarded by full/empty mbarriers.
 //   warp 1    MMA issuer (one thread): S_j = Q_i K_j^T into one of two
@@ -26,15 +26,15 @@
 //             signalled with tcgen05.commit on mbarriers.
 //   warps 2-5 softmax warpgroup: thread t owns query row t (TMEM lane t).  It
 //             loads its score row from TMEM, applies the mask, updates the
-//             running max / sum, writes P (bf16, or fp32 for the TF32 path)
-//             back into the score buffer for the next MMA, and rescales its O
+//             running max / sum, writes P (fp32 rounded to TF32) back into
+//             the score buffer for the next MMA, and rescales its O
 //             row in TMEM when the running max grows.  After the last tile it
 //             normalises O, stages it in shared memory for a TMA store and
 //             writes L.
-//   warp 6    (fp32 inputs only) operand rounding, with warp 7 taking the V
-//             tiles from d = 64 up: rounds each Q, K and V tile in shared
-//             memory to TF32 (round to nearest) once its TMA copy has landed
-//             and only then releases it to the MMA issuer, so
+//   warps 6-7 operand rounding, warp 6 for Q and the K tiles, warp 7 for the
+//             V tiles: rounds each tile in shared memory to TF32 (round to
+//             nearest) once its TMA copy has landed and only then releases it
+//             to the MMA issuer, so
 //             the tensor core reads the operands exactly instead of dropping
 //             their 13 low bits (a biased error); the softmax group rounds P
 //             the same way.  The backward pass rounds its copies identically,
@@ -73,17 +73,15 @@ struct FwdParams {
 template <int ES, int D>
 struct FwdCfg {
     using G = TileGeom<ES, D>;
-    // fp32: from d = 64 up, Q / K and V are rounded by separate warps (measured:
-    // 1.45x at d = 128, 1.08x at d = 64); at d <= 32 one warp rounds all three
-    // (the split measured 10-15 % slower there).
-    static constexpr bool kRoundSplit = G::kF32 && D >= 64;
-    static constexpr int kThreads = G::kF32 ? (kRoundSplit ? 256 : 224) : 192;
+    // Q / K and V are rounded by separate warps (measured 1.45x at d = 128 and
+    // 1.08x at d = 64 against one rounding warp).
+    static constexpr int kThreads = 256;
     static constexpr int kBudget = 227 * 1024 - 2048;
     // fp32 at d = 128: Q sits in tensor memory (columns 384-511, beside the two
     // score buffers and O), written there rounded by the softmax threads; S =
     // Q K^T reads its A operand from TMEM, and the 64 KB of shared memory this
     // frees gives K a second ring stage.
-    static constexpr bool kQInTmem = G::kF32 && D == 128;
+    static constexpr bool kQInTmem = D == 128;
     static constexpr uint32_t kQCol = 384;
     static constexpr int kQBytes = kQInTmem ? 0 : G::kTileBytesK;   // Q staged in shared memory
     static constexpr int kFree = kBudget - kQBytes;
@@ -105,7 +103,7 @@ struct FwdCfg {
     // whole-tile hand-offs left the tensor pipe idle while each 64 KB tile was
     // loaded and rounded.  At d <= 80 the parts' extra waits cost more than they
     // overlap (measured 16 % slower at d = 64, 15 % at d = 80).
-    static constexpr bool kParted = G::kF32 && D == 128;
+    static constexpr bool kParted = D == 128;
     static constexpr int kKParts = kParted ? G::kNBoxK : 1;
     static constexpr int kVParts = kParted ? 4 : 1;   // 4 measured 3-4 % faster than 2, 7 % than 1
     static constexpr int kKPartBytes = G::kTileBytesK / kKParts;
@@ -162,6 +160,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     ptx::pdl_wait();
     using Cfg = FwdCfg<ES, D>;
     using G = typename Cfg::G;
+    static_assert(ES == 4 && D >= 64, "the one-tile kernel serves fp32 inputs from d = 64 up");
     constexpr int KST = Cfg::kKSt;
     constexpr int VST = Cfg::kVSt;
     constexpr int KP = Cfg::kKParts;
@@ -174,14 +173,14 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     __shared__ uint64_t bar_k_full[KS], bar_k_empty[KS];
     __shared__ uint64_t bar_v_full[VS], bar_v_empty[VS];
     __shared__ uint64_t bar_s_full[2], bar_p_full[2], bar_o_done, bar_drain;
-    // fp32: tiles released by the rounding warp (the MMA issuer waits on these).
+    // Tiles released by the rounding warps (the MMA issuer waits on these).
     __shared__ uint64_t bar_q_ready, bar_k_ready[KS], bar_v_ready[VS];
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
     __shared__ int s_cnt;                      // block-sparse: key tiles of this query tile
-    uint64_t* const q_go = G::kF32 ? &bar_q_ready : &bar_q_full;
-    uint64_t* const k_go = G::kF32 ? bar_k_ready : bar_k_full;
-    uint64_t* const v_go = G::kF32 ? bar_v_ready : bar_v_full;
+    uint64_t* const q_go = &bar_q_ready;
+    uint64_t* const k_go = bar_k_ready;
+    uint64_t* const v_go = bar_v_ready;
 
     const uint32_t raw = ptx::smem_addr(smem_raw);
     uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -329,10 +328,7 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     for (int k2 = 0; k2 < Cfg::kVStepsPart; ++k2) {
                         const int kk = h * Cfg::kVStepsPart + k2;
                         const uint64_t bdesc = desc_mnmajor<G>(v_addr, k2, Cfg::kVPartRows);
-                        if constexpr (G::kF32)
-                            ptx::mma_tf32_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
-                        else
-                            ptx::mma_f16_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+                        ptx::mma_tf32_ts(tmem + Cfg::kOCol, p_tmem + kk * 8, bdesc, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
                     }
                     ptx::mma_commit(&bar_v_empty[sl]);
                 }
@@ -354,10 +350,8 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             const uint64_t bdesc = desc_kmajor<G>(k_addr, kk);
                             if constexpr (QT)
                                 ptx::mma_tf32_ts(s_tmem, tmem + Cfg::kQCol + kk * G::kKStep, bdesc, idesc_qk, kk > 0 ? 1u : 0u);
-                            else if constexpr (G::kF32)
-                                ptx::mma_tf32_ss(s_tmem, desc_kmajor<G>(q_addr, kk), bdesc, idesc_qk, kk > 0 ? 1u : 0u);
                             else
-                                ptx::mma_f16_ss(s_tmem, desc_kmajor<G>(q_addr, kk), bdesc, idesc_qk, kk > 0 ? 1u : 0u);
+                                ptx::mma_tf32_ss(s_tmem, desc_kmajor<G>(q_addr, kk), bdesc, idesc_qk, kk > 0 ? 1u : 0u);
                         }
                     }
                     ptx::mma_commit(&bar_k_empty[sl]);
@@ -467,23 +461,13 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 rs += pc;
             }
             l += rs;
-            // P back into the score buffer (A operand of the PV MMA).
-            if constexpr (G::kF32) {
+            // P, rounded to TF32, back into the score buffer (A operand of the PV MMA).
 #pragma unroll
-                for (int c0 = 0; c0 < 128; c0 += 32) {
-                    uint32_t u[32];
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+                uint32_t u[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) u[c] = ptx::to_tf32_rna(s[c0 + c]);
-                    ptx::tmem_st32(s_tmem + c0, u);
-                }
-            } else {
-#pragma unroll
-                for (int c0 = 0; c0 < 64; c0 += 32) {
-                    uint32_t u[32];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) u[c] = ptx::pack_bf16x2(s[2 * (c0 + c)], s[2 * (c0 + c) + 1]);
-                    ptx::tmem_st32(s_tmem + c0, u);
-                }
+                for (int c = 0; c < 32; ++c) u[c] = ptx::to_tf32_rna(s[c0 + c]);
+                ptx::tmem_st32(s_tmem + c0, u);
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -503,32 +487,16 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     ptx::tmem_ld16(o_tmem + c0, u);
                     ptx::tmem_wait_ld();
                 }
-                if constexpr (G::kF32) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int col = c0 + 4 * q4;
-                        if (col < D) {
-                            uint4 w;
-                            w.x = __float_as_uint(__uint_as_float(u[4 * q4 + 0]) * inv_l);
-                            w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * inv_l);
-                            w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * inv_l);
-                            w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * inv_l);
-                            *reinterpret_cast<uint4*>(sO + kmajor_chunk_offset<G>(r, col)) = w;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int h8 = 0; h8 < 2; ++h8) {
-                        const int col = c0 + 8 * h8;
-                        if (col < D) {
-                            uint4 w;
-                            const float* f = reinterpret_cast<const float*>(u) + 8 * h8;
-                            w.x = ptx::pack_bf16x2(f[0] * inv_l, f[1] * inv_l);
-                            w.y = ptx::pack_bf16x2(f[2] * inv_l, f[3] * inv_l);
-                            w.z = ptx::pack_bf16x2(f[4] * inv_l, f[5] * inv_l);
-                            w.w = ptx::pack_bf16x2(f[6] * inv_l, f[7] * inv_l);
-                            *reinterpret_cast<uint4*>(sO + kmajor_chunk_offset<G>(r, col)) = w;
-                        }
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int col = c0 + 4 * q4;
+                    if (col < D) {
+                        uint4 w;
+                        w.x = __float_as_uint(__uint_as_float(u[4 * q4 + 0]) * inv_l);
+                        w.y = __float_as_uint(__uint_as_float(u[4 * q4 + 1]) * inv_l);
+                        w.z = __float_as_uint(__uint_as_float(u[4 * q4 + 2]) * inv_l);
+                        w.w = __float_as_uint(__uint_as_float(u[4 * q4 + 3]) * inv_l);
+                        *reinterpret_cast<uint4*>(sO + kmajor_chunk_offset<G>(r, col)) = w;
                     }
                 }
             }
@@ -546,39 +514,31 @@ fa2_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ptx::tma_store_wait_all();
         }
     } else {
-        // ------------------------------------------------ TF32 rounding (fp32 only)
-        if constexpr (G::kF32) {
-            // warp 6: Q and the K parts (and the V tiles unless warp 7 has them).
-            constexpr bool kB = Cfg::kRoundSplit;
-            if (warp == 6) {
-                bool ok = n_kv > 0 && (QT || ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo));
-                if (ok && !QT) {
-                    round_tf32_smem<G::kTileBytesK, kB>(sQ, lane);
-                    if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
+        // ------------------------------------------------ TF32 rounding
+        if (warp == 6) {
+            // Q (unless it is in tensor memory) and the K parts.
+            bool ok = n_kv > 0 && (QT || ptx::mbar_wait(&bar_q_full, 0, &abort_flag, tmo));
+            if (ok && !QT) {
+                round_tf32_smem<G::kTileBytesK, true>(sQ, lane);
+                if (lane == 0) ptx::mbar_arrive(&bar_q_ready);
+            }
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int ks = j % KST;
+                for (int b = 0; ok && b < KP; ++b) {
+                    if (!ptx::mbar_wait(&bar_k_full[ks * KP + b], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                    round_tf32_smem<Cfg::kKPartBytes, true>(sK + ks * G::kTileBytesK + b * Cfg::kKPartBytes, lane);
+                    if (lane == 0) ptx::mbar_arrive(&bar_k_ready[ks * KP + b]);
                 }
-                for (int j = 0; ok && j < n_kv; ++j) {
-                    const int ks = j % KST;
-                    for (int b = 0; ok && b < KP; ++b) {
-                        if (!ptx::mbar_wait(&bar_k_full[ks * KP + b], (j / KST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                        round_tf32_smem<Cfg::kKPartBytes, kB>(sK + ks * G::kTileBytesK + b * Cfg::kKPartBytes, lane);
-                        if (lane == 0) ptx::mbar_arrive(&bar_k_ready[ks * KP + b]);
-                    }
-                    if constexpr (!Cfg::kRoundSplit) {
-                        const int vs = j % VST;
-                        if (!ok || !ptx::mbar_wait(&bar_v_full[vs], (j / VST) & 1, &abort_flag, tmo)) break;
-                        round_tf32_smem<G::kTileBytesMN, kB>(sV + vs * G::kTileBytesMN, lane);
-                        if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs]);
-                    }
-                }
-            } else if constexpr (Cfg::kRoundSplit) {
-                bool ok = true;
-                for (int j = 0; ok && j < n_kv; ++j) {
-                    const int vs = j % VST;
-                    for (int h = 0; h < VP; ++h) {
-                        if (!ptx::mbar_wait(&bar_v_full[vs * VP + h], (j / VST) & 1, &abort_flag, tmo)) { ok = false; break; }
-                        round_tf32_smem<Cfg::kVPartBytes, kB>(sV + vs * G::kTileBytesMN + h * Cfg::kVPartBytes, lane);
-                        if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs * VP + h]);
-                    }
+            }
+        } else {
+            // The V parts.
+            bool ok = true;
+            for (int j = 0; ok && j < n_kv; ++j) {
+                const int vs = j % VST;
+                for (int h = 0; h < VP; ++h) {
+                    if (!ptx::mbar_wait(&bar_v_full[vs * VP + h], (j / VST) & 1, &abort_flag, tmo)) { ok = false; break; }
+                    round_tf32_smem<Cfg::kVPartBytes, true>(sV + vs * G::kTileBytesMN + h * Cfg::kVPartBytes, lane);
+                    if (lane == 0) ptx::mbar_arrive(&bar_v_ready[vs * VP + h]);
                 }
             }
         }
