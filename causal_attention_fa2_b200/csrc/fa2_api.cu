@@ -524,7 +524,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             return st;
         auto kern = block_mask ? fa2_bwd32_dkdv_kernel<D, true> : fa2_bwd32_dkdv_kernel<D, false>;
         if ((st = set_smem(kern, Cfg::kSmemKV)) != FA2_OK) return st;
-        launch_pdl(kern, dim3(grid_kv), dim3(Cfg::kThreads), Cfg::kSmemKV, stream, mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
+        launch_pdl(kern, dim3(grid_kv), dim3(Cfg::kThreadsKV), Cfg::kSmemKV, stream, mqk, mqmn, mk, mv, mdok, mdomn, mdk, mdv, p);
         if (cudaGetLastError() != cudaSuccess || !mark(3)) return FA2_ERR_CUDA;
     }
     return FA2_OK;

@@ -42,6 +42,11 @@ template <int D>
 struct Bwd32Cfg {
     using G = TileGeom<4, D>;
     static constexpr int kThreads = 192;
+    // dK/dV pass at d <= 32, where its elementwise work outweighs the MMAs: two
+    // P / dS warpgroups take alternate query sub-tiles (S^T and dP^T double
+    // buffered in TMEM), so one group's exponentials overlap the other's MMAs.
+    static constexpr int kGroupsKV = D <= 32 ? 2 : 1;
+    static constexpr int kThreadsKV = 64 + 128 * kGroupsKV;
     // 227 KB minus the 1024-byte alignment pad and the static shared memory.
     static constexpr int kBudget = 227 * 1024 - 1024 - 1024;
     __host__ __device__ static constexpr int tile_k(int rows) { return G::kNBoxK * rows * G::kRowBK; }
@@ -270,7 +275,7 @@ __device__ __forceinline__ void bwd32_stage_rows(uint32_t acc_col, int r, float 
 // With a block mask (SPARSE) only the sub-tiles of query tiles whose block with
 // key tile j is set are visited, found by each thread walking the mask column.
 template <int D, bool SPARSE = false>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Bwd32Cfg<D>::kThreadsKV, 1)
 fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_constant__ CUtensorMap tm_qmn,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const __grid_constant__ CUtensorMap tm_dok, const __grid_constant__ CUtensorMap tm_domn,
@@ -291,7 +296,9 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full, bar_full[ST], bar_empty[ST];
-    __shared__ uint64_t bar_s_full, bar_dp_full, bar_p_ready, bar_ds_ready, bar_dkv_full, bar_drain;
+    constexpr int NG = Cfg::kGroupsKV;                  // P / dS warpgroups (buffers)
+    static_assert(NG == 1 || (!Cfg::kKInTmem && NG * W <= 128), "S^T / dP^T buffers exceed their TMEM columns");
+    __shared__ uint64_t bar_s_full[NG], bar_dp_full[NG], bar_p_ready[NG], bar_ds_ready[NG], bar_dkv_full, bar_drain;
     __shared__ uint64_t bar_kt_ready;                   // K written to tensor memory (KT)
     // Part-staged (PP): full / empty barrier per part slot: Q K-major slots 0 and
     // 1, then dO K-major, Q MN-major, dO MN-major.
@@ -361,10 +368,12 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             ptx::mbar_init(&bar_full[s], 1);
             ptx::mbar_init(&bar_empty[s], 1);
         }
-        ptx::mbar_init(&bar_s_full, 1);
-        ptx::mbar_init(&bar_dp_full, 1);
-        ptx::mbar_init(&bar_p_ready, 4);
-        ptx::mbar_init(&bar_ds_ready, 4);
+        for (int b = 0; b < NG; ++b) {
+            ptx::mbar_init(&bar_s_full[b], 1);
+            ptx::mbar_init(&bar_dp_full[b], 1);
+            ptx::mbar_init(&bar_p_ready[b], 4);
+            ptx::mbar_init(&bar_ds_ready[b], 4);
+        }
         ptx::mbar_init(&bar_dkv_full, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::mbar_init(&bar_kt_ready, 4);
@@ -514,14 +523,15 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                     ptx::tc_fence_after();
                 }
                 const uint32_t qa = ptx::smem_addr(PP ? pp_addr(kPartQk, it) : st_qk(s));
+                const int b = it % NG;
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (KT)
                         ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColKT + kk * G::kKStep, desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
-                        ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ss(tmem + Cfg::kColS + b * W, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(&bar_s_full);
+                ptx::mma_commit(&bar_s_full[b]);
                 release_part(kPartQk, it);
                 return true;
             };
@@ -530,40 +540,47 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             auto issue_dp = [&](int it) -> bool {
                 if (!wait_part(kPartDok, it)) return false;
                 const uint32_t da = ptx::smem_addr(PP ? pp_addr(kPartDok, it) : st_dok(it % ST));
+                const int b = it % NG;
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk)
-                    ptx::mma_tf32_ss(tmem + Cfg::kColDPkv, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
-                ptx::mma_commit(&bar_dp_full);
+                    ptx::mma_tf32_ss(tmem + Cfg::kColDPkv + b * W, desc_kmajor<G>(v_addr, kk), desc_kmajor<G>(da, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                ptx::mma_commit(&bar_dp_full[b]);
                 release_part(kPartDok, it);
                 return true;
             };
             bool ok = ptx::mbar_wait(&bar_kv_full, 0, &abort_flag, tmo);
             if (KT && ok) ok = ptx::mbar_wait(&bar_kt_ready, 0, &abort_flag, tmo);
-            if (ok) ok = issue_s(0);
-            if (ok) ok = issue_dp(0);
+            for (int i = 0; ok && i < NG && i < n_it; ++i) {
+                ok = issue_s(i);
+                if (ok) ok = issue_dp(i);
+            }
+            // Sub-tile it + NG reuses the buffers of sub-tile it: its S^T follows
+            // dV(it), its dP^T follows dK(it) (the MMAs that read them).
             for (int it = 0; ok && it < n_it; ++it) {
                 const int s = it % ST;
+                const int b = it % NG;
+                const uint32_t ph = static_cast<uint32_t>(it / NG) & 1u;
                 // dV_j += P^T dO_i   (Eq. 15); P^T read from the score columns.
-                if (!ptx::mbar_wait(&bar_p_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                if (!ptx::mbar_wait(&bar_p_ready[b], ph, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
                 if (!wait_part(kPartDomn, it)) { ok = false; break; }
                 const uint32_t dmn = ptx::smem_addr(PP ? pp_addr(kPartDomn, it) : st_domn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + b * W + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 release_part(kPartDomn, it);
-                if (it + 1 < n_it && !issue_s(it + 1)) { ok = false; break; }
+                if (it + NG < n_it && !issue_s(it + NG)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
-                if (!ptx::mbar_wait(&bar_ds_ready, it & 1, &abort_flag, tmo)) { ok = false; break; }
+                if (!ptx::mbar_wait(&bar_ds_ready[b], ph, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
                 if (!wait_part(kPartQmn, it)) { ok = false; break; }
                 const uint32_t qmn = ptx::smem_addr(PP ? pp_addr(kPartQmn, it) : st_qmn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPkv + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPkv + b * W + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 if constexpr (PP) release_part(kPartQmn, it);
                 else ptx::mma_commit(&bar_empty[s]);
-                if (it + 1 < n_it && !issue_dp(it + 1)) { ok = false; break; }
+                if (it + NG < n_it && !issue_dp(it + NG)) { ok = false; break; }
             }
             if (ok) {
                 ptx::mma_commit(&bar_dkv_full);
@@ -573,7 +590,8 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             }
         }
     } else {
-        // ------------------------------------------------ P / dS warpgroup
+        // ------------------------------------------------ P / dS warpgroup(s)
+        const int grp = (warp - 2) >> 2;                 // takes sub-tiles it = grp (mod NG)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // key row inside the tile
         const bool key_valid = kv_row0 + r < p.Nk;
@@ -604,7 +622,9 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 if (lane == 0) ptx::mbar_arrive(&bar_kt_ready);
             }
         }
-        for (int it = 0; it < n_it; ++it) {
+        const uint32_t col_s = Cfg::kColS + grp * W, col_dp = Cfg::kColDPkv + grp * W;
+        for (int it = grp; it < n_it; it += NG) {
+            const uint32_t ph = static_cast<uint32_t>(it / NG) & 1u;
             const int q0 = q_row_of(it);
             const size_t qv = static_cast<size_t>(q_head_of(it)) * p.n_pad + q0;
             const float* l2q = p.l2 + qv;
@@ -612,10 +632,10 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             // Some query of this sub-tile precedes some key of the tile.
             const bool mask = p.causal && q0 < kv_row0 + kTileRows - 1;
             // ---- P^T = exp2(S^T * scale*log2(e) - L*log2(e))   (Eq. 14), in place
-            if (!ptx::mbar_wait(&bar_s_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar_s_full[grp], ph, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
             uint32_t pu[W];
-            tmem_ld_cols<W>(lane_base + Cfg::kColS, pu);
+            tmem_ld_cols<W>(lane_base + col_s, pu);
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < W; c += 4) {
@@ -628,20 +648,21 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                     pu[c + h] = __float_as_uint(pe);
                 }
             }
-            bwd32_store_p<W>(lane_base + Cfg::kColS, pu);
+            bwd32_store_p<W>(lane_base + col_s, pu);
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_p_ready);
+            if (lane == 0) ptx::mbar_arrive(&bar_p_ready[grp]);
             // ---- dS^T = P^T o (dP^T - D)   (Eq. 17), in place over dP^T
-            if (!ptx::mbar_wait(&bar_dp_full, it & 1, &abort_flag, tmo)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar_dp_full[grp], ph, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            bwd32_ds_inplace<W>(lane_base + Cfg::kColDPkv, pu, [&](int c) { return __ldg(dvq + c); });
+            bwd32_ds_inplace<W>(lane_base + col_dp, pu, [&](int c) { return __ldg(dvq + c); });
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready[grp]);
         }
-        // ---------------- epilogue: dV -> sV, dK * scale -> sK, then TMA stores.
+        // ---------------- epilogue (group 0): dV -> sV, dK * scale -> sK, then TMA stores.
+        if (grp == 0) {
         if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
@@ -657,6 +678,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
             }
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
+        }
         }
     }
 
