@@ -511,7 +511,7 @@ fa2_status launch_backward32_t(const void* q, const void* k, const void* v, cons
             return st;
         auto kern = block_mask ? fa2_bwd32_dq_kernel<D, true> : fa2_bwd32_dq_kernel<D, false>;
         if ((st = set_smem(kern, Cfg::kSmemQ)) != FA2_OK) return st;
-        launch_pdl(kern, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemQ, stream, mq, mdo, mkk, mkmn, mvk, mdq, p);
+        launch_pdl(kern, dim3(grid), dim3(Cfg::kThreadsQ), Cfg::kSmemQ, stream, mq, mdo, mkk, mkmn, mvk, mdq, p);
         if (cudaGetLastError() != cudaSuccess || !mark(2)) return FA2_ERR_CUDA;
     }
     {

@@ -47,6 +47,10 @@ struct Bwd32Cfg {
     // buffered in TMEM), so one group's exponentials overlap the other's MMAs.
     static constexpr int kGroupsKV = D <= 32 ? 2 : 1;
     static constexpr int kThreadsKV = 64 + 128 * kGroupsKV;
+    // dQ pass likewise at d <= 32: two warpgroups on alternate key sub-tiles of
+    // 64 rows (one group took 128-row sub-tiles).
+    static constexpr int kGroupsQ = D <= 32 ? 2 : 1;
+    static constexpr int kThreadsQ = 64 + 128 * kGroupsQ;
     // 227 KB minus the 1024-byte alignment pad and the static shared memory.
     static constexpr int kBudget = 227 * 1024 - 1024 - 1024;
     __host__ __device__ static constexpr int tile_k(int rows) { return G::kNBoxK * rows * G::kRowBK; }
@@ -94,7 +98,7 @@ struct Bwd32Cfg {
     static constexpr bool kPartStaged = kKInTmem;
     static constexpr int kWkv = kPartStaged ? 64 : (pick_kv() > 64 ? 64 : pick_kv());
     static constexpr int kStKV = kPartStaged ? 1 : stages_for(kv_stage(kWkv), kResidentKV);
-    static constexpr int kWq = pick_q();
+    static constexpr int kWq = kGroupsQ == 2 ? 64 : pick_q();
     static constexpr int kStQ = stages_for(q_stage(kWq), kResidentQ);
     static_assert((kPartStaged || kStKV >= 2) && kStQ >= 2, "shared memory too small for two pipeline stages");
     static constexpr int kSmemKV = 1024 + kResidentKV +
@@ -700,7 +704,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 // With a block mask (SPARSE) only the sub-tiles of key tiles whose block with
 // query tile i is set are visited, found by each thread walking the mask row.
 template <int D, bool SPARSE = false>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Bwd32Cfg<D>::kThreadsQ, 1)
 fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_kk, const __grid_constant__ CUtensorMap tm_kmn,
                     const __grid_constant__ CUtensorMap tm_vk, const __grid_constant__ CUtensorMap tm_dq,
@@ -718,8 +722,10 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     constexpr int SB = Cfg::q_stage(W);
 
     extern __shared__ uint8_t smem_raw[];
+    constexpr int NG = Cfg::kGroupsQ;                   // P / dS warpgroups (S, dP buffers)
+    static_assert(NG == 1 || (!Cfg::kQInTmem && NG * W <= 128), "S / dP buffers exceed their TMEM columns");
     __shared__ uint64_t bar_qdo_full, bar_full[ST], bar_empty[ST];
-    __shared__ uint64_t bar_s_full, bar_dp_full, bar_s_read, bar_ds_ready, bar_dq_done, bar_drain;
+    __shared__ uint64_t bar_s_full[NG], bar_dp_full[NG], bar_s_read[NG], bar_ds_ready[NG], bar_dq_done, bar_drain;
     __shared__ uint64_t bar_qt_ready;                   // Q and dO written to tensor memory (QT)
     __shared__ uint32_t tmem_slot;
     __shared__ volatile uint32_t abort_flag;
@@ -774,10 +780,12 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             ptx::mbar_init(&bar_full[s], 1);
             ptx::mbar_init(&bar_empty[s], 1);
         }
-        ptx::mbar_init(&bar_s_full, 1);
-        ptx::mbar_init(&bar_dp_full, 1);
-        ptx::mbar_init(&bar_s_read, 4);
-        ptx::mbar_init(&bar_ds_ready, 4);
+        for (int b = 0; b < NG; ++b) {
+            ptx::mbar_init(&bar_s_full[b], 1);
+            ptx::mbar_init(&bar_dp_full[b], 1);
+            ptx::mbar_init(&bar_s_read[b], 4);
+            ptx::mbar_init(&bar_ds_ready[b], 4);
+        }
         ptx::mbar_init(&bar_dq_done, 1);
         ptx::mbar_init(&bar_drain, 1);
         ptx::mbar_init(&bar_qt_ready, 4);
@@ -843,47 +851,54 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (!ptx::mbar_wait(&bar_full[s], (j / ST) & 1, &abort_flag, tmo)) return false;
                 ptx::tc_fence_after();
                 const uint32_t ka = ptx::smem_addr(st_kk(s));
+                const int b = j % NG;
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (QT)
                         ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColQT + kk * G::kKStep, desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
-                        ptx::mma_tf32_ss(tmem + Cfg::kColS, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ss(tmem + Cfg::kColS + b * W, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(&bar_s_full);
+                ptx::mma_commit(&bar_s_full[b]);
                 return true;
             };
             // dP = dO_i V_j^T   (Eq. 16); the stage is already full.
             auto issue_dp = [&](int j) {
                 const uint32_t va = ptx::smem_addr(st_vk(j % ST));
+                const int b = j % NG;
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (QT)
                         ptx::mma_tf32_ts(tmem + Cfg::kColDPq, tmem + Cfg::kColDOT + kk * G::kKStep, desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
-                        ptx::mma_tf32_ss(tmem + Cfg::kColDP, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ss(tmem + Cfg::kColDP + b * W, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                ptx::mma_commit(&bar_dp_full);
+                ptx::mma_commit(&bar_dp_full[b]);
             };
             bool ok = QT ? ptx::mbar_wait(&bar_qt_ready, 0, &abort_flag, tmo)
                          : ptx::mbar_wait(&bar_qdo_full, 0, &abort_flag, tmo);
-            if (ok) ok = issue_s(0);
-            if (ok) issue_dp(0);
+            for (int i = 0; ok && i < NG && i < n_kv; ++i) {
+                ok = issue_s(i);
+                if (ok) issue_dp(i);
+            }
+            // Sub-tile j + NG reuses the buffers of sub-tile j: its S once the
+            // warpgroup has read S(j), its dP after dQ(j).
             for (int j = 0; ok && j < n_kv; ++j) {
-                // Next scores as soon as the warpgroup has read S(j).
-                if (j + 1 < n_kv) {
-                    if (!ptx::mbar_wait(&bar_s_read, j & 1, &abort_flag, tmo)) { ok = false; break; }
-                    if (!issue_s(j + 1)) { ok = false; break; }
+                const int b = j % NG;
+                const uint32_t ph = static_cast<uint32_t>(j / NG) & 1u;
+                if (j + NG < n_kv) {
+                    if (!ptx::mbar_wait(&bar_s_read[b], ph, &abort_flag, tmo)) { ok = false; break; }
+                    if (!issue_s(j + NG)) { ok = false; break; }
                 }
                 // dQ_i += dS K_j   (Eq. 18 without the scale); dS from the dP columns.
-                if (!ptx::mbar_wait(&bar_ds_ready, j & 1, &abort_flag, tmo)) { ok = false; break; }
+                if (!ptx::mbar_wait(&bar_ds_ready[b], ph, &abort_flag, tmo)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t kmn = ptx::smem_addr(st_kmn(j % ST));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDQq, tmem + Cfg::kColDPq + kk * G::kKStep, desc_mnmajor<G>(kmn, kk, W), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDQq, tmem + Cfg::kColDPq + b * W + kk * G::kKStep, desc_mnmajor<G>(kmn, kk, W), idesc_dq, (j > 0 || kk > 0) ? 1u : 0u);
                 ptx::mma_commit(&bar_empty[j % ST]);
-                if (j + 1 < n_kv) issue_dp(j + 1);
+                if (j + NG < n_kv) issue_dp(j + NG);
             }
             if (ok) {
                 ptx::mma_commit(&bar_dq_done);
@@ -931,19 +946,22 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (lane == 0) ptx::mbar_arrive(&bar_qt_ready);
             }
         }
-        for (int j = 0; j < n_kv; ++j) {
+        const int grp = (warp - 2) >> 2;                 // takes sub-tiles j = grp (mod NG)
+        const uint32_t col_s = Cfg::kColS + grp * W, col_dp = Cfg::kColDPq + grp * W;
+        for (int j = grp; j < n_kv; j += NG) {
+            const uint32_t ph = static_cast<uint32_t>(j / NG) & 1u;
             const int k0 = kvs_of(j) * W;
             const bool mask = p.causal && k0 + W - 1 > q_row0;   // some key follows some query
             const int kv_valid = p.Nk - k0;                         // key columns < Nk
             // ---- P = exp2(S * scale*log2(e) - L*log2(e))   (Eq. 14), kept in registers
-            if (!ptx::mbar_wait(&bar_s_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar_s_full[grp], ph, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
             uint32_t pu[W];
-            tmem_ld_cols<W>(lane_base + Cfg::kColS, pu);
+            tmem_ld_cols<W>(lane_base + col_s, pu);
             ptx::tmem_wait_ld();
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_s_read);
+            if (lane == 0) ptx::mbar_arrive(&bar_s_read[grp]);
 #pragma unroll
             for (int c = 0; c < W; ++c) {
                 float pe = ptx::ex2_approx(fmaf(__uint_as_float(pu[c]), sl2, -l2r));
@@ -951,15 +969,16 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 pu[c] = __float_as_uint(pe);
             }
             // ---- dS = P o (dP - D)   (Eq. 17) -> TMEM over dP
-            if (!ptx::mbar_wait(&bar_dp_full, j & 1, &abort_flag, tmo)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar_dp_full[grp], ph, &abort_flag, tmo)) { ok = false; break; }
             ptx::tc_fence_after();
-            bwd32_ds_inplace<W>(lane_base + Cfg::kColDPq, pu, [&](int) { return dr; });
+            bwd32_ds_inplace<W>(lane_base + col_dp, pu, [&](int) { return dr; });
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready);
+            if (lane == 0) ptx::mbar_arrive(&bar_ds_ready[grp]);
         }
-        // ---------------- epilogue: dQ * scale -> sQ -> TMA store (zeros when no
-        // key tile was visited; nothing was loaded into sQ then).
+        // ---------------- epilogue (group 0): dQ * scale -> sQ -> TMA store (zeros
+        // when no key tile was visited; nothing was loaded into sQ then).
+        if (grp == 0) {
         if (ok && n_kv > 0) ok = ptx::mbar_wait(&bar_dq_done, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
@@ -972,6 +991,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ptx::tma_store_3d(&tm_dq, sDQ + bx * kTileRows * G::kRowBK, bx * G::kBoxK, q_row0, bh);
             ptx::tma_store_commit();
             ptx::tma_store_wait_all();
+        }
         }
     }
 
