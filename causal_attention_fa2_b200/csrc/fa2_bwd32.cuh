@@ -42,10 +42,10 @@ template <int D>
 struct Bwd32Cfg {
     using G = TileGeom<4, D>;
     static constexpr int kThreads = 192;
-    // dK/dV pass at d <= 32, where its elementwise work outweighs the MMAs: two
+    // dK/dV pass at d <= 64, where its elementwise work outweighs the MMAs: two
     // P / dS warpgroups take alternate query sub-tiles (S^T and dP^T double
     // buffered in TMEM), so one group's exponentials overlap the other's MMAs.
-    static constexpr int kGroupsKV = D <= 32 ? 2 : 1;
+    static constexpr int kGroupsKV = D <= 64 ? 2 : 1;
     static constexpr int kThreadsKV = 64 + 128 * kGroupsKV;
     // dQ pass likewise at d <= 32: two warpgroups on alternate key sub-tiles of
     // 64 rows (one group took 128-row sub-tiles).
@@ -61,7 +61,9 @@ struct Bwd32Cfg {
     // streamed query rows come in sub-tiles of 32 rows instead of 16.  The pass
     // is bound by the tcgen05 pipe, and the narrow S^T / dP^T MMAs (N = W) are
     // most of its instructions: W = 32 halves them per query row.
-    static constexpr bool kKInTmem = (D == 128);
+    // (At d = 64 K in TMEM leaves room for a third stage, which the two groups
+    // need: sub-tile i + 2 is loaded while i and i + 1 are being worked on.)
+    static constexpr bool kKInTmem = (D == 64 || D == 128);
     static constexpr int kResidentKV = (kKInTmem ? 1 : 2) * tile_k(kTileRows);
     // dQ pass at d = 64 and 128, likewise: Q and dO in tensor memory (the A
     // operands of S = Q K^T and dP = dO V^T), nothing resident in shared memory,
@@ -95,7 +97,7 @@ struct Bwd32Cfg {
     // second slot for Q K-major, the part each sub-tile needs first.  Two whole
     // stages of 64 rows do not fit beside V; 32-row sub-tiles left the tcgen05
     // instruction pipe the busiest unit of the pass.
-    static constexpr bool kPartStaged = kKInTmem;
+    static constexpr bool kPartStaged = D == 128;
     static constexpr int kWkv = kPartStaged ? 64 : (pick_kv() > 64 ? 64 : pick_kv());
     static constexpr int kStKV = kPartStaged ? 1 : stages_for(kv_stage(kWkv), kResidentKV);
     static constexpr int kWq = kGroupsQ == 2 ? 64 : pick_q();
@@ -108,9 +110,13 @@ struct Bwd32Cfg {
     static constexpr uint32_t kTmemCols = 512;
     // dK/dV pass: S^T | dP^T | dV | dK.   dQ pass: S | dP | dQ.
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
-    // dK/dV pass with K in tensor memory: S^T | dP^T | K | dV | dK.
-    static constexpr uint32_t kColDPkv = kKInTmem ? 64 : kColDP, kColKT = 128;
-    static_assert(!kKInTmem || kWkv <= 64, "S^T and dP^T must fit below the K columns");
+    // dK/dV pass, general: S^T (per group) | dP^T (per group) | [K] | dV | dK.
+    static constexpr uint32_t kColDPkv = (kKInTmem || kGroupsKV == 2) ? kGroupsKV * kWkv : kColDP;
+    static constexpr uint32_t kColKT = 2 * kGroupsKV * kWkv;
+    static constexpr uint32_t kColDVkv = kKInTmem ? kColKT + G::kStepsD * G::kKStep : kColDV;
+    static constexpr uint32_t kColDKkv = kKInTmem ? kColDVkv + G::kNOut : kColDK;
+    static_assert(kColDPkv + kGroupsKV * kWkv <= (kKInTmem ? kColKT : kColDV) && kColDKkv + G::kNOut <= kTmemCols,
+                  "dK/dV pass columns overlap or exceed TMEM");
     // dQ pass with Q and dO in tensor memory: S | dP | dQ | Q | dO.
     static constexpr uint32_t kColDPq = kQInTmem ? kWq : kColDP, kColDQq = kQInTmem ? 2 * kWq : kColDQ;
     static constexpr uint32_t kColQT = 2 * kWq + G::kNOut, kColDOT = kColQT + G::kStepsD * G::kKStep;
@@ -301,7 +307,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kv_full, bar_full[ST], bar_empty[ST];
     constexpr int NG = Cfg::kGroupsKV;                  // P / dS warpgroups (buffers)
-    static_assert(NG == 1 || (!Cfg::kKInTmem && NG * W <= 128), "S^T / dP^T buffers exceed their TMEM columns");
+    static_assert(NG == 1 || (!Cfg::kPartStaged && NG * W <= 128), "S^T / dP^T buffers exceed their TMEM columns");
     __shared__ uint64_t bar_s_full[NG], bar_dp_full[NG], bar_p_ready[NG], bar_ds_ready[NG], bar_dkv_full, bar_drain;
     __shared__ uint64_t bar_kt_ready;                   // K written to tensor memory (KT)
     // Part-staged (PP): full / empty barrier per part slot: Q K-major slots 0 and
@@ -531,7 +537,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (KT)
-                        ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColKT + kk * G::kKStep, desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ts(tmem + Cfg::kColS + b * W, tmem + Cfg::kColKT + kk * G::kKStep, desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
                         ptx::mma_tf32_ss(tmem + Cfg::kColS + b * W, desc_kmajor<G>(k_addr, kk), desc_kmajor<G>(qa, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
@@ -571,7 +577,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 const uint32_t dmn = ptx::smem_addr(PP ? pp_addr(kPartDomn, it) : st_domn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDV, tmem + Cfg::kColS + b * W + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDVkv, tmem + Cfg::kColS + b * W + kk * G::kKStep, desc_mnmajor<G>(dmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 release_part(kPartDomn, it);
                 if (it + NG < n_it && !issue_s(it + NG)) { ok = false; break; }
                 // dK_j += dS^T Q_i   (Eq. 19 without the scale); dS^T from the dP^T columns.
@@ -581,7 +587,7 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
                 const uint32_t qmn = ptx::smem_addr(PP ? pp_addr(kPartQmn, it) : st_qmn(s));
 #pragma unroll
                 for (int kk = 0; kk < W / G::kKStep; ++kk)
-                    ptx::mma_tf32_ts(tmem + Cfg::kColDK, tmem + Cfg::kColDPkv + b * W + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_tf32_ts(tmem + Cfg::kColDKkv, tmem + Cfg::kColDPkv + b * W + kk * G::kKStep, desc_mnmajor<G>(qmn, kk, W), idesc_kv, (it > 0 || kk > 0) ? 1u : 0u);
                 if constexpr (PP) release_part(kPartQmn, it);
                 else ptx::mma_commit(&bar_empty[s]);
                 if (it + NG < n_it && !issue_dp(it + NG)) { ok = false; break; }
@@ -603,8 +609,8 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         const float sl2 = p.scale_log2;
         bool ok = true;
         if constexpr (KT) {
-            // K row r (TF32-rounded copy) into tensor memory; zeros past Nk.
-            if (n_it > 0) {
+            // K row r (TF32-rounded copy) into tensor memory; zeros past Nk (group 0).
+            if (n_it > 0 && grp == 0) {
                 const float4* krow = reinterpret_cast<const float4*>(
                     p.k32 + (static_cast<size_t>(bh) * p.Nk + (key_valid ? kv_row0 + r : 0)) * D);
 #pragma unroll
@@ -670,8 +676,8 @@ fa2_bwd32_dkdv_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_co
         if (ok && n_it > 0) ok = ptx::mbar_wait(&bar_dkv_full, 0, &abort_flag, tmo);
         if (ok) {
             ptx::tc_fence_after();
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDV, r, 1.f, sV, n_it == 0);
-            bwd32_stage_rows<G>(lane_base + Cfg::kColDK, r, p.scale, sDK, n_it == 0);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDVkv, r, 1.f, sV, n_it == 0);
+            bwd32_stage_rows<G>(lane_base + Cfg::kColDKkv, r, p.scale, sDK, n_it == 0);
             ptx::fence_async_smem();
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
