@@ -48,7 +48,8 @@ struct Bwd32Cfg {
     static constexpr int kGroupsKV = D <= 64 ? 2 : 1;
     static constexpr int kThreadsKV = 64 + 128 * kGroupsKV;
     // dQ pass likewise at d <= 32: two warpgroups on alternate key sub-tiles of
-    // 64 rows (one group took 128-row sub-tiles).
+    // 64 rows (one group took 128-row sub-tiles; at d = 64, with Q and dO in
+    // TMEM, two groups measured 1-3 % slower).
     static constexpr int kGroupsQ = D <= 32 ? 2 : 1;
     static constexpr int kThreadsQ = 64 + 128 * kGroupsQ;
     // 227 KB minus the 1024-byte alignment pad and the static shared memory.
@@ -118,8 +119,11 @@ struct Bwd32Cfg {
     static_assert(kColDPkv + kGroupsKV * kWkv <= (kKInTmem ? kColKT : kColDV) && kColDKkv + G::kNOut <= kTmemCols,
                   "dK/dV pass columns overlap or exceed TMEM");
     // dQ pass with Q and dO in tensor memory: S | dP | dQ | Q | dO.
-    static constexpr uint32_t kColDPq = kQInTmem ? kWq : kColDP, kColDQq = kQInTmem ? 2 * kWq : kColDQ;
-    static constexpr uint32_t kColQT = 2 * kWq + G::kNOut, kColDOT = kColQT + G::kStepsD * G::kKStep;
+    // dQ pass, general: S (per group) | dP (per group) | dQ | [Q | dO].
+    static constexpr uint32_t kColDPq = kQInTmem ? kGroupsQ * kWq : kColDP;
+    static constexpr uint32_t kColDQq = kQInTmem ? 2 * kGroupsQ * kWq : kColDQ;
+    static constexpr uint32_t kColQT = kColDQq + G::kNOut, kColDOT = kColQT + G::kStepsD * G::kKStep;
+    static_assert(kGroupsQ * kWq <= kColDPq && kColDPq + kGroupsQ * kWq <= kColDQq, "dQ pass S / dP columns overlap");
     static_assert(!kQInTmem || kColDOT + G::kStepsD * G::kKStep <= kTmemCols, "dQ pass columns exceed TMEM");
 };
 
@@ -729,7 +733,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     extern __shared__ uint8_t smem_raw[];
     constexpr int NG = Cfg::kGroupsQ;                   // P / dS warpgroups (S, dP buffers)
-    static_assert(NG == 1 || (!Cfg::kQInTmem && NG * W <= 128), "S / dP buffers exceed their TMEM columns");
+    static_assert(NG == 1 || NG * W <= 128, "S / dP buffers exceed their TMEM columns");
     __shared__ uint64_t bar_qdo_full, bar_full[ST], bar_empty[ST];
     __shared__ uint64_t bar_s_full[NG], bar_dp_full[NG], bar_s_read[NG], bar_ds_ready[NG], bar_dq_done, bar_drain;
     __shared__ uint64_t bar_qt_ready;                   // Q and dO written to tensor memory (QT)
@@ -861,7 +865,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (QT)
-                        ptx::mma_tf32_ts(tmem + Cfg::kColS, tmem + Cfg::kColQT + kk * G::kKStep, desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ts(tmem + Cfg::kColS + b * W, tmem + Cfg::kColQT + kk * G::kKStep, desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
                         ptx::mma_tf32_ss(tmem + Cfg::kColS + b * W, desc_kmajor<G>(q_addr, kk), desc_kmajor<G>(ka, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
@@ -875,7 +879,7 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int kk = 0; kk < G::kStepsD; ++kk) {
                     if constexpr (QT)
-                        ptx::mma_tf32_ts(tmem + Cfg::kColDPq, tmem + Cfg::kColDOT + kk * G::kKStep, desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
+                        ptx::mma_tf32_ts(tmem + Cfg::kColDPq + b * W, tmem + Cfg::kColDOT + kk * G::kKStep, desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                     else
                         ptx::mma_tf32_ss(tmem + Cfg::kColDP + b * W, desc_kmajor<G>(do_addr, kk), desc_kmajor<G>(va, kk, W), idesc_s, kk > 0 ? 1u : 0u);
                 }
@@ -914,7 +918,8 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
     } else {
-        // ------------------------------------------------ P / dS warpgroup
+        // ------------------------------------------------ P / dS warpgroup(s)
+        const int grp = (warp - 2) >> 2;                 // takes sub-tiles j = grp (mod NG)
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;               // query row inside the tile
         const uint32_t lane_base = tmem + ptx::tmem_lane_offset(quarter * 32);
@@ -924,8 +929,9 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float dr = p.dvec[vrow];                   // D_i (0 past N)
         bool ok = true;
         if constexpr (QT) {
-            // Q and dO row r (TF32-rounded copies) into tensor memory; zeros past N.
-            if (n_kv > 0) {
+            // Q and dO row r (TF32-rounded copies) into tensor memory; zeros past N
+            // (group 0).
+            if (n_kv > 0 && grp == 0) {
                 const bool row_valid = q_row0 + r < p.N;
                 const size_t row_off = (static_cast<size_t>(bh) * p.N + (row_valid ? q_row0 + r : 0)) * D;
 #pragma unroll
@@ -952,7 +958,6 @@ fa2_bwd32_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (lane == 0) ptx::mbar_arrive(&bar_qt_ready);
             }
         }
-        const int grp = (warp - 2) >> 2;                 // takes sub-tiles j = grp (mod NG)
         const uint32_t col_s = Cfg::kColS + grp * W, col_dp = Cfg::kColDPq + grp * W;
         for (int j = grp; j < n_kv; j += NG) {
             const uint32_t ph = static_cast<uint32_t>(j / NG) & 1u;
