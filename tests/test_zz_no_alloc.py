@@ -36,6 +36,7 @@ def _call_noalloc(lib, q, k, v, o, lse, do, dq, dk, dv, causal, scale, dtype):
 # (most of its use); fp16 runs the 16-bit kernels with fp16 operands.
 CASES = [(2, 4, 1000, 64, True, "bf16"), (1, 8, 2048, 128, False, "bf16"),
          (1, 4, 700, 128, True, "fp32"), (2, 2, 333, 80, False, "fp32"),
+         (1, 3, 500, 64, True, "fp32"), (1, 2, 300, 32, False, "fp32"),
          (1, 4, 1000, 64, True, "fp16")]
 
 
