@@ -200,6 +200,25 @@ def test_forward_and_backward_deterministic(dtype):
     torch.testing.assert_close(h1[0].float(), g1[0].float(), atol=1e-3, rtol=1e-2)
 
 
+@pytest.mark.parametrize("B,H,N,d,dtype", [(1, 8, 2048, 128, "bf16"), (2, 4, 1024, 64, "bf16"),
+                                              (1, 4, 1024, 16, "fp32"), (1, 4, 1024, 32, "fp32"),
+                                              (1, 4, 1024, 64, "fp32"), (1, 4, 1024, 128, "fp32")])
+def test_two_pass_backward_repeats_bitwise(B, H, N, d, dtype):
+    """Twelve back-to-back runs of the two-pass backward give the same bits:
+    a check for races between the kernels' warp roles (ping-pong groups, double
+    buffers, parted stages), which would show as run-to-run differences."""
+    import causal_attention_fa2_b200 as fa2
+    dev = torch.device("cuda", 0)
+    inp = fa2_inputs.make_inputs(B, H, N, d, dtype, seed=77 + d)
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa2.forward(q, k, v)
+    ref = fa2.backward(q, k, v, o, lse, do, mode="two-pass")
+    runs = [fa2.backward(q, k, v, o, lse, do, mode="two-pass") for _ in range(11)]
+    torch.cuda.synchronize()
+    for g in runs:
+        assert all(torch.equal(a, b) for a, b in zip(ref, g))
+
+
 def test_autograd_function_matches_direct_calls():
     import causal_attention_fa2_b200 as fa2
     dev = torch.device("cuda", 0)
