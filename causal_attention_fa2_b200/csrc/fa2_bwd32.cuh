@@ -57,13 +57,13 @@ struct Bwd32Cfg {
     __host__ __device__ static constexpr int tile_k(int rows) { return G::kNBoxK * rows * G::kRowBK; }
     __host__ __device__ static constexpr int tile_mn(int rows) { return G::kNBoxMN * rows * G::kRowBMN; }
     static constexpr int kResident = 2 * tile_k(kTileRows);
-    // dK/dV pass at d = 128: K sits in tensor memory (the S^T = K Q^T MMA reads
-    // its A operand there), so only V is resident in shared memory and the
-    // streamed query rows come in sub-tiles of 32 rows instead of 16.  The pass
-    // is bound by the tcgen05 pipe, and the narrow S^T / dP^T MMAs (N = W) are
-    // most of its instructions: W = 32 halves them per query row.
-    // (At d = 64 K in TMEM leaves room for a third stage, which the two groups
-    // need: sub-tile i + 2 is loaded while i and i + 1 are being worked on.)
+    // dK/dV pass at d = 64 and 128: K sits in tensor memory (the S^T = K Q^T MMA
+    // reads its A operand there), so only V is resident in shared memory.  At
+    // d = 128 that leaves room for 64-row query sub-tiles (part-staged, below)
+    // instead of 16: the pass was bound by the tcgen05 instruction pipe, the
+    // narrow S^T / dP^T MMAs (N = W) being most of its instructions.  At d = 64
+    // it leaves room for a third stage, which the two groups need (sub-tile
+    // i + 2 loads while i and i + 1 are being worked on).
     static constexpr bool kKInTmem = (D == 64 || D == 128);
     static constexpr int kResidentKV = (kKInTmem ? 1 : 2) * tile_k(kTileRows);
     // dQ pass at d = 64 and 128, likewise: Q and dO in tensor memory (the A
@@ -118,7 +118,6 @@ struct Bwd32Cfg {
     static constexpr uint32_t kColDKkv = kKInTmem ? kColDVkv + G::kNOut : kColDK;
     static_assert(kColDPkv + kGroupsKV * kWkv <= (kKInTmem ? kColKT : kColDV) && kColDKkv + G::kNOut <= kTmemCols,
                   "dK/dV pass columns overlap or exceed TMEM");
-    // dQ pass with Q and dO in tensor memory: S | dP | dQ | Q | dO.
     // dQ pass, general: S (per group) | dP (per group) | dQ | [Q | dO].
     static constexpr uint32_t kColDPq = kQInTmem ? kGroupsQ * kWq : kColDP;
     static constexpr uint32_t kColDQq = kQInTmem ? 2 * kGroupsQ * kWq : kColDQ;
