@@ -114,12 +114,17 @@ inline BwdWorkspace bwd_workspace_layout(int BH, int N, int BH_kv, int Nk, int d
 // ------------------------------------------------------------------ pre-processing
 
 // Geometry of the pre-pass: a row of d 16-bit values is read as 16-byte
-// vectors by kTPR threads (d / 8 rounded up to a power of two), so one warp
-// covers 32 / kTPR rows and one 256-thread block 8 * 32 / kTPR rows.
+// vectors, kPer of them per thread, by kTPR threads (rounded up to a power of
+// two), so one warp covers 32 / kTPR rows and one 256-thread block 8 * 32 / kTPR
+// rows.
 template <int D>
 struct BwdPreCfg {
     static constexpr int kVec = 8;                                  // elements per 16-byte load
-    static constexpr int kUsed = (D + kVec - 1) / kVec;            // threads that load
+    static constexpr int kChunks = (D + kVec - 1) / kVec;          // 16-byte chunks per row
+    // Two chunks of O and of dO per thread from d = 64 up, so four 16-byte loads
+    // are in flight per thread.
+    static constexpr int kPer = kChunks >= 8 ? 2 : 1;
+    static constexpr int kUsed = (kChunks + kPer - 1) / kPer;      // threads that load
     static constexpr int kTPR = kUsed <= 2 ? 2 : kUsed <= 4 ? 4 : kUsed <= 8 ? 8 : 16;
     static constexpr int kRowsPerBlock = 8 * 32 / kTPR;
 };
@@ -147,23 +152,33 @@ fa2_bwd_pre_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ 
     const int n = static_cast<int>(row - bh * n_pad);
     float acc = 0.f;
     if (dq_acc && live && sub < C::kUsed) {
-        float4* z = reinterpret_cast<float4*>(dq_acc + row * D + sub * C::kVec);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int e = 0; e < C::kPer; ++e) {
+            float4* z = reinterpret_cast<float4*>(dq_acc + row * D + (sub * C::kPer + e) * C::kVec);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
     if (live && n < N && sub < C::kUsed) {
-        const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * C::kVec;
-        const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + base));
-        const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + base));
-        const uint32_t aw[4] = {a.x, a.y, a.z, a.w};
-        const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+        const size_t base = (static_cast<size_t>(bh) * N + n) * D + sub * C::kPer * C::kVec;
+        uint4 a[C::kPer], b[C::kPer];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            float a0, a1, b0, b1;
-            TileGeom<2, D, F16>::unpack2(aw[w], a0, a1);
-            TileGeom<2, D, F16>::unpack2(bw[w], b0, b1);
-            acc = fmaf(a0, b0, acc);
-            acc = fmaf(a1, b1, acc);
+        for (int e = 0; e < C::kPer; ++e) {
+            a[e] = __ldg(reinterpret_cast<const uint4*>(o + base) + e);
+            b[e] = __ldg(reinterpret_cast<const uint4*>(dout + base) + e);
+        }
+#pragma unroll
+        for (int e = 0; e < C::kPer; ++e) {
+            const uint32_t aw[4] = {a[e].x, a[e].y, a[e].z, a[e].w};
+            const uint32_t bw[4] = {b[e].x, b[e].y, b[e].z, b[e].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                float a0, a1, b0, b1;
+                TileGeom<2, D, F16>::unpack2(aw[w], a0, a1);
+                TileGeom<2, D, F16>::unpack2(bw[w], b0, b1);
+                acc = fmaf(a0, b0, acc);
+                acc = fmaf(a1, b1, acc);
+            }
         }
     }
 #pragma unroll
