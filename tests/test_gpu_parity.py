@@ -99,17 +99,42 @@ def test_fp16_10b_shape_heads(oracle_mod):
             print(f"ERR fp16-10b head {hh} {name} max_abs {e:.3e}")
 
 
-@pytest.mark.parametrize("scale", [0.09, 0.14])
+@pytest.mark.parametrize("scale", [0.09, 0.14, 0.2])
 def test_nondefault_scale(oracle_mod, scale):
-    """A scale other than 1/sqrt(d) must enter S, dQ and dK.  (Much sharper
-    scales (0.2 and above at d=64) push the rounding of the kernel's O inside
-    D = rowsum(O o dO) past the 1e-2 tolerance on a few dQ/dK elements: a
-    property of the method's D formula on rounded outputs, not of the
-    kernels.)"""
+    """A scale other than 1/sqrt(d) must enter S, dQ and dK.  At d = 64 the
+    default is 0.125; 0.2 is 1.6 times sharper, and over six seeds at N = 256
+    and 640 its worst dQ / dK element used 0.84 of the bound."""
     inp = fa2_inputs.make_inputs(1, 2, 256, 64, "bf16", seed=5)
     got = gpu_fwd_bwd(inp, True, scale)
     ref = _oracle(oracle_mod, inp, True, scale)
     for name in ("o", "lse", "dq", "dk", "dv"):
+        assert_close(to64(got[name]), ref[name], "bf16", name)
+
+
+@pytest.mark.xfail(strict=True, raises=AssertionError,
+                   reason="16-bit backward roundings (D from the 16-bit O, 16-bit dS) "
+                          "pass the bound at 3.2x the default scale")
+def test_sharp_scale_known_exceedance(oracle_mod):
+    """The known limit of the 16-bit backward, pinned: at scale 0.4 (3.2 times
+    the default 1/sqrt(64)) the softmax is sharp enough that the backward's
+    roundings (D = rowsum(O o dO) taken from the 16-bit O, dS rounded to 16 bits
+    before the dQ MMA) move a few dQ elements past the 1e-2 bound (this seed:
+    3.9 times the bound at row 155 of head 1; O and L stay inside it, checked by
+    the test below).  A change that removes the exceedance turns this into an unexpected
+    pass, which fails the run until the pin is updated."""
+    inp = fa2_inputs.make_inputs(1, 2, 256, 64, "bf16", seed=3)
+    got = gpu_fwd_bwd(inp, True, 0.4, mode="two-pass")
+    ref = _oracle(oracle_mod, inp, True, 0.4)
+    assert_close(to64(got["dq"]), ref["dq"], "bf16", "dq")
+
+
+def test_sharp_scale_forward(oracle_mod):
+    """The forward at the same sharp scale (0.4, d = 64) stays inside the bound:
+    the exceedance above belongs to the backward."""
+    inp = fa2_inputs.make_inputs(1, 2, 256, 64, "bf16", seed=3)
+    got = gpu_fwd_bwd(inp, True, 0.4, do_backward=False)
+    ref = _oracle(oracle_mod, inp, True, 0.4, backward=False)
+    for name in ("o", "lse"):
         assert_close(to64(got[name]), ref[name], "bf16", name)
 
 
