@@ -45,9 +45,9 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of each
 # bf16 d=128 kernel on the 10B head shape, from one ncu capture of the current
 # kernel build; None where no capture of the current build exists.
-FWD_TRAFFIC_BYTES = 209_842_944   # 186.0 MB read + 23.8 MB written
-DKDV_TRAFFIC_BYTES = 204_046_336  # 153.5 MB read + 50.5 MB written (two-pass dK/dV pass)
-DQ_TRAFFIC_BYTES = 178_741_248    # 154.2 MB read + 24.5 MB written (two-pass dQ pass)
+FWD_TRAFFIC_BYTES = 207_431_168   # 185.2 MB read + 22.2 MB written
+DKDV_TRAFFIC_BYTES = 201_089_792  # 153.4 MB read + 47.7 MB written (two-pass dK/dV pass)
+DQ_TRAFFIC_BYTES = 177_845_760    # 154.3 MB read + 23.5 MB written (two-pass dQ pass)
 FUSED_TRAFFIC_BYTES = None        # no capture of the one-pass backward's current build
 TRAFFIC_WORKLOAD = "10b-b1h36-n4096-d128"
 
